@@ -1,0 +1,496 @@
+#!/usr/bin/env python
+"""Benchmark: one LSA attention layer in prefill (index build + key selection +
+exact sparse attention) on the 1,048,576-token workload, on N GPUs.
+
+Each GPU processes its own independent layer instance (same recipe, seed
+offset by rank): weak scaling with no data-path collective.  Timing: W
+untimed warm-up steps, then K steps between CUDA events on the launching
+stream, bracketed by barrier + synchronize, max over ranks.  Inputs stay
+resident in HBM and are larger than L2 (Q alone is 4 GiB).
+
+Prints ONE JSON line on rank 0.  `--impl reference` times the CPU oracle
+instead (bounded sample, scaled to the whole layer).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "LSA prefill tokens/s per layer (index+select+attn) at 1M ctx; % of roofline"
+UNIT = "tokens/s"
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=5)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--workload", default="prefill_1m")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--cpu-sample-queries", type=int, default=96)
+    return ap.parse_args()
+
+
+# ------------------------------------------------------------------ plumbing
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int, device) -> float:
+    """Max of a host float over ranks (timing only; not a data-path exchange)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, power, reasons = [], [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+                power.append(float(parts[3]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        loaded = [s for s, p in zip(sm, power) if p > 200] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "power_w_max": max(power) if power else None,
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"], "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+
+
+def kernel_source_sha(fname: str) -> str:
+    path = os.path.join(ROOT, "hierarchical_latent_key_gemm_b200", "csrc", fname)
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str, workload: str, src: str):
+    """DRAM bytes per launch recorded from an ncu capture (profiles/traffic.json),
+    or None when absent or when the kernel source changed since."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    e = d.get(kernel, {}).get(workload)
+    if not e or e.get("source_sha") != kernel_source_sha(src):
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import torch
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    from hierarchical_latent_key_gemm_b200 import lsa
+    from hierarchical_latent_key_gemm_b200.workloads import WORKLOADS, describe, input_bytes, make_inputs
+
+    w = WORKLOADS[args.workload]
+    if w.decode_steps:
+        raise SystemExit("bench.py times prefill workloads; decode is measured by its own tests")
+    lsa.lib()
+    seed = args.seed + 1000 * rank
+    inp = make_inputs(w, seed=seed, device=dev)
+    Q, K, V, W = inp["Q"], inp["K"], inp["V"], inp["W"]
+    N = w.n_tokens
+    dt = lsa.LSA_BF16 if w.dtype == "bf16" else lsa.LSA_F32
+    bp = lsa.make_build_params(w.batch, N, N, w.hkv, w.d, w.r, w.pool, dt, w.level_sizes, w.lloyd_iters,
+                               w.grid_log2, w.sink, 0)
+    sp = lsa.make_select_params(w.hq, w.beam, w.topk, w.sink, w.window)
+    max_sel = w.max_sel
+    idx = torch.empty((w.batch, N, w.hkv, max_sel), dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.batch, N, w.hkv), dtype=torch.int32, device=dev)
+    O = torch.empty_like(Q)
+    lse = torch.empty((w.batch, N, w.hq), dtype=torch.float32, device=dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record()
+        ix = lsa.lsa_build_index(bp, K, W)
+        if ev:
+            ev[1].record()
+        lsa.lsa_select(ix, sp, Q, idx=idx, cnt=cnt, max_sel=max_sel)
+        if ev:
+            ev[2].record()
+        lsa.lsa_sparse_attn(Q, K, V, idx, cnt, w.hkv, O=O, lse=lse)
+        if ev:
+            ev[3].record()
+        return ix
+
+    for _ in range(args.warmup):
+        step().free()
+    torch.cuda.synchronize()
+    st = lsa.lsa_check(None)
+    if st != lsa.LSA_OK:
+        raise SystemExit(f"device error after warm-up: {lsa.strerror(st)}")
+
+    clocks = ClockSampler(local)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    launches0 = lsa.lsa_launch_count()
+    t0.record()
+    for k in range(args.steps):
+        step(evs[k]).free()
+    t1.record()
+    torch.cuda.synchronize()
+    launches = lsa.lsa_launch_count() - launches0
+    clk = clocks.stop()
+    barrier(world)
+    ms_local = t0.elapsed_time(t1)
+    ms = max_over_ranks(ms_local, world, dev)
+    ms_step = ms / args.steps
+    value = world * N * w.batch / (ms_step / 1e3)
+
+    build_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    select_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    attn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+
+    peaks = measured_peaks()
+    sel_rows = int(cnt.sum(dtype=torch.int64).item())
+    attn_bytes = sel_rows * w.d * 2 * 2                       # gathered K and V rows (bf16)
+    stages = {"build_ms": build_ms, "select_ms": select_ms, "attn_ms": attn_ms}
+    # the single most expensive kernel is the sparse-attention launch (one per step)
+    achieved = attn_bytes / (attn_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": "attn_bf16_kernel<128>", "achieved": achieved, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+                "traffic": recorded_traffic("attn_bf16_kernel<128>", w.name, "attn.cu"),
+                "algorithmic_bytes_per_launch": attn_bytes,
+                "peak_source": peaks["source"],
+                "note": "achieved = sum over (query, KV head) of |Sel| * d * 2 B * 2 (K and V) / mean kernel time"}
+
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, w, inp, bp, sp, idx, cnt, O, lse, dev, world)
+
+    extra = None
+    if not args.no_extra and rank == 0:
+        extra = run_extra(w, inp, bp, sp, dev, select_ms, idx, cnt)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_oracle_estimate(w, inp, args.cpu_sample_queries)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": describe(w), "global_batch": w.batch * world, "seq_len": N,
+                       "parallelism": f"dp{world} (one independent layer instance per GPU)",
+                       "l2": "inputs larger than L2 (Q 4 GiB, K and V 0.5 GiB each); no flush needed",
+                       "seed": args.seed},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
+            "clocks": clk, "stages": stages, "extra": extra,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def run_e2e(args, w, inp, bp, sp, idx, cnt, O, lse, dev, world):
+    """Same metric through the public API with HOST buffers: each step copies
+    Q, K, V, W from pinned host memory and reads O back."""
+    import torch
+    from hierarchical_latent_key_gemm_b200 import lsa
+    hQ = inp["Q"].cpu().pin_memory()
+    hK = inp["K"].cpu().pin_memory()
+    hV = inp["V"].cpu().pin_memory()
+    hW = inp["W"].cpu().pin_memory()
+    hO = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
+    dQ, dK, dV, dW = (torch.empty_like(inp[k]) for k in ("Q", "K", "V", "W"))
+
+    def step():
+        dQ.copy_(hQ, non_blocking=True)
+        dK.copy_(hK, non_blocking=True)
+        dV.copy_(hV, non_blocking=True)
+        dW.copy_(hW, non_blocking=True)
+        ix = lsa.lsa_build_index(bp, dK, dW)
+        lsa.lsa_select(ix, sp, dQ, idx=idx, cnt=cnt, max_sel=idx.shape[-1])
+        lsa.lsa_sparse_attn(dQ, dK, dV, idx, cnt, w.hkv, O=O, lse=lse)
+        hO.copy_(O, non_blocking=True)
+        return ix
+
+    n = max(1, min(args.steps, 3))
+    step().free()
+    torch.cuda.synchronize()
+    barrier(world)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for _ in range(n):
+        step().free()
+    t1.record()
+    torch.cuda.synchronize()
+    ms = max_over_ranks(t0.elapsed_time(t1), world, dev) / n
+    h2d = sum(t.numel() * t.element_size() for t in (hQ, hK, hV, hW))
+    d2h = hO.numel() * hO.element_size()
+    return {"value": world * w.n_tokens * w.batch / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def run_extra(w, inp, bp, sp, dev, select_ms, idx, cnt):
+    """Not timed in the headline: full-scan indexer on a query sample (speedup
+    and recall of the tree against exact full-scan top-K), needle hit-rates,
+    index bytes."""
+    import torch
+    from hierarchical_latent_key_gemm_b200 import lsa
+    Q, K = inp["Q"], inp["K"]
+    N = w.n_tokens
+    ix = lsa.lsa_build_index(bp, K, inp["W"])
+    info = ix.info()
+    ns = 2048
+    pos = torch.linspace(0, N - 1, ns, device=dev).round().to(torch.int64)
+    pos = torch.unique(pos)
+    qs = Q[:, pos].contiguous()
+    qpos = pos[None, :].repeat(w.batch, 1).contiguous()
+    lsa.lsa_fullscan_select(ix, sp, qs, q_pos=qpos)  # warm-up
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    fidx, fcnt = lsa.lsa_fullscan_select(ix, sp, qs, q_pos=qpos)
+    e1.record()
+    torch.cuda.synchronize()
+    full_ms_sample = e0.elapsed_time(e1)
+    full_ms_est = full_ms_sample * N / pos.numel()
+    tidx = idx[:, pos]
+    tcnt = cnt[:, pos]
+    # recall of the tree's long-range picks against the exact full-scan top-K
+    hit = tot = 0
+    for b in range(w.batch):
+        for h in range(w.hkv):
+            for k in range(pos.numel()):
+                f = set(fidx[b, k, h, : fcnt[b, k, h]].tolist())
+                t = set(tidx[b, k, h, : tcnt[b, k, h]].tolist())
+                i = int(pos[k])
+                lo = max(0, i - w.window + 1)
+                base = set(range(min(w.sink, lo))) | set(range(lo, i + 1))
+                f -= base
+                t -= base
+                tot += len(f)
+                hit += len(f & t)
+    needles = inp["needles"]
+    nh_tree = nh_full = 0
+    for (b, h, p, qp) in needles:
+        row = idx[b, qp, h, : cnt[b, qp, h]]
+        nh_tree += int((row == p).any().item())
+    if needles:
+        npos = torch.tensor([qp for (_, _, _, qp) in needles], device=dev)
+        nq_ = Q[:, npos].contiguous()
+        nqpos = npos[None, :].repeat(w.batch, 1).contiguous()
+        nf, nfc = lsa.lsa_fullscan_select(ix, sp, nq_, q_pos=nqpos)
+        for k, (b, h, p, qp) in enumerate(needles):
+            nh_full += int((nf[b, k, h, : nfc[b, k, h]] == p).any().item())
+    ix.free()
+    return {"fullscan_ms_estimate": full_ms_est, "fullscan_sample_queries": int(pos.numel()),
+            "tree_select_ms": select_ms, "tree_vs_fullscan_speedup": full_ms_est / select_ms,
+            "tree_recall_vs_fullscan_topk": hit / max(1, tot),
+            "needle_hit_rate_tree": nh_tree / max(1, len(needles)),
+            "needle_hit_rate_fullscan": nh_full / max(1, len(needles)), "needles": len(needles),
+            "index_device_bytes": int(info.device_bytes),
+            "select_queries_per_s": N * w.batch * w.hkv / (select_ms / 1e3)}
+
+
+# ------------------------------------------------------------------ CPU oracle
+def cpu_cores() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [p.get("num_threads", 0) for p in threadpool_info() if p.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def cpu_oracle_estimate(w, inp, sample_queries: int) -> dict:
+    """Time the oracle, as it stands, on a bounded sample of the workload and
+    scale to one whole layer: latents of every block; one full-size Lloyd
+    round of one KV head (x rounds x heads); the upper tree levels in full;
+    select + attention on sampled queries (x all queries x heads)."""
+    import numpy as np
+    import oracle as O
+    K = inp["K"]
+    Q = inp["Q"]
+    V = inp["V"]
+    Wm = inp["W"].double().cpu().numpy()
+    N, G = w.n_tokens, w.group
+    t_start = time.perf_counter()
+    # latents (all heads)
+    t = time.perf_counter()
+    Kls = []
+    Kh = []
+    for h in range(w.hkv):
+        kh = K[0, :N, h].float().cpu().numpy().astype(np.float64)
+        Kh.append(kh)
+        Kls.append(O.project_pool(kh, Wm, w.pool))
+    t_lat = time.perf_counter() - t
+    # one Lloyd round of head 0 at full size
+    t = time.perf_counter()
+    C0 = O.kmeans_init(Kls[0], w.level_sizes[-1])
+    lab, _ = O.kmeans_assign(Kls[0], C0)
+    C1 = O.kmeans_update(Kls[0], lab, C0, w.grid_log2)
+    t_round = time.perf_counter() - t
+    # upper levels in full, on the leaf centroids of that round
+    t = time.perf_counter()
+    cents = [None] * len(w.level_sizes)
+    parents = [None] * len(w.level_sizes)
+    cents[-1] = C1
+    pts = C1
+    for l in range(len(w.level_sizes) - 2, -1, -1):
+        r = O.kmeans(pts, w.level_sizes[l], w.lloyd_iters, w.grid_log2)
+        parents[l + 1] = r.labels
+        cents[l] = r.centroids
+        pts = r.centroids
+    t_upper = time.perf_counter() - t
+    tree = O.Tree(w.pool, w.sink, list(w.level_sizes), cents, parents, lab, [[]] * len(w.level_sizes)).finish()
+    # select + attention on sampled queries
+    rng = np.random.default_rng(0)
+    rows = np.sort(rng.integers(w.sink + w.window + w.pool, N, sample_queries))
+    Vh = V[0, :N, 0].float().cpu().numpy().astype(np.float64)
+    t = time.perf_counter()
+    for i in rows:
+        q = Q[0, int(i), 0:G].float().cpu().numpy().astype(np.float64)
+        qb = O.query_latent(q[None], Wm)[0]
+        blk = O.select_blocks(tree, Kls[0], qb, int(i), w.beam, w.topk, w.window)
+        sel = O.selection_tokens(blk, int(i), w.sink, w.window, w.pool)
+        O.sparse_attention(q, Kh[0], Vh, sel)
+    t_query = (time.perf_counter() - t) / len(rows)
+    est = t_lat + t_round * w.lloyd_iters * w.hkv + t_upper * w.hkv + t_query * N * w.hkv * w.batch
+    wall = time.perf_counter() - t_start
+    return {"value": N * w.batch / est, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+            "sample": (f"numpy fp64 oracle: latents of all {w.hkv} KV heads in full ({t_lat:.1f} s); one full-size "
+                       f"Lloyd round of one KV head ({t_round:.1f} s) x {w.lloyd_iters} rounds x {w.hkv} heads; "
+                       f"upper levels in full ({t_upper:.1f} s) x {w.hkv}; select+attention on {len(rows)} "
+                       f"sampled queries ({t_query * 1e3:.1f} ms each) x {N} queries x {w.hkv} heads; "
+                       f"estimated layer time {est:.0f} s from {wall:.0f} s of CPU work"),
+            "estimated_layer_s": est}
+
+
+def run_reference(args):
+    import torch
+    rank, world, local = dist_env()
+    if rank != 0:
+        return
+    from hierarchical_latent_key_gemm_b200.workloads import WORKLOADS, describe, make_inputs
+    w = WORKLOADS[args.workload]
+    dev = torch.device("cuda", local) if torch.cuda.is_available() else torch.device("cpu")
+    inp = make_inputs(w, seed=args.seed, device=dev)
+    vals = []
+    cpu = None
+    for k in range(args.warmup + args.steps):
+        r = cpu_oracle_estimate(w, inp, max(8, args.cpu_sample_queries // 4))
+        if k >= args.warmup:
+            vals.append(r["value"])
+            cpu = r
+    value = statistics.mean(vals)
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": 1e3 * w.n_tokens / value, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": describe(w), "global_batch": w.batch, "seq_len": w.n_tokens,
+                       "parallelism": "host cores of rank 0"},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu["cores"], "kind": "oracle",
+                             "sample": cpu["sample"]},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,170 @@
+// Internal declarations shared by the LSA CUDA translation units.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include <vector>
+
+#include "lsa.h"
+
+namespace lsa {
+
+constexpr uint32_t kIndexMagic = 0x4C534131u;   // "LSA1"
+constexpr uint32_t kFreedMagic = 0xDEADBEEFu;
+constexpr int64_t kNoPos = INT64_MAX;           // minpos of a node with no candidate block
+
+// Error bits latched by kernels into a device word.
+enum : int32_t {
+    kErrDevice = 1,     // out-of-range index met and skipped
+    kErrInexact = 2,    // integer-grid precondition broken
+    kErrCapacity = 4,   // a leaf had no free slot on append
+    kErrTimeout = 8,    // reserved for bounded waits
+};
+
+__device__ __forceinline__ void latch(int32_t* err, int32_t bit) {
+    if (err) atomicOr(err, bit);
+}
+
+// ----------------------------------------------------------- allocation
+// Every device allocation of the library goes through Arena, so a failed
+// build frees all it took and the test hook can force a failure.
+struct Arena {
+    std::vector<void*> ptrs;
+    int64_t bytes = 0;
+    cudaStream_t stream = nullptr;
+    bool async = false;    // stream-ordered scratch (cudaMallocAsync) vs persistent
+    int status = LSA_OK;
+
+    template <typename T>
+    T* alloc(int64_t count) {
+        if (status != LSA_OK) return nullptr;
+        void* p = nullptr;
+        int64_t nbytes = count * (int64_t)sizeof(T);
+        if (nbytes <= 0) nbytes = 256;
+        nbytes = (nbytes + 255) & ~int64_t(255);
+        if (!alloc_raw(&p, nbytes)) {
+            status = LSA_ERR_OOM;
+            return nullptr;
+        }
+        ptrs.push_back(p);
+        bytes += nbytes;
+        return static_cast<T*>(p);
+    }
+    bool alloc_raw(void** p, int64_t nbytes);
+    void release();
+    ~Arena() { release(); }
+};
+
+// Counts down the OOM test hook; true = this allocation must fail.
+bool debug_alloc_should_fail();
+
+// Host-side count of kernel launches issued by the library (diagnostics).
+void note_launch();
+
+}  // namespace lsa
+
+struct lsa_index {
+    uint32_t magic;
+    lsa_build_params p;
+    int device;
+    int64_t units;         // batch * hkv
+    int64_t nb;            // complete blocks indexed per unit
+    int64_t nb_cap;        // block capacity per unit (row stride of Kl)
+    int64_t n_tokens;      // tokens indexed per sequence
+    int64_t slots;         // total bucket slots over all units
+    int32_t L;             // leaves
+    float* W;              // [d][r]
+    float* Kl;             // [units][nb_cap][r] latent keys, block order
+    float* Klp;            // [slots][r] latent keys, bucket order
+    int32_t* blk;          // [slots] block id (within its unit) of every slot
+    int32_t* leaf_start;   // [units*L] first slot of each leaf (global slot index)
+    int32_t* leaf_cnt;     // [units*L] blocks in each leaf
+    int32_t* leaf_cap;     // [units*L] slots reserved for each leaf
+    int32_t* leaf_of_block;// [units][nb_cap]
+    float* cent[LSA_MAX_LEVELS];      // [units*n_l][r]
+    int64_t* minpos[LSA_MAX_LEVELS];  // [units*n_l]
+    int32_t* parent[LSA_MAX_LEVELS];  // [units*n_l] node id at level l-1 (l >= 1)
+    int32_t* child_off[LSA_MAX_LEVELS];  // [units*n_l + 1] into child_ids (l < levels-1)
+    int32_t* child_ids[LSA_MAX_LEVELS];  // [units*n_{l+1}] child id within the unit
+    double* objective[LSA_MAX_LEVELS];   // [iters][units]
+    int32_t* err;          // latched kernel error bits
+    lsa::Arena* mem;       // owns every device allocation above
+};
+
+namespace lsa {
+
+int cuda_status(cudaError_t e);
+int err_bits_to_status(int32_t bits);
+
+// Library-wide error word for calls that have no index (attention, stages).
+int32_t* global_err_word();
+
+// ---------------------------------------------------------------- sort/scan
+// Exclusive prefix sum of n int32 values; out[n] receives the total when
+// out_len > n.  scratch: see scan_scratch_elems.
+int64_t scan_scratch_elems(int64_t n);
+void scan_exclusive(const int32_t* in, int32_t* out, int64_t n, int32_t* scratch, cudaStream_t s);
+
+// Stable LSD radix sort of (key, value) pairs by the low `bits` bits of key.
+// Buffers: k0/v0 hold the input; the sorted result lands in *kout/*vout
+// (one of the two buffer pairs).
+int64_t radix_scratch_elems(int64_t n);
+void radix_sort(uint32_t* k0, int32_t* v0, uint32_t* k1, int32_t* v1, int64_t n, int bits,
+                int32_t* scratch, cudaStream_t s, uint32_t** kout, int32_t** vout);
+
+// ---------------------------------------------------------------- k-means
+struct KmeansOut {
+    int32_t* labels;    // [units*n] local labels (last assign)
+    float* C;           // [units*k][r] last update
+    int32_t* perm;      // [units*n] global point ids (u*n+i) sorted by (u, label), stable
+    int32_t* off;       // [units*k + 1] global offsets into perm
+    double* objective;  // [iters][units] or null
+};
+// X: [units][ldx][r] (rows 0..n-1 of each unit are the points); labels are
+// written at out.labels[u*ldl + i].
+int run_kmeans(const float* X, int64_t ldx, int64_t units, int64_t n, int r, int k, int iters,
+               int grid_log2, KmeansOut out, int64_t ldl, int32_t* err, cudaStream_t s, Arena& scratch);
+
+// Stable grouping of points by label (see run_kmeans); workspace sized for
+// (units, n, k) by alloc_group_work.
+struct GroupWork {
+    int64_t total = 0, nc = 0;
+    uint32_t *k0 = nullptr, *k1 = nullptr;
+    int32_t *v0 = nullptr, *v1 = nullptr, *counts = nullptr, *scratch = nullptr;
+};
+GroupWork alloc_group_work(int64_t units, int64_t n, int k, Arena& A);
+int group_by_label(const int32_t* labels, int64_t ldl, int64_t units, int64_t n, int k, int32_t* perm,
+                   int32_t* off, int32_t* err, cudaStream_t s, const GroupWork& w);
+
+// ---------------------------------------------------------------- latents
+int launch_project_pool(const void* K, const float* W, int64_t batch, int64_t n_blocks,
+                        int64_t ld_tokens, int hkv, int d, int r, int pool, int dtype,
+                        float* Kl, int64_t kl_unit_stride, cudaStream_t s);
+int launch_query_latent(const void* Q, const float* W, int64_t batch, int64_t nq, int hq, int hkv,
+                        int d, int r, int dtype, float* qbar, cudaStream_t s);
+
+// ---------------------------------------------------------------- select
+int launch_select(const lsa_index* ix, const lsa_select_params* sp, const float* qbar, int64_t nq,
+                  const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt, int max_sel,
+                  bool fullscan, cudaStream_t s);
+
+// ---------------------------------------------------------------- attention
+int launch_sparse_attn(const void* Q, const void* K, const void* V, const int32_t* idx,
+                       const int32_t* cnt, int64_t batch, int64_t nq, int hq, int hkv, int d,
+                       int dtype, int max_sel, int64_t ld_tokens, void* O, float* lse,
+                       int32_t* err, cudaStream_t s);
+
+// ---------------------------------------------------------------- append
+int launch_append(lsa_index* ix, const void* K, int64_t first_block, int64_t n_new_blocks,
+                  cudaStream_t s);
+
+// ---------------------------------------------------------------- tree finish
+// Given leaf labels with their stable order, the upper-level parents with
+// theirs, and the centroids, lay out the buckets, child lists and minpos.
+int finish_tree(lsa_index* ix, const int32_t* leaf_perm, const int32_t* leaf_off,
+                const int32_t* const* up_perm, const int32_t* const* up_off, cudaStream_t s,
+                Arena& scratch);
+
+}  // namespace lsa

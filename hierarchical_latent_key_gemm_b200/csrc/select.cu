@@ -1,0 +1,451 @@
+// Key selection: tree search and the full-scan baseline.
+//
+// Tree search ("a query scores cluster centroids and descends into the best
+// few buckets", tree-search wiki note, TL;DR; "scores the clusters, and then
+// scores the keys within the selected clusters", 10M-token attention post;
+// LSA explainer, "How does LSA work?" steps 2-3): per (query, KV head), level
+// by level, score the eligible nodes (all top nodes, then the children of the
+// kept ones) and keep the best `beam`; score the candidate blocks inside the
+// kept leaves and keep the best ceil(K/P); emit sink + blocks + window.
+//
+// Full scan (the "old indexer" of the wiki note's flowchart): the same top-K
+// over every candidate block, no tree.
+//
+// One CTA per (query, KV head).  Candidates stream through a shared-memory
+// buffer: scores are appended, and whenever the buffer holds more than k
+// items a block-wide radix select (on the order-preserving bit pattern of the
+// fp32 score, then on the id for ties) compacts it to the top k.  Order is
+// total: (score desc, id asc), so the result does not depend on the order in
+// which warps append.  Each score is a fp32 dot product of the fp32 latent
+// query with an fp32 latent row: sub-warp groups of r/8 lanes load one row
+// with two 16-byte loads per lane and reduce by xor shuffles.
+#include "lsa_internal.cuh"
+
+namespace lsa {
+namespace {
+
+constexpr int kSelThreads = 128;
+constexpr int kMaxBeam = 1024;
+
+struct SelArgs {
+    const float* cent[LSA_MAX_LEVELS];
+    const int64_t* minpos[LSA_MAX_LEVELS];
+    const int32_t* child_off[LSA_MAX_LEVELS];
+    const int32_t* child_ids[LSA_MAX_LEVELS];
+    int n_l[LSA_MAX_LEVELS];
+    int levels;
+    const float* Klp;
+    const int32_t* blk;
+    const int32_t* leaf_start;
+    const int32_t* leaf_cnt;
+    const float* Kl;
+    int64_t nb_cap, nb;
+    int pool, sink, window, beam, kb, hkv;
+    int64_t nq;
+    const float* qbar;
+    const int64_t* q_pos;
+    int64_t q_pos0;
+    int32_t* idx;
+    int32_t* cnt;
+    int max_sel;
+    int cap;
+};
+
+struct SelShared {
+    int hist[256];
+    int bc[4];
+    int count;
+    int count2;
+    int nkept;
+    int kk[kMaxBeam];
+    int pre[kMaxBeam + 1];
+    int lo[kMaxBeam];
+};
+
+// Order-preserving map of a float onto uint32 (-0 and +0 map together).
+__device__ __forceinline__ uint32_t fkey(float f) {
+    const uint32_t u = __float_as_uint(__fadd_rn(f, 0.0f));
+    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ int warp_incl_scan(int v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        int t = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += t;
+    }
+    return v;
+}
+
+// k-th largest key among n items (1 <= k <= n).  mode 0: key = fkey(score);
+// mode 1: key = ~id, restricted to items with fkey(score) == tkey.
+// Returns the key; *need = how many items equal to it are in the top k,
+// *eq = how many items equal it.
+__device__ uint32_t block_kth(const float* s, const int* id, int n, int k, int mode, uint32_t tkey,
+                              SelShared& sh, int* need, int* eq) {
+    uint32_t prefix = 0, pmask = 0;
+    int kk = k, eqc = 0;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int b = threadIdx.x; b < 256; b += blockDim.x) sh.hist[b] = 0;
+        __syncthreads();
+        for (int i = threadIdx.x; i < n; i += blockDim.x) {
+            uint32_t key;
+            bool act;
+            if (mode == 0) {
+                key = fkey(s[i]);
+                act = true;
+            } else {
+                act = fkey(s[i]) == tkey;
+                key = ~(uint32_t)id[i];
+            }
+            if (act && (key & pmask) == prefix) atomicAdd(&sh.hist[(key >> shift) & 255u], 1);
+        }
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            const int lane = threadIdx.x;
+            int c[8], sum = 0;
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                c[t] = sh.hist[255 - lane * 8 - t];
+                sum += c[t];
+            }
+            const int incl = warp_incl_scan(sum);
+            const int excl = incl - sum;
+            if (excl < kk && kk <= incl) {
+                int run = excl;
+#pragma unroll
+                for (int t = 0; t < 8; ++t) {
+                    if (run + c[t] >= kk) {
+                        sh.bc[0] = 255 - lane * 8 - t;
+                        sh.bc[1] = kk - run;
+                        sh.bc[2] = c[t];
+                        break;
+                    }
+                    run += c[t];
+                }
+            }
+        }
+        __syncthreads();
+        const int dg = sh.bc[0];
+        kk = sh.bc[1];
+        eqc = sh.bc[2];
+        prefix |= (uint32_t)dg << shift;
+        pmask |= 255u << shift;
+        __syncthreads();
+    }
+    *need = kk;
+    *eq = eqc;
+    return prefix;
+}
+
+// Keep the top k of the n items in (s, id); result in (ds, di)[0..k).
+__device__ void topk_compact(const float* s, const int* id, int n, int k, float* ds, int* di, SelShared& sh) {
+    int need, eq;
+    const uint32_t T = block_kth(s, id, n, k, 0, 0u, sh, &need, &eq);
+    const bool split = need < eq;
+    uint32_t T2 = 0;
+    if (split) {
+        int need2, eq2;
+        T2 = block_kth(s, id, n, need, 1, T, sh, &need2, &eq2);
+    }
+    if (threadIdx.x == 0) sh.count2 = 0;
+    __syncthreads();
+    for (int i = threadIdx.x; i < n; i += blockDim.x) {
+        const uint32_t key = fkey(s[i]);
+        const bool take = key > T || (key == T && (!split || ~(uint32_t)id[i] >= T2));
+        if (take) {
+            const int p = atomicAdd(&sh.count2, 1);
+            ds[p] = s[i];
+            di[p] = id[i];
+        }
+    }
+    __syncthreads();
+}
+
+// Exclusive scan of sh.pre[0..n) in place (values are counts), sh.pre[n] = total.
+__device__ void scan_pre(SelShared& sh, int n) {
+    __syncthreads();
+    if (threadIdx.x < 32) {
+        const int lane = threadIdx.x;
+        int carry = 0;
+        for (int base = 0; base < n; base += 32) {
+            const int v = (base + lane < n) ? sh.pre[base + lane] : 0;
+            const int incl = warp_incl_scan(v);
+            if (base + lane < n) sh.pre[base + lane] = carry + incl - v;
+            carry += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        if (lane == 0) sh.pre[n] = carry;
+    }
+    __syncthreads();
+}
+
+__device__ __forceinline__ int find_owner(const SelShared& sh, int nk, int t) {
+    int lo = 0, hi = nk;  // sh.pre[lo] <= t < sh.pre[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (sh.pre[mid] <= t) lo = mid; else hi = mid;
+    }
+    return lo;
+}
+
+template <int R, bool FULL>
+__global__ __launch_bounds__(kSelThreads) void select_kernel(const SelArgs a) {
+    extern __shared__ float4 dyn4[];
+    __shared__ SelShared sh;
+    float* bsb[2];
+    int* bib[2];
+    bsb[0] = reinterpret_cast<float*>(dyn4);
+    bib[0] = reinterpret_cast<int*>(bsb[0] + a.cap);
+    bsb[1] = reinterpret_cast<float*>(bib[0] + a.cap);
+    bib[1] = reinterpret_cast<int*>(bsb[1] + a.cap);
+
+    constexpr int LPC = R / 8;              // lanes per candidate row
+    constexpr int CPW = 32 / LPC;           // candidates per warp
+    constexpr int NG = (kSelThreads / 32) * CPW;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane / LPC, gl = lane % LPC, gid = warp * CPW + g;
+    const unsigned gmask = (LPC == 32) ? 0xffffffffu : (((1u << LPC) - 1u) << (g * LPC));
+
+    const int64_t qi = blockIdx.x;
+    const int u = blockIdx.y;
+    const int64_t bseq = u / a.hkv;
+    const int h = u % a.hkv;
+    const int64_t row = (bseq * a.nq + qi) * a.hkv + h;
+    const int64_t pos = a.q_pos ? a.q_pos[bseq * a.nq + qi] : a.q_pos0 + qi;
+    const int64_t bound = pos - a.window - a.pool + 1;
+    const int64_t b_lo = (a.sink + a.pool - 1) / a.pool;
+    const int64_t b_hi = bound >= 0 ? bound / a.pool : -1;
+
+    float qv[8];
+    {
+        const float4* qp = reinterpret_cast<const float4*>(a.qbar + row * R + gl * 8);
+        const float4 x0 = qp[0], x1 = qp[1];
+        qv[0] = x0.x; qv[1] = x0.y; qv[2] = x0.z; qv[3] = x0.w;
+        qv[4] = x1.x; qv[5] = x1.y; qv[6] = x1.z; qv[7] = x1.w;
+    }
+    auto dot = [&](const float* p) -> float {
+        const float4* v = reinterpret_cast<const float4*>(p + gl * 8);
+        const float4 y0 = __ldg(v), y1 = __ldg(v + 1);
+        float s = 0.f;
+        s = __fmaf_rn(qv[0], y0.x, s); s = __fmaf_rn(qv[1], y0.y, s);
+        s = __fmaf_rn(qv[2], y0.z, s); s = __fmaf_rn(qv[3], y0.w, s);
+        s = __fmaf_rn(qv[4], y1.x, s); s = __fmaf_rn(qv[5], y1.y, s);
+        s = __fmaf_rn(qv[6], y1.z, s); s = __fmaf_rn(qv[7], y1.w, s);
+#pragma unroll
+        for (int o = LPC / 2; o >= 1; o >>= 1) s = __fadd_rn(s, __shfl_xor_sync(gmask, s, o));
+        return s;
+    };
+
+    int cur = 0;
+    if (threadIdx.x == 0) { sh.count = 0; sh.nkept = 0; }
+    __syncthreads();
+
+    // Push candidates t in [0, total) through the buffer, keeping the top k.
+    // get(t, &id, &rowptr) returns false when t is not eligible.
+    auto stream_topk = [&](int total, int k, auto&& get) {
+        if (k <= 0) return;  // nothing is kept; the buffer stays empty
+        const int chunk = a.cap - k;
+        for (int t0 = 0; t0 < total; t0 += chunk) {
+            const int t1 = min(total, t0 + chunk);
+            float* bs = bsb[cur];
+            int* bi = bib[cur];
+            for (int t = t0 + gid; t < t1; t += NG) {
+                int id;
+                const float* rp;
+                if (get(t, &id, &rp)) {
+                    const float sc = dot(rp);
+                    if (gl == 0) {
+                        const int p = atomicAdd(&sh.count, 1);
+                        bs[p] = sc;
+                        bi[p] = id;
+                    }
+                }
+            }
+            __syncthreads();
+            const int n = sh.count;
+            if (n > k) {
+                topk_compact(bs, bi, n, k, bsb[cur ^ 1], bib[cur ^ 1], sh);
+                cur ^= 1;
+                if (threadIdx.x == 0) sh.count = k;
+            }
+            __syncthreads();
+        }
+    };
+
+    int nsel;
+    if (!FULL) {
+        for (int l = 0; l < a.levels; ++l) {
+            const int nl = a.n_l[l];
+            const float* cent = a.cent[l] + (int64_t)u * nl * R;
+            const int64_t* mp = a.minpos[l] + (int64_t)u * nl;
+            const int nk = sh.nkept;
+            const int total = (l == 0) ? nl : sh.pre[nk];
+            const int32_t* coff = l > 0 ? a.child_off[l - 1] + (int64_t)u * a.n_l[l - 1] : nullptr;
+            const int32_t* cids = l > 0 ? a.child_ids[l - 1] : nullptr;
+            if (threadIdx.x == 0) sh.count = 0;
+            __syncthreads();
+            stream_topk(total, a.beam, [&](int t, int* id, const float** rp) -> bool {
+                int node;
+                if (l == 0) {
+                    node = t;
+                } else {
+                    const int p = find_owner(sh, nk, t);
+                    node = cids[coff[sh.kk[p]] + (t - sh.pre[p])];
+                }
+                if (mp[node] > bound) return false;
+                *id = node;
+                *rp = cent + (int64_t)node * R;
+                return true;
+            });
+            const int n = sh.count;
+            for (int e = threadIdx.x; e < n; e += blockDim.x) sh.kk[e] = bib[cur][e];
+            __syncthreads();
+            if (threadIdx.x == 0) sh.nkept = n;
+            if (l + 1 < a.levels) {
+                const int32_t* co = a.child_off[l] + (int64_t)u * nl;
+                for (int e = threadIdx.x; e < n; e += blockDim.x) {
+                    const int node = bib[cur][e];
+                    sh.pre[e] = co[node + 1] - co[node];
+                }
+                scan_pre(sh, n);
+            }
+            __syncthreads();
+        }
+        // candidate slot range of every kept leaf
+        const int nk = sh.nkept;
+        const int L = a.n_l[a.levels - 1];
+        for (int e = threadIdx.x; e < nk; e += blockDim.x) {
+            const int leaf = sh.kk[e];
+            const int64_t c = (int64_t)u * L + leaf;
+            const int st = a.leaf_start[c];
+            const int cntl = a.leaf_cnt[c];
+            const int32_t* bl = a.blk + st;
+            int lo = 0, hi = cntl;  // first index with bl >= b_lo
+            while (lo < hi) { const int m = (lo + hi) >> 1; if (bl[m] < b_lo) lo = m + 1; else hi = m; }
+            int lo2 = lo, hi2 = cntl; // first index with bl > b_hi
+            while (lo2 < hi2) { const int m = (lo2 + hi2) >> 1; if (bl[m] <= b_hi) lo2 = m + 1; else hi2 = m; }
+            sh.lo[e] = st + lo;
+            sh.pre[e] = lo2 - lo;
+        }
+        scan_pre(sh, nk);
+        if (threadIdx.x == 0) sh.count = 0;
+        __syncthreads();
+        stream_topk(sh.pre[nk], a.kb, [&](int t, int* id, const float** rp) -> bool {
+            const int p = find_owner(sh, nk, t);
+            const int64_t slot = sh.lo[p] + (t - sh.pre[p]);
+            *id = a.blk[slot];
+            *rp = a.Klp + slot * R;
+            return true;
+        });
+    } else {
+        const int64_t hi = min(a.nb - 1, b_hi);
+        const int total = hi >= b_lo ? (int)(hi - b_lo + 1) : 0;
+        const float* kl = a.Kl + (int64_t)u * a.nb_cap * R;
+        stream_topk(total, a.kb, [&](int t, int* id, const float** rp) -> bool {
+            const int64_t b = b_lo + t;
+            *id = (int)b;
+            *rp = kl + b * R;
+            return true;
+        });
+    }
+    nsel = sh.count;
+
+    // ascending block ids (bitonic sort, padded to a power of two)
+    int M = 1;
+    while (M < nsel) M <<= 1;
+    int* arr = bib[cur ^ 1];
+    for (int e = threadIdx.x; e < M; e += blockDim.x) arr[e] = e < nsel ? bib[cur][e] : INT32_MAX;
+    __syncthreads();
+    for (int size = 2; size <= M; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            for (int t = threadIdx.x; t < (M >> 1); t += blockDim.x) {
+                const int i = 2 * stride * (t / stride) + (t % stride);
+                const int j = i + stride;
+                const bool asc = (i & size) == 0;
+                const int x = arr[i], y = arr[j];
+                if ((x > y) == asc) { arr[i] = y; arr[j] = x; }
+            }
+            __syncthreads();
+        }
+    }
+
+    const int64_t lo_w = max((int64_t)0, pos - a.window + 1);
+    const int64_t ns = min((int64_t)a.sink, lo_w);
+    const int64_t nblk_tok = (int64_t)nsel * a.pool;
+    const int64_t total = ns + nblk_tok + (pos - lo_w + 1);
+    int32_t* out = a.idx + row * a.max_sel;
+    for (int e = threadIdx.x; e < a.max_sel; e += blockDim.x) {
+        int64_t v;
+        if (e < ns) v = e;
+        else if (e < ns + nblk_tok) { const int64_t t = e - ns; v = (int64_t)arr[t / a.pool] * a.pool + t % a.pool; }
+        else if (e < total) v = lo_w + (e - ns - nblk_tok);
+        else v = -1;
+        out[e] = (int32_t)v;
+    }
+    if (threadIdx.x == 0) a.cnt[row] = (int32_t)total;
+}
+
+template <int R>
+int launch_select_r(const SelArgs& a, int64_t nq, int64_t units, bool fullscan, cudaStream_t s) {
+    const size_t smem = (size_t)a.cap * 16;
+    auto kern = fullscan ? select_kernel<R, true> : select_kernel<R, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_status(e);
+    dim3 grid((unsigned)nq, (unsigned)units);
+    note_launch();
+    kern<<<grid, kSelThreads, smem, s>>>(a);
+    return cuda_status(cudaGetLastError());
+}
+
+}  // namespace
+
+int launch_select(const lsa_index* ix, const lsa_select_params* sp, const float* qbar, int64_t nq,
+                  const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt, int max_sel, bool fullscan,
+                  cudaStream_t s) {
+    const lsa_build_params& p = ix->p;
+    if (sp->beam > kMaxBeam) return LSA_ERR_INVALID_ARG;
+    SelArgs a{};
+    for (int l = 0; l < p.levels; ++l) {
+        a.cent[l] = ix->cent[l];
+        a.minpos[l] = ix->minpos[l];
+        a.child_off[l] = ix->child_off[l];
+        a.child_ids[l] = ix->child_ids[l];
+        a.n_l[l] = p.level_sizes[l];
+    }
+    a.levels = p.levels;
+    a.Klp = ix->Klp;
+    a.blk = ix->blk;
+    a.leaf_start = ix->leaf_start;
+    a.leaf_cnt = ix->leaf_cnt;
+    a.Kl = ix->Kl;
+    a.nb_cap = ix->nb_cap;
+    a.nb = ix->nb;
+    a.pool = p.pool;
+    a.sink = p.sink;
+    a.window = sp->window;
+    a.beam = sp->beam;
+    a.kb = (sp->topk + p.pool - 1) / p.pool;
+    a.hkv = p.hkv;
+    a.nq = nq;
+    a.qbar = qbar;
+    a.q_pos = q_pos;
+    a.q_pos0 = q_pos0;
+    a.idx = idx;
+    a.cnt = cnt;
+    a.max_sel = max_sel;
+    const int kmax = a.kb > a.beam ? a.kb : a.beam;
+    int cap = 2048;
+    while (cap < 2 * kmax) cap <<= 1;
+    a.cap = cap;
+    if (nq <= 0) return LSA_OK;
+    switch (p.r) {
+        case 16: return launch_select_r<16>(a, nq, ix->units, fullscan, s);
+        case 32: return launch_select_r<32>(a, nq, ix->units, fullscan, s);
+        case 64: return launch_select_r<64>(a, nq, ix->units, fullscan, s);
+        case 128: return launch_select_r<128>(a, nq, ix->units, fullscan, s);
+        default: return LSA_ERR_INVALID_ARG;
+    }
+}
+
+}  // namespace lsa

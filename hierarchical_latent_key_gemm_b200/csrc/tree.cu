@@ -1,0 +1,108 @@
+// Bucket layout of a built tree.
+//
+// Leaves store their blocks contiguously ("descends into the best few
+// buckets", tree-search wiki note, TL;DR): slots [leaf_start, leaf_start +
+// leaf_cnt) hold the member blocks in ascending block order, followed by
+// free slots that decode appends fill.  The latent keys are copied into the
+// same order (Klp), so scoring a bucket reads one contiguous run.  Child
+// lists of every upper node are ascending child ids.  minpos of a node is the
+// smallest start position of a member block at or after the sink (kNoPos if
+// none); a node is eligible for the query at i iff minpos <= i - W - P + 1.
+#include "lsa_internal.cuh"
+
+namespace lsa {
+namespace {
+
+__global__ void leaf_cap_kernel(const int32_t* __restrict__ off, int64_t nc, int64_t append_blocks, int64_t denom,
+                                int32_t* __restrict__ cap) {
+    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= nc) return;
+    const int64_t cnt = off[c + 1] - off[c];
+    int64_t slack = 0;
+    if (append_blocks > 0) slack = 2 + (2 * append_blocks * (cnt + 1) + denom - 1) / denom;
+    cap[c] = (int32_t)(cnt + slack);
+}
+
+__global__ void leaf_layout_kernel(const int32_t* __restrict__ perm, const int32_t* __restrict__ off, int64_t nb,
+                                   int L, int64_t nc, const int32_t* __restrict__ leaf_start,
+                                   int32_t* __restrict__ leaf_cnt, const float* __restrict__ Kl, int64_t nb_cap,
+                                   int r, float* __restrict__ Klp, int32_t* __restrict__ blk, int pool, int sink,
+                                   int64_t* __restrict__ minpos) {
+    const int64_t c = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (c >= nc) return;
+    const int64_t u = c / L;
+    const int32_t s = off[c], e = off[c + 1];
+    const int32_t st = leaf_start[c];
+    int64_t mp = kNoPos;
+    for (int32_t m = s; m < e; ++m) {
+        const int64_t i = perm[m] - u * nb;
+        const int64_t slot = st + (m - s);
+        if (lane == 0) blk[slot] = (int32_t)i;
+        for (int dim = lane; dim < r; dim += 32) Klp[slot * r + dim] = Kl[(u * nb_cap + i) * r + dim];
+        if (mp == kNoPos && i * pool >= sink) mp = i * pool;
+    }
+    if (lane == 0) {
+        leaf_cnt[c] = e - s;
+        minpos[c] = mp;
+    }
+}
+
+__global__ void child_ids_kernel(const int32_t* __restrict__ perm, int64_t total, int64_t n_child,
+                                 int32_t* __restrict__ child_ids) {
+    const int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (p >= total) return;
+    const int64_t g = perm[p];
+    child_ids[p] = (int32_t)(g % n_child);
+}
+
+__global__ void minpos_up_kernel(const int32_t* __restrict__ child_off, const int32_t* __restrict__ child_ids,
+                                 int64_t nc, int n_l, int n_child, const int64_t* __restrict__ mp_child,
+                                 int64_t* __restrict__ mp) {
+    const int64_t c = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (c >= nc) return;
+    const int64_t u = c / n_l;
+    int64_t best = kNoPos;
+    for (int32_t q = child_off[c]; q < child_off[c + 1]; ++q) {
+        const int64_t v = mp_child[u * n_child + child_ids[q]];
+        if (v < best) best = v;
+    }
+    mp[c] = best;
+}
+
+}  // namespace
+
+int finish_tree(lsa_index* ix, const int32_t* leaf_perm, const int32_t* leaf_off, const int32_t* const* up_perm,
+                const int32_t* const* up_off, cudaStream_t s, Arena& A) {
+    const lsa_build_params& p = ix->p;
+    const int levels = p.levels;
+    const int L = ix->L;
+    const int64_t U = ix->units;
+    const int64_t nc = U * L;
+    const int64_t append_blocks = p.append_capacity > 0 ? (p.append_capacity + p.pool - 1) / p.pool + 1 : 0;
+    int32_t* cap = A.alloc<int32_t>(nc);
+    int32_t* sc = A.alloc<int32_t>(scan_scratch_elems(nc) + 1);
+    if (A.status != LSA_OK) return A.status;
+    note_launch();
+    leaf_cap_kernel<<<(unsigned)((nc + 255) / 256), 256, 0, s>>>(leaf_off, nc, append_blocks, ix->nb + L, cap);
+    cudaMemcpyAsync(ix->leaf_cap, cap, nc * sizeof(int32_t), cudaMemcpyDeviceToDevice, s);
+    scan_exclusive(cap, ix->leaf_start, nc, sc, s);
+    note_launch();
+    leaf_layout_kernel<<<(unsigned)((nc * 32 + 255) / 256), 256, 0, s>>>(
+        leaf_perm, leaf_off, ix->nb, L, nc, ix->leaf_start, ix->leaf_cnt, ix->Kl, ix->nb_cap, p.r, ix->Klp, ix->blk,
+        p.pool, p.sink, ix->minpos[levels - 1]);
+    for (int l = levels - 2; l >= 0; --l) {
+        const int n_l = p.level_sizes[l], n_child = p.level_sizes[l + 1];
+        const int64_t tot = U * n_child;
+        cudaMemcpyAsync(ix->child_off[l], up_off[l], (U * n_l + 1) * sizeof(int32_t), cudaMemcpyDeviceToDevice, s);
+        note_launch();
+        child_ids_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, s>>>(up_perm[l], tot, n_child, ix->child_ids[l]);
+        note_launch();
+        minpos_up_kernel<<<(unsigned)((U * n_l + 255) / 256), 256, 0, s>>>(ix->child_off[l], ix->child_ids[l],
+                                                                           U * n_l, n_l, n_child,
+                                                                           ix->minpos[l + 1], ix->minpos[l]);
+    }
+    return cuda_status(cudaGetLastError());
+}
+
+}  // namespace lsa

@@ -1,0 +1,302 @@
+"""Python binding of liblsa.so (the C ABI declared in include/lsa.h).
+
+Argument marshalling only: every step of the path runs in the library's CUDA
+kernels.  Tensors are torch tensors used as device memory; the stream is
+torch's current stream unless one is given.  The binding refuses to run
+without the compiled library (there is no fallback).
+"""
+from __future__ import annotations
+
+import ctypes as C
+import os
+from dataclasses import dataclass
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "liblsa.so")
+
+LSA_OK, LSA_ERR_INVALID_ARG, LSA_ERR_CUDA, LSA_ERR_OOM = 0, 1, 2, 3
+LSA_ERR_INEXACT, LSA_ERR_TIMEOUT, LSA_ERR_DEVICE, LSA_ERR_CAPACITY = 4, 5, 6, 7
+LSA_F32, LSA_BF16 = 0, 1
+LSA_MAX_LEVELS = 4
+(LSA_GET_CENTROIDS, LSA_GET_PARENT, LSA_GET_LEAF_OF_BLOCK, LSA_GET_MINPOS,
+ LSA_GET_OBJECTIVE, LSA_GET_LATENT, LSA_GET_LEAF_COUNT) = range(7)
+
+
+class LsaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {strerror(status)} (status {status})")
+
+
+class BuildParams(C.Structure):
+    _fields_ = [("batch", C.c_int64), ("n_tokens", C.c_int64), ("ld_tokens", C.c_int64),
+                ("hkv", C.c_int32), ("d", C.c_int32), ("r", C.c_int32), ("pool", C.c_int32),
+                ("dtype", C.c_int32), ("levels", C.c_int32), ("level_sizes", C.c_int32 * LSA_MAX_LEVELS),
+                ("lloyd_iters", C.c_int32), ("grid_log2", C.c_int32), ("sink", C.c_int32),
+                ("append_capacity", C.c_int64)]
+
+
+class SelectParams(C.Structure):
+    _fields_ = [("hq", C.c_int32), ("beam", C.c_int32), ("topk", C.c_int32), ("sink", C.c_int32),
+                ("window", C.c_int32)]
+
+
+class IndexInfo(C.Structure):
+    _fields_ = [("units", C.c_int64), ("n_tokens", C.c_int64), ("n_blocks", C.c_int64),
+                ("block_capacity", C.c_int64), ("device_bytes", C.c_int64), ("levels", C.c_int32),
+                ("level_sizes", C.c_int32 * LSA_MAX_LEVELS), ("r", C.c_int32), ("pool", C.c_int32),
+                ("sink", C.c_int32), ("grid_log2", C.c_int32)]
+
+
+_vp, _i64, _i32 = C.c_void_p, C.c_int64, C.c_int32
+_SIGS = {
+    "lsa_build_index": (_i32, [C.POINTER(BuildParams), _vp, _vp, _vp, C.POINTER(_vp)]),
+    "lsa_build_index_from_tree": (_i32, [C.POINTER(BuildParams), _vp, _vp, _vp, C.POINTER(_vp), C.POINTER(_vp),
+                                         _vp, C.POINTER(_vp)]),
+    "lsa_select": (_i32, [_vp, C.POINTER(SelectParams), _vp, _i64, _vp, _i64, _vp, _vp, _i32, _vp]),
+    "lsa_fullscan_select": (_i32, [_vp, C.POINTER(SelectParams), _vp, _i64, _vp, _i64, _vp, _vp, _i32, _vp]),
+    "lsa_sparse_attn": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _i64, _vp, _vp,
+                               _vp]),
+    "lsa_append": (_i32, [_vp, _vp, _i64, _vp]),
+    "lsa_project_pool": (_i32, [_vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
+    "lsa_query_latent": (_i32, [_vp, _vp, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
+    "lsa_kmeans": (_i32, [_vp, _i64, _i64, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp]),
+    "lsa_index_get": (_i32, [_vp, _i32, _i32, _vp, _i64, _vp]),
+    "lsa_index_info": (_i32, [_vp, C.POINTER(IndexInfo)]),
+    "lsa_check": (_i32, [_vp, _vp]),
+    "lsa_free_index": (None, [_vp]),
+    "lsa_strerror": (C.c_char_p, [_i32]),
+    "lsa_debug_fail_alloc_after": (None, [_i32]),
+    "lsa_launch_count": (_i64, []),
+}
+
+_lib = None
+
+
+def lib():
+    """The loaded library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: run `python -m hierarchical_latent_key_gemm_b200.build` "
+                               "(the LSA path has no CPU fallback)")
+        L = C.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(L, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = L
+    return _lib
+
+
+def strerror(status: int) -> str:
+    return lib().lsa_strerror(int(status)).decode()
+
+
+def _ok(status, where):
+    if status != LSA_OK:
+        raise LsaError(status, where)
+
+
+def _stream(stream):
+    if stream is None:
+        return C.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, torch.cuda.Stream):
+        return C.c_void_p(stream.cuda_stream)
+    return C.c_void_p(int(stream))
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensor must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return C.c_void_p(t.data_ptr())
+
+
+def dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return LSA_F32
+    if t.dtype == torch.bfloat16:
+        return LSA_BF16
+    raise ValueError(f"unsupported dtype {t.dtype}")
+
+
+@dataclass
+class Index:
+    """Owner of an lsa_index handle (freed by free() or garbage collection)."""
+    handle: C.c_void_p
+    params: BuildParams
+
+    def free(self):
+        if self.handle:
+            lib().lsa_free_index(self.handle)
+            self.handle = C.c_void_p(None)
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
+
+    def info(self) -> IndexInfo:
+        out = IndexInfo()
+        _ok(lib().lsa_index_info(self.handle, C.byref(out)), "lsa_index_info")
+        return out
+
+    def get(self, what: int, level: int = 0, device="cuda") -> torch.Tensor:
+        """Copy one index array out (see LSA_GET_*)."""
+        inf = self.info()
+        U, r, nb = inf.units, inf.r, inf.n_blocks
+        sizes = list(inf.level_sizes)[: inf.levels]
+        L = sizes[-1]
+        it = self.params.lloyd_iters
+        shape, dt = {
+            LSA_GET_CENTROIDS: ((U, sizes[level], r), torch.float32),
+            LSA_GET_PARENT: ((U, sizes[level]), torch.int32),
+            LSA_GET_LEAF_OF_BLOCK: ((U, nb), torch.int32),
+            LSA_GET_MINPOS: ((U, sizes[level]), torch.int64),
+            LSA_GET_OBJECTIVE: ((it, U), torch.float64),
+            LSA_GET_LATENT: ((U, nb, r), torch.float32),
+            LSA_GET_LEAF_COUNT: ((U, L), torch.int32),
+        }[what]
+        out = torch.empty(shape, dtype=dt, device=device)
+        nbytes = out.numel() * out.element_size()
+        _ok(lib().lsa_index_get(self.handle, what, level, C.c_void_p(out.data_ptr()), nbytes, _stream(None)),
+            "lsa_index_get")
+        return out
+
+
+def make_build_params(batch, n_tokens, ld_tokens, hkv, d, r, pool, dtype, level_sizes, lloyd_iters, grid_log2,
+                      sink, append_capacity=0) -> BuildParams:
+    p = BuildParams()
+    p.batch, p.n_tokens, p.ld_tokens = int(batch), int(n_tokens), int(ld_tokens)
+    p.hkv, p.d, p.r, p.pool, p.dtype = int(hkv), int(d), int(r), int(pool), int(dtype)
+    p.levels = len(level_sizes)
+    for i, s in enumerate(level_sizes):
+        p.level_sizes[i] = int(s)
+    p.lloyd_iters, p.grid_log2, p.sink = int(lloyd_iters), int(grid_log2), int(sink)
+    p.append_capacity = int(append_capacity)
+    return p
+
+
+def make_select_params(hq, beam, topk, sink, window) -> SelectParams:
+    s = SelectParams()
+    s.hq, s.beam, s.topk, s.sink, s.window = int(hq), int(beam), int(topk), int(sink), int(window)
+    return s
+
+
+def lsa_build_index(params: BuildParams, K: torch.Tensor, W: torch.Tensor, stream=None) -> Index:
+    h = C.c_void_p()
+    _ok(lib().lsa_build_index(C.byref(params), _ptr(K), _ptr(W), _stream(stream), C.byref(h)), "lsa_build_index")
+    return Index(h, params)
+
+
+def lsa_build_index_from_tree(params: BuildParams, K, W, leaf_of_block, parents, centroids, stream=None) -> Index:
+    """parents[l] for l >= 1 and centroids[l] for every level are device tensors."""
+    L = params.levels
+    par = (C.c_void_p * L)(*([None] + [C.c_void_p(parents[l].data_ptr()) for l in range(1, L)]))
+    cen = (C.c_void_p * L)(*[C.c_void_p(centroids[l].data_ptr()) for l in range(L)])
+    for t in list(parents[1:]) + list(centroids) + [leaf_of_block]:
+        _ptr(t)
+    h = C.c_void_p()
+    _ok(lib().lsa_build_index_from_tree(C.byref(params), _ptr(K), _ptr(W), _ptr(leaf_of_block), par, cen,
+                                        _stream(stream), C.byref(h)), "lsa_build_index_from_tree")
+    return Index(h, params)
+
+
+def _select(fn, name, index, sp, Q, q_pos=None, q_pos0=0, idx=None, cnt=None, max_sel=None, stream=None):
+    p = index.params
+    B, nq = Q.shape[0], Q.shape[1]
+    kb = -(-sp.topk // p.pool)
+    if max_sel is None:
+        max_sel = kb * p.pool + p.sink + sp.window
+    if idx is None:
+        idx = torch.empty((B, nq, p.hkv, max_sel), dtype=torch.int32, device=Q.device)
+    if cnt is None:
+        cnt = torch.empty((B, nq, p.hkv), dtype=torch.int32, device=Q.device)
+    st = fn(index.handle, C.byref(sp), _ptr(Q), int(nq), _ptr(q_pos), int(q_pos0), _ptr(idx), _ptr(cnt),
+            int(max_sel), _stream(stream))
+    _ok(st, name)
+    return idx, cnt
+
+
+def lsa_select(index, sp, Q, **kw):
+    return _select(lib().lsa_select, "lsa_select", index, sp, Q, **kw)
+
+
+def lsa_fullscan_select(index, sp, Q, **kw):
+    return _select(lib().lsa_fullscan_select, "lsa_fullscan_select", index, sp, Q, **kw)
+
+
+def lsa_sparse_attn(Q, K, V, idx, cnt, hkv, O=None, lse=None, want_lse=True, stream=None):
+    B, nq, hq, d = Q.shape
+    ld_tokens = K.shape[1]
+    max_sel = idx.shape[-1]
+    if O is None:
+        O = torch.empty_like(Q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, nq, hq), dtype=torch.float32, device=Q.device)
+    st = lib().lsa_sparse_attn(_ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(cnt), int(B), int(nq), int(hq), int(hkv),
+                               int(d), dtype_code(Q), int(max_sel), int(ld_tokens), _ptr(O), _ptr(lse),
+                               _stream(stream))
+    _ok(st, "lsa_sparse_attn")
+    return O, lse
+
+
+def lsa_append(index: Index, K: torch.Tensor, n_new: int, stream=None):
+    _ok(lib().lsa_append(index.handle, _ptr(K), int(n_new), _stream(stream)), "lsa_append")
+
+
+def lsa_project_pool(K, W, n_tokens, pool, Kl=None, stream=None):
+    B, ld, hkv, d = K.shape
+    r = W.shape[1]
+    nb = n_tokens // pool
+    if Kl is None:
+        Kl = torch.empty((B * hkv, nb, r), dtype=torch.float32, device=K.device)
+    _ok(lib().lsa_project_pool(_ptr(K), _ptr(W), int(B), int(n_tokens), int(ld), int(hkv), int(d), int(r),
+                               int(pool), dtype_code(K), _ptr(Kl), _stream(stream)), "lsa_project_pool")
+    return Kl
+
+
+def lsa_query_latent(Q, W, hkv, qbar=None, stream=None):
+    B, nq, hq, d = Q.shape
+    r = W.shape[1]
+    if qbar is None:
+        qbar = torch.empty((B, nq, hkv, r), dtype=torch.float32, device=Q.device)
+    _ok(lib().lsa_query_latent(_ptr(Q), _ptr(W), int(B), int(nq), int(hq), int(hkv), int(d), int(r),
+                               dtype_code(Q), _ptr(qbar), _stream(stream)), "lsa_query_latent")
+    return qbar
+
+
+def lsa_kmeans(X, k, iters, grid_log2=0, stream=None):
+    U, n, r = X.shape
+    labels = torch.empty((U, n), dtype=torch.int32, device=X.device)
+    Cc = torch.empty((U, k, r), dtype=torch.float32, device=X.device)
+    obj = torch.empty((iters, U), dtype=torch.float64, device=X.device)
+    _ok(lib().lsa_kmeans(_ptr(X), int(U), int(n), int(r), int(k), int(iters), int(grid_log2), _ptr(labels),
+                         _ptr(Cc), _ptr(obj), _stream(stream)), "lsa_kmeans")
+    return labels, Cc, obj
+
+
+def lsa_check(index: Index | None = None, stream=None) -> int:
+    return int(lib().lsa_check(index.handle if index is not None else None, _stream(stream)))
+
+
+def lsa_launch_count() -> int:
+    return int(lib().lsa_launch_count())
+
+
+def lsa_debug_fail_alloc_after(n: int):
+    lib().lsa_debug_fail_alloc_after(int(n))
+
+
+def exported_symbols_from_header(header_path: str) -> list:
+    """Function names declared in include/lsa.h (used by the ABI test)."""
+    import re
+    txt = open(header_path).read()
+    return sorted(set(re.findall(r"^\s*(?:int|void|int64_t|const char\*)\s+(lsa_\w+)\s*\(", txt, re.M)))

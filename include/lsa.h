@@ -1,0 +1,250 @@
+/*
+ * lsa.h - C ABI of the Latent Sparse Attention (LSA) hot path on NVIDIA B200.
+ *
+ * LSA replaces the full key scan of a sparse-attention indexer by a search
+ * through a hierarchy of key clusters built in a low-rank latent space, and
+ * then runs exact softmax attention over the keys it picked.
+ *
+ * Sources (web pages on LSA), cited below by key and section:
+ *  [p1] "The 10M-token attention layer spends 98% of its time finding tokens"
+ *  [p2] "Latent Sparse Attention speeds up the search for useful tokens in very
+ *       long contexts", "Reduce the cost of finding the tokens to attend to"
+ *  [p3] "Latent Sparse Attention: tree search over keys for 10M-token context",
+ *       TL;DR and flowchart
+ *  [p4] "Researchers report 72.4x faster attention-layer prefill at 10 million
+ *       tokens", "Search the clusters, not every key", "Prompt processing is
+ *       not response generation"
+ *  [p5] "Latent Sparse Attention (LSA): The 72.4x and 22.7x Speedups, and What
+ *       They Compare Against", "How does LSA work?" steps 1-3, "Prefill,
+ *       decode and training", "Can I run LSA?"
+ *
+ * Conventions for every call:
+ *  - Pointers named "device" must be CUDA device memory of the current device
+ *    (or managed memory); "host" pointers are ordinary host memory.
+ *  - Tensors are dense, row-major, with the layouts stated per argument.
+ *    Head-of-sequence layouts: K and V are [batch][ld_tokens][hkv][d];
+ *    Q is [batch][nq][hq][d].  dtype is LSA_F32 or LSA_BF16 (IEEE bf16).
+ *  - All work is enqueued on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) and is asynchronous unless stated otherwise.  Argument errors are
+ *    detected on the host and returned before anything is enqueued.
+ *  - Errors found by a kernel (an index out of range, a broken exactness
+ *    precondition, a full leaf) are latched in a device word of the index or
+ *    of the library and reported by lsa_check(), which synchronises.
+ *  - The caller owns every buffer it passes.  An lsa_index owns the device
+ *    memory of the latent keys, centroids and bucket lists; it keeps no
+ *    pointer to the caller's K, Q, V or W after a call returns.
+ *  - No call aborts or throws.  Every int-returning call returns an
+ *    lsa_status code.
+ */
+#ifndef LSA_H_
+#define LSA_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct lsa_index lsa_index;
+
+typedef enum {
+    LSA_OK = 0,
+    LSA_ERR_INVALID_ARG = 1,   /* bad pointer, size, layout or parameter */
+    LSA_ERR_CUDA = 2,          /* a CUDA runtime call failed */
+    LSA_ERR_OOM = 3,           /* device allocation failed; nothing leaked */
+    LSA_ERR_INEXACT = 4,       /* integer-grid mode met a value off its exact range */
+    LSA_ERR_TIMEOUT = 5,       /* reserved: a bounded device wait gave up */
+    LSA_ERR_DEVICE = 6,        /* a kernel met an out-of-range index and skipped it */
+    LSA_ERR_CAPACITY = 7       /* lsa_append found a leaf with no free slot */
+} lsa_status;
+
+typedef enum { LSA_F32 = 0, LSA_BF16 = 1 } lsa_dtype;
+
+#define LSA_MAX_LEVELS 4
+
+/* Index construction parameters.  [p5 "How does LSA work?" step 1: keys are
+ * pooled and clustered into buckets in a learned latent space, organised as a
+ * hierarchy; p2: the hierarchical tree variant.] */
+typedef struct {
+    int64_t batch;          /* sequences (>= 1) */
+    int64_t n_tokens;       /* tokens per sequence to index (>= 1) */
+    int64_t ld_tokens;      /* token capacity per sequence of the K buffer (>= n_tokens) */
+    int32_t hkv;            /* KV heads; every (sequence, KV head) is one unit with its own tree */
+    int32_t d;              /* head dimension: 64 or 128 */
+    int32_t r;              /* latent rank: 16, 32, 64 or 128 */
+    int32_t pool;           /* P keys per pooled block, 1..16 */
+    int32_t dtype;          /* lsa_dtype of K */
+    int32_t levels;         /* tree depth 1..LSA_MAX_LEVELS (1 = flat buckets) */
+    int32_t level_sizes[LSA_MAX_LEVELS]; /* nodes per level, top first, leaves last, non-decreasing */
+    int32_t lloyd_iters;    /* Lloyd rounds per level (>= 1) */
+    int32_t grid_log2;      /* 0: float centroids; g in 1..8: centroids rounded half-to-even
+                               onto multiples of 2^-g (exact integer workloads) */
+    int32_t sink;           /* S: blocks that start before token S are never candidates */
+    int64_t append_capacity;/* tokens per sequence lsa_append may add after the build (>= 0) */
+} lsa_build_params;
+
+/* Selection parameters.  [p5 "How does LSA work?" steps 2-3; p3 TL;DR] */
+typedef struct {
+    int32_t hq;             /* query heads; a multiple of hkv; each KV head's group of
+                               hq/hkv query heads shares one selection (mean latent query) */
+    int32_t beam;           /* B: nodes kept per tree level (1..1024) */
+    int32_t topk;           /* K: long-range budget in tokens; ceil(K/P) blocks are taken */
+    int32_t sink;           /* S: must equal the build's sink */
+    int32_t window;         /* W: causal local window in tokens (>= 1) */
+} lsa_select_params;
+
+/* Host-side description of an index (lsa_index_info). */
+typedef struct {
+    int64_t units;          /* batch * hkv */
+    int64_t n_tokens;       /* tokens indexed so far, per sequence */
+    int64_t n_blocks;       /* complete blocks indexed so far, per unit */
+    int64_t block_capacity; /* blocks per unit the slot arrays can hold */
+    int64_t device_bytes;   /* device memory held by the index */
+    int32_t levels;
+    int32_t level_sizes[LSA_MAX_LEVELS];
+    int32_t r, pool, sink, grid_log2;
+} lsa_index_info_t;
+
+/* What lsa_index_get copies out. */
+typedef enum {
+    LSA_GET_CENTROIDS = 0,     /* float  [units][level_sizes[level]][r] */
+    LSA_GET_PARENT = 1,        /* int32  [units][level_sizes[level]]  (level >= 1) */
+    LSA_GET_LEAF_OF_BLOCK = 2, /* int32  [units][n_blocks] */
+    LSA_GET_MINPOS = 3,        /* int64  [units][level_sizes[level]]  (INT64_MAX = none) */
+    LSA_GET_OBJECTIVE = 4,     /* double [lloyd_iters][units] of that level's k-means */
+    LSA_GET_LATENT = 5,        /* float  [units][n_blocks][r] latent keys in block order */
+    LSA_GET_LEAF_COUNT = 6     /* int32  [units][leaves] blocks per leaf */
+} lsa_get_what;
+
+/* ----------------------------------------------------------------- calls */
+
+/* Build the bucket hierarchy of every (sequence, KV head).
+ *  K: device, [batch][ld_tokens][hkv][d] of dtype; tokens [0, n_tokens) are read.
+ *  W: device, float [d][r], the latent map (row = input dimension).
+ * Steps: latent keys Kl[b] = W^T * mean(K[bP .. bP+P-1]) for every complete
+ * block; Lloyd k-means of the latent keys into level_sizes[levels-1] leaves
+ * (centroid j starts at point floor(j*n/k); ties to the lower id; an empty
+ * cluster keeps its centroid); then k-means of each level's centroids into
+ * the level above.  [p1 "first groups keys into clusters"; p5 step 1; p2]
+ * On success *out receives a new index owned by the caller (lsa_free_index).
+ * On failure *out is set to NULL and no device memory is left allocated.
+ * The build is enqueued on `stream`; lsa_check() reports device-side errors. */
+int lsa_build_index(const lsa_build_params* params, const void* K, const float* W,
+                    void* stream, lsa_index** out);
+
+/* Same index, but with the clustering given instead of computed (for
+ * decoupled checks and for trees made elsewhere).
+ *  leaf_of_block: device int32 [units][n_blocks], leaf id of every block.
+ *  parents[l] for l = 1..levels-1: device int32 [units][level_sizes[l]],
+ *      parent (at level l-1) of every level-l node; parents[0] is ignored.
+ *  centroids[l] for l = 0..levels-1: device float [units][level_sizes[l]][r].
+ * Latent keys are still computed from K and W. */
+int lsa_build_index_from_tree(const lsa_build_params* params, const void* K, const float* W,
+                              const int32_t* leaf_of_block, const int32_t* const* parents,
+                              const float* const* centroids, void* stream, lsa_index** out);
+
+/* Tree-search selection for nq queries per sequence.
+ *  Q: device [batch][nq][hq][d] of the index's dtype.
+ *  q_pos: device int64 [batch][nq] query positions, or NULL for
+ *      position(query j) = q_pos0 + j in every sequence.
+ *  idx: device int32 [batch][nq][hkv][max_sel]; cnt: device int32 [batch][nq][hkv].
+ * For the query at position i and KV head h: latent query = mean over the
+ * group's heads of W^T q; at each level score the eligible nodes (all top
+ * nodes, then the children of the kept ones) by latent dot product and keep the
+ * best `beam`; score the candidate blocks of the kept leaves and keep the best
+ * ceil(K/P).  A block is a candidate iff it starts at or after S and ends at or
+ * before i - W; a node is eligible iff it holds a candidate.  Ties go to the
+ * lower id.  The row of idx lists, ascending, the sink [0, min(S, i+1)), the
+ * tokens of the chosen blocks and the window [max(0, i-W+1), i]; cnt holds its
+ * length and the rest of the row is -1.  max_sel must be at least
+ * ceil(K/P)*P + S + W.  [p3 TL;DR "scores cluster centroids and descends into
+ * the best few buckets"; p1; p5 steps 2-3] */
+int lsa_select(const lsa_index* index, const lsa_select_params* params, const void* Q,
+               int64_t nq, const int64_t* q_pos, int64_t q_pos0,
+               int32_t* idx, int32_t* cnt, int32_t max_sel, void* stream);
+
+/* The quadratic baseline indexer: every candidate block is scored, no tree.
+ * Same arguments and output format as lsa_select (beam is ignored).
+ * [p3 flowchart, red path "Full key scan"] */
+int lsa_fullscan_select(const lsa_index* index, const lsa_select_params* params, const void* Q,
+                        int64_t nq, const int64_t* q_pos, int64_t q_pos0,
+                        int32_t* idx, int32_t* cnt, int32_t max_sel, void* stream);
+
+/* Exact softmax attention over selected tokens.
+ *  Q: device [batch][nq][hq][d]; K, V: device [batch][ld_tokens][hkv][d];
+ *  idx/cnt as written by lsa_select (entries past cnt are ignored).
+ *  O: device [batch][nq][hq][d] of dtype; lse: device float [batch][nq][hq]
+ *  or NULL (natural log of the softmax denominator of the scaled scores).
+ * O[q,h] = sum_j softmax_j(q_h . k_j / sqrt(d)) v_j over the row of KV head
+ * h / (hq/hkv); fp32 accumulation.  A row with cnt = 0 yields O = 0 and
+ * lse = -inf.  An index outside [0, ld_tokens) is skipped and latched as
+ * LSA_ERR_DEVICE.  [p5 step 3 "the attention kernel is unchanged"; p3
+ * flowchart "exact over subset"] */
+int lsa_sparse_attn(const void* Q, const void* K, const void* V, const int32_t* idx,
+                    const int32_t* cnt, int64_t batch, int64_t nq, int32_t hq, int32_t hkv,
+                    int32_t d, int32_t dtype, int32_t max_sel, int64_t ld_tokens,
+                    void* O, float* lse, void* stream);
+
+/* Decode: index tokens [n_tokens, n_tokens + n_new) that the caller has
+ * already written into K (same layout and ld_tokens as the build).  Every
+ * block this completes is pooled, mapped, and placed in its nearest leaf
+ * (squared distance over all leaves, frozen centroids, ties to the lower id)
+ * after that leaf's older blocks; node eligibility is updated.  A leaf with
+ * no free slot latches LSA_ERR_CAPACITY and the block stays unindexed.
+ * [p5 "Prefill, decode and training"; p4 "Prompt processing is not response
+ * generation"] */
+int lsa_append(lsa_index* index, const void* K, int64_t n_new, void* stream);
+
+/* Stage calls, exposed for checks and for callers that compose the path. */
+
+/* Kl[u][b][:] = W^T * mean of the P keys of block b, for every complete block
+ * of tokens [0, n_tokens).  Kl: device float [batch*hkv][n_tokens/P][r]. */
+int lsa_project_pool(const void* K, const float* W, int64_t batch, int64_t n_tokens,
+                     int64_t ld_tokens, int32_t hkv, int32_t d, int32_t r, int32_t pool,
+                     int32_t dtype, float* Kl, void* stream);
+
+/* qbar[b][j][h][:] = mean over the group of KV head h of W^T Q[b][j][g][:].
+ * qbar: device float [batch][nq][hkv][r]. */
+int lsa_query_latent(const void* Q, const float* W, int64_t batch, int64_t nq, int32_t hq,
+                     int32_t hkv, int32_t d, int32_t r, int32_t dtype, float* qbar, void* stream);
+
+/* Lloyd k-means of `units` independent point sets.
+ *  X: device float [units][n][r]; labels: device int32 [units][n];
+ *  C: device float [units][k][r] (output); objective: device double
+ *  [iters][units] (sum of squared distances after each assign) or NULL.
+ * Same rules as the build (stride init, ties low, empty keeps, grid). */
+int lsa_kmeans(const float* X, int64_t units, int64_t n, int32_t r, int32_t k, int32_t iters,
+               int32_t grid_log2, int32_t* labels, float* C, double* objective, void* stream);
+
+/* Copy one array of the index to `dst` (device or host memory, dst_bytes
+ * large enough; see lsa_get_what for shapes).  Synchronises `stream`. */
+int lsa_index_get(const lsa_index* index, int32_t what, int32_t level, void* dst,
+                  int64_t dst_bytes, void* stream);
+
+/* Host-side description; does not touch the device. */
+int lsa_index_info(const lsa_index* index, lsa_index_info_t* out);
+
+/* Synchronise `stream`, then return and clear the first error latched by a
+ * kernel of this index (or of index-free calls when index is NULL). */
+int lsa_check(lsa_index* index, void* stream);
+
+/* Free an index (NULL is a no-op).  A pointer that is not a live index is
+ * detected by its magic word and ignored. */
+void lsa_free_index(lsa_index* index);
+
+/* Static text for a status code. */
+const char* lsa_strerror(int status);
+
+/* Test hook: make the n-th next device allocation of the library fail
+ * (n >= 1), to exercise the LSA_ERR_OOM path; n = 0 disarms it. */
+void lsa_debug_fail_alloc_after(int32_t n);
+
+/* Number of kernels the library has launched in this process (a host-side
+ * counter, incremented at every launch; for accounting in benchmarks). */
+int64_t lsa_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LSA_H_ */

@@ -1,0 +1,68 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every function include/lsa.h declares, and the binding's structs match the C
+layout (compiled here with gcc)."""
+import ctypes as C
+import os
+import subprocess
+import tempfile
+
+import pytest
+
+from hierarchical_latent_key_gemm_b200 import lsa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "lsa.h")
+
+
+def test_library_exports_every_declared_symbol():
+    L = lsa.lib()
+    names = lsa.exported_symbols_from_header(HEADER)
+    assert len(names) >= 15
+    missing = [n for n in names if not hasattr(L, n)]
+    assert not missing, missing
+    # the binding declares a signature for each of them
+    assert sorted(names) == sorted(lsa._SIGS)
+
+
+def test_status_strings_and_null_handles():
+    for s in range(8):
+        assert lsa.strerror(s) and lsa.strerror(s) != "unknown status"
+    assert lsa.strerror(99) == "unknown status"
+    L = lsa.lib()
+    info = lsa.IndexInfo()
+    assert L.lsa_index_info(None, C.byref(info)) == lsa.LSA_ERR_INVALID_ARG
+    L.lsa_free_index(None)  # no-op
+    bogus = C.c_void_p(0x1234)
+    L.lsa_free_index(bogus)  # not a live index: ignored, never dereferenced
+    assert L.lsa_index_info(bogus, C.byref(info)) == lsa.LSA_ERR_INVALID_ARG
+
+
+def test_struct_layout_matches_c_header():
+    src = r'''
+#include <stddef.h>
+#include <stdio.h>
+#include "lsa.h"
+int main(void) {
+  printf("%zu %zu %zu %zu %zu\n", sizeof(lsa_build_params), offsetof(lsa_build_params, level_sizes),
+         offsetof(lsa_build_params, append_capacity), sizeof(lsa_select_params), sizeof(lsa_index_info_t));
+  printf("%zu %zu\n", offsetof(lsa_index_info_t, level_sizes), offsetof(lsa_index_info_t, grid_log2));
+  return 0;
+}
+'''
+    with tempfile.TemporaryDirectory() as td:
+        c = os.path.join(td, "t.c")
+        exe = os.path.join(td, "t")
+        open(c, "w").write(src)
+        subprocess.run(["gcc", "-I", os.path.dirname(HEADER), c, "-o", exe], check=True)
+        out = subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split()
+    got = [int(x) for x in out]
+    want = [C.sizeof(lsa.BuildParams), lsa.BuildParams.level_sizes.offset, lsa.BuildParams.append_capacity.offset,
+            C.sizeof(lsa.SelectParams), C.sizeof(lsa.IndexInfo), lsa.IndexInfo.level_sizes.offset,
+            lsa.IndexInfo.grid_log2.offset]
+    assert got == want
+
+
+def test_binding_rejects_host_tensors():
+    import torch
+    with pytest.raises(ValueError):
+        lsa._ptr(torch.zeros(4))
