@@ -122,13 +122,36 @@ int check_build_params(const lsa_build_params* p) {
     return LSA_OK;
 }
 
+// The library allocates from the device's default stream-ordered pool.  Freed
+// blocks stay cached in the pool (up to 16 GiB) so that rebuilding an index of
+// the same shape does not go back to the driver.  This is a setting of this
+// process's pool, not of the GPU.
+void keep_pool_memory() {
+    static std::mutex mu;
+    static bool done[128] = {false};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128) return;
+    std::lock_guard<std::mutex> lk(mu);
+    if (done[dev]) return;
+    cudaMemPool_t pool;
+    if (cudaDeviceGetDefaultMemPool(&pool, dev) == cudaSuccess) {
+        uint64_t thr = uint64_t(16) << 30;
+        cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &thr);
+    }
+    cudaGetLastError();
+    done[dev] = true;
+}
+
 // Allocates every persistent array of an index (no kernel launched).
 int alloc_index(const lsa_build_params* p, const float* W, cudaStream_t s, lsa_index** out) {
+    keep_pool_memory();
     lsa_index* ix = new (std::nothrow) lsa_index();
     if (!ix) return LSA_ERR_OOM;
     std::memset(ix, 0, sizeof(*ix));
     ix->mem = new (std::nothrow) Arena();
     if (!ix->mem) { delete ix; return LSA_ERR_OOM; }
+    ix->mem->async = true;
+    ix->mem->stream = s;
     ix->p = *p;
     cudaGetDevice(&ix->device);
     ix->units = p->batch * p->hkv;
@@ -193,7 +216,10 @@ void destroy_index(lsa_index* ix) {
     }
     ix->magic = kFreedMagic;
     if (ix->mem) {
+        // the caller's streams may still use the index: wait for them, then
+        // return the memory to the pool on the legacy stream
         cudaDeviceSynchronize();
+        ix->mem->stream = nullptr;
         ix->mem->release();
         delete ix->mem;
     }
@@ -314,6 +340,7 @@ int do_select(const lsa_index* ix, const lsa_select_params* sp, const void* Q, i
     if (st != LSA_OK || nq == 0) return st;
     cudaStream_t s = as_stream(stream);
     const lsa_build_params& p = ix->p;
+    keep_pool_memory();
     Arena scratch;
     scratch.async = true;
     scratch.stream = s;

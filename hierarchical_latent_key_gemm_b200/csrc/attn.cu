@@ -8,7 +8,8 @@
 //
 // bf16 path: the G heads (zero-padded to 16) are the M side of
 // mma.sync.m16n8k16 tiles; S = Q K^T over 16-key slices, online softmax in
-// fp32 registers, O += P V with P reused from the S accumulators.  K/V rows
+// fp32 registers, O += P V with P reused from the S accumulators (P split
+// into two bf16 terms so the weights keep about 16 significant bits).  K/V rows
 // are gathered with 16-byte cp.async into an XOR-swizzled 3-stage ring of
 // 64-key tiles; each of the 4 warps owns 16 keys of every tile and the warps'
 // partial (max, sum, O) are merged at the end.
@@ -50,9 +51,14 @@ __device__ __forceinline__ void mma_bf16(float* c, const uint32_t* a, uint32_t b
         : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
+
+// Two bf16 pairs whose sum carries a/b to about 16 significant bits.
+__device__ __forceinline__ void split_pack(float a, float b, uint32_t& hi, uint32_t& lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(a - hf.x, b - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
 // byte offset of 16-byte chunk c of row r in a swizzled [rows][D] bf16 tile
@@ -198,11 +204,12 @@ __global__ __launch_bounds__(kAttThreads) void attn_bf16_kernel(
             o[i][0] *= al0; o[i][1] *= al0;
             o[i][2] *= al1; o[i][3] *= al1;
         }
-        uint32_t pa[4];
-        pa[0] = pack_bf16(p[0][0], p[0][1]);
-        pa[1] = pack_bf16(p[0][2], p[0][3]);
-        pa[2] = pack_bf16(p[1][0], p[1][1]);
-        pa[3] = pack_bf16(p[1][2], p[1][3]);
+        // P = hi + lo, both bf16: the weights keep ~16 significant bits
+        uint32_t pa[4], pl[4];
+        split_pack(p[0][0], p[0][1], pa[0], pl[0]);
+        split_pack(p[0][2], p[0][3], pa[1], pl[1]);
+        split_pack(p[1][0], p[1][1], pa[2], pl[2]);
+        split_pack(p[1][2], p[1][3], pa[3], pl[3]);
         // O += P V
         {
             const int vr = key0 + (lane & 7) + 8 * ((lane >> 3) & 1);
@@ -213,6 +220,8 @@ __global__ __launch_bounds__(kAttThreads) void attn_bf16_kernel(
                 ldsm_x4_t(vb + swz<D>(vr, c), b0, b1, b2, b3);
                 mma_bf16(o[nt], pa, b0, b1);
                 mma_bf16(o[nt + 1], pa, b2, b3);
+                mma_bf16(o[nt], pl, b0, b1);
+                mma_bf16(o[nt + 1], pl, b2, b3);
             }
         }
     }

@@ -21,7 +21,6 @@ Workload shapes (one attention layer each):
 from __future__ import annotations
 
 import dataclasses
-import math
 from dataclasses import dataclass
 
 import torch
@@ -122,8 +121,8 @@ def make_map(w: Workload, seed: int = 0, device="cpu") -> torch.Tensor:
     else:
         A = torch.randn(w.d, w.r, generator=g, dtype=torch.float64)
         Qm, Rm = torch.linalg.qr(A)
-        Wm = (Qm * torch.sign(torch.diagonal(Rm))[None, :]).to(torch.float32)
-    return Wm.to(device)
+        Wm = (Qm * torch.sign(torch.diagonal(Rm))[None, :]).to(torch.float32).contiguous()
+    return Wm.contiguous().to(device)
 
 
 def _segment_weights(w: Workload, n: int, seed: int, device) -> torch.Tensor | None:
@@ -264,4 +263,3 @@ def _fanouts(sizes):
 
 
 __all__ = ["Workload", "WORKLOADS", "make_inputs", "make_map", "input_bytes", "describe", "torch_dtype"]
-_ = math

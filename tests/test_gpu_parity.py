@@ -314,17 +314,19 @@ def _attn_case(w, seed, rows):
     _assert_clean()
     Kn = inp["K"][0].float().numpy().astype(np.float64)
     Vn = inp["V"][0].float().numpy().astype(np.float64)
-    errs, lerr = [], []
+    errs, lerr, ulps = [], [], []
     for h in range(w.hkv):
         for k, i in enumerate(rows):
             q = TU.unit_queries(inp["Q"], 0, h, G, [i])[0]
             o, l = O.sparse_attention(q, Kn[:, h], Vn[:, h], sels_all[h][k])
             got = O_[0, k, h * G:(h + 1) * G].double().cpu().numpy()
             errs.append(np.abs(got - o))
+            # one bf16 ulp of the oracle value: 2^(floor(log2|o|) - 7)
+            ulps.append(np.exp2(np.floor(np.log2(np.maximum(np.abs(o), 1e-30))) - 7))
             lerr.append(np.abs(lse[0, k, h * G:(h + 1) * G].double().cpu().numpy() - l))
     e = np.concatenate([x.ravel() for x in errs])
     le = np.concatenate(lerr)
-    return e, le
+    return e, le, np.concatenate([x.ravel() for x in ulps])
 
 
 @pytest.mark.parametrize("name,over", [
@@ -339,9 +341,15 @@ def test_attention_on_oracle_index_sets(name, over):
     rng = np.random.default_rng(5)
     rows = np.unique(np.concatenate([[0, 1, 2, w.sink + w.window + w.pool], rng.integers(0, w.n_tokens, 120),
                                      [w.n_tokens - 1]]))
-    e, le = _attn_case(w, 5, rows)
+    e, le, ulp = _attn_case(w, 5, rows)
     if w.dtype == "f32":
         assert e.max() <= 1e-4 and le.max() <= 1e-4
+    elif w.kind == "int":
+        # |O| reaches 4 here, so the bf16 output rounding alone exceeds the
+        # float workloads' mean-abs bound: compare within one bf16 ulp of the
+        # oracle value (plus fp32 accumulation slack) instead
+        assert np.all(e <= ulp + 1e-3) and e.max() <= BF16_MAX_ABS
+        assert le.max() <= 1e-2
     else:
         assert e.max() <= BF16_MAX_ABS and e.mean() <= BF16_MEAN_ABS
         assert le.max() <= 1e-2
@@ -443,17 +451,22 @@ def test_edge_cases_and_errors():
     assert lsa.lsa_check(None) == lsa.LSA_ERR_DEVICE
     assert torch.isfinite(O_.float()).all()
     assert lsa.lsa_check(None) == lsa.LSA_OK
-    # allocation failure: reported, nothing leaked
-    torch.cuda.synchronize()
-    free0 = torch.cuda.mem_get_info()[0]
-    for n in (1, 3, 9, 21, 30, 40, 46):
-        lsa.lsa_debug_fail_alloc_after(n)
-        with pytest.raises(lsa.LsaError) as ei:
-            lsa.lsa_build_index(TU.build_params(w), d["K"], d["W"])
-        assert ei.value.status == lsa.LSA_ERR_OOM
-    lsa.lsa_debug_fail_alloc_after(0)
-    torch.cuda.synchronize()
-    assert abs(torch.cuda.mem_get_info()[0] - free0) < (64 << 20)
+    # allocation failure: reported, and nothing leaked (repeating the failing
+    # builds does not lower free memory; freed blocks stay in the pool)
+    frees = []
+    for _ in range(3):
+        for n in (1, 3, 9, 21, 30, 40, 46):
+            lsa.lsa_debug_fail_alloc_after(n)
+            with pytest.raises(lsa.LsaError) as ei:
+                lsa.lsa_build_index(TU.build_params(w), d["K"], d["W"])
+            assert ei.value.status == lsa.LSA_ERR_OOM
+        lsa.lsa_debug_fail_alloc_after(0)
+        torch.cuda.synchronize()
+        frees.append(torch.cuda.mem_get_info()[0])
+    assert abs(frees[2] - frees[1]) < (16 << 20)
+    ok = lsa.lsa_build_index(TU.build_params(w), d["K"], d["W"])
+    assert lsa.lsa_check(ok) == lsa.LSA_OK
+    ok.free()
     # double free is harmless
     h = ix.handle
     ix.free()
