@@ -565,3 +565,52 @@ void lsa_debug_fail_alloc_after(int32_t n) { g_fail_after.store(n > 0 ? n : 0); 
 int64_t lsa_launch_count(void) { return g_launches.load(); }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free selection.  The scratch of lsa_select (the latent queries)
+// lives in a fixed device array here, for callers that cannot allocate while
+// they serve.  In host code g_noalloc_qbar only stands in for the device
+// variable: kernels receive the address cudaGetSymbolAddress returns for the
+// current device.
+namespace {
+
+static __device__ __align__(256) float g_noalloc_qbar[LSA_SELECT_NOALLOC_MAX_FLOATS];
+
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[128] = {nullptr};
+
+// Device address of g_noalloc_qbar on the current device, looked up once per
+// device with that device current.
+int noalloc_scratch(float** out) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_status(e);
+    if (dev < 0 || dev >= 128) return LSA_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_noalloc_mu);
+    if (!g_noalloc_ptr[dev]) {
+        void* p = nullptr;
+        e = cudaGetSymbolAddress(&p, g_noalloc_qbar);
+        if (e != cudaSuccess) return cuda_status(e);
+        g_noalloc_ptr[dev] = static_cast<float*>(p);
+    }
+    *out = g_noalloc_ptr[dev];
+    return LSA_OK;
+}
+
+}  // namespace
+
+extern "C" int lsa_select_noalloc(const lsa_index* index, const lsa_select_params* params, const void* Q,
+                                  int64_t nq, const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt,
+                                  int32_t max_sel, void* stream) {
+    int st = check_select(index, params, Q, nq, q_pos, q_pos0, idx, cnt, max_sel);
+    if (st != LSA_OK || nq == 0) return st;
+    const lsa_build_params& p = index->p;
+    if (p.batch * nq * p.hkv * (int64_t)p.r > LSA_SELECT_NOALLOC_MAX_FLOATS) return LSA_ERR_INVALID_ARG;
+    float* qbar = nullptr;
+    st = noalloc_scratch(&qbar);
+    if (st != LSA_OK) return st;
+    cudaStream_t s = as_stream(stream);
+    st = launch_query_latent(Q, index->W, p.batch, nq, params->hq, p.hkv, p.d, p.r, p.dtype, qbar, s);
+    if (st == LSA_OK) st = launch_select(index, params, qbar, nq, q_pos, q_pos0, idx, cnt, max_sel, false, s);
+    return st;
+}

@@ -57,6 +57,7 @@ _SIGS = {
                                          _vp, C.POINTER(_vp)]),
     "lsa_select": (_i32, [_vp, C.POINTER(SelectParams), _vp, _i64, _vp, _i64, _vp, _vp, _i32, _vp]),
     "lsa_fullscan_select": (_i32, [_vp, C.POINTER(SelectParams), _vp, _i64, _vp, _i64, _vp, _vp, _i32, _vp]),
+    "lsa_select_noalloc": (_i32, [_vp, C.POINTER(SelectParams), _vp, _i64, _vp, _i64, _vp, _vp, _i32, _vp]),
     "lsa_sparse_attn": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _i64, _vp, _vp,
                                _vp]),
     "lsa_append": (_i32, [_vp, _vp, _i64, _vp]),
@@ -227,6 +228,24 @@ def _select(fn, name, index, sp, Q, q_pos=None, q_pos0=0, idx=None, cnt=None, ma
 
 def lsa_select(index, sp, Q, **kw):
     return _select(lib().lsa_select, "lsa_select", index, sp, Q, **kw)
+
+
+LSA_SELECT_NOALLOC_MAX_FLOATS = 1 << 20
+
+
+def lsa_select_noalloc(index, sp, Q, idx, cnt, q_pos=None, q_pos0=0, stream=None):
+    """Allocation-free selection: the caller passes idx and cnt, and the latent
+    queries use the library's fixed 4 MiB device buffer (see include/lsa.h).
+    batch * nq * hkv * r must not exceed LSA_SELECT_NOALLOC_MAX_FLOATS."""
+    p = index.params
+    need = Q.shape[0] * Q.shape[1] * p.hkv * p.r
+    if need > LSA_SELECT_NOALLOC_MAX_FLOATS:
+        raise ValueError(f"lsa_select_noalloc: {need} latent-query floats exceed the fixed buffer of "
+                         f"{LSA_SELECT_NOALLOC_MAX_FLOATS}; select in smaller query chunks")
+    st = lib().lsa_select_noalloc(index.handle, C.byref(sp), _ptr(Q), int(Q.shape[1]), _ptr(q_pos), int(q_pos0),
+                                  _ptr(idx), _ptr(cnt), int(idx.shape[-1]), _stream(stream))
+    _ok(st, "lsa_select_noalloc")
+    return idx, cnt
 
 
 def lsa_fullscan_select(index, sp, Q, **kw):

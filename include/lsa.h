@@ -163,6 +163,33 @@ int lsa_select(const lsa_index* index, const lsa_select_params* params, const vo
                int64_t nq, const int64_t* q_pos, int64_t q_pos0,
                int32_t* idx, int32_t* cnt, int32_t max_sel, void* stream);
 
+/* Allocation-free form of lsa_select.  The pages have no counterpart: this
+ * is a deployment aid.  lsa_select takes its scratch (the latent queries,
+ * batch*nq*hkv*r floats) from the device's stream-ordered pool.  Some callers
+ * cannot allocate device memory while they serve: a framework whose caching
+ * allocator already owns the device's memory, a decode loop that must never
+ * stall on an allocation or trigger a pool trim, a process that fixes its
+ * memory budget before it starts serving.  This call instead uses one fixed
+ * buffer of LSA_SELECT_NOALLOC_MAX_FLOATS floats (4 MiB), declared by the
+ * library as a device variable; every GPU that loads the library holds those
+ * 4 MiB until the process exits.
+ *  - Arguments, results and errors are those of lsa_select.
+ *  - batch*nq*hkv*r above LSA_SELECT_NOALLOC_MAX_FLOATS returns
+ *    LSA_ERR_INVALID_ARG before anything is enqueued (split the queries into
+ *    chunks and pass q_pos0 per chunk).
+ *  - It calls no cudaMalloc, cudaFree or other allocating routine.
+ *  - Its first call on a device looks up the buffer's device address, once
+ *    per device, with that device current; make that first call before any
+ *    stream capture.
+ *  - Every call shares the one buffer and it keeps the last call's contents.
+ *    Each call rewrites all of the part it reads, so nothing needs clearing,
+ *    but calls whose GPU work can overlap (e.g. two streams with no ordering
+ *    between them) race on the buffer and must not be issued that way. */
+#define LSA_SELECT_NOALLOC_MAX_FLOATS 1048576
+int lsa_select_noalloc(const lsa_index* index, const lsa_select_params* params, const void* Q,
+                       int64_t nq, const int64_t* q_pos, int64_t q_pos0,
+                       int32_t* idx, int32_t* cnt, int32_t max_sel, void* stream);
+
 /* The quadratic baseline indexer: every candidate block is scored, no tree.
  * Same arguments and output format as lsa_select (beam is ignored).
  * [p3 flowchart, red path "Full key scan"] */
