@@ -103,30 +103,45 @@ __global__ __launch_bounds__(kAttThreads) void attn_bf16_kernel(
     }
 
     const int ntile = (n + kTileKeys - 1) / kTileKeys;
-    auto load_tile = [&](int t) {
+    // Each thread gathers the same 16-byte column c of RPT rows of every tile;
+    // its token ids are read one tile ahead into registers, so the gathers
+    // never wait on an index load.
+    constexpr int RPT = kTileKeys * CH / kAttThreads;
+    constexpr int ROW_STEP = kAttThreads / CH;
+    const int c_col = tid % CH, r_base = tid / CH;
+    auto fetch_tokens = [&](int t, int* tk) {
+#pragma unroll
+        for (int k = 0; k < RPT; ++k) {
+            const int j = t * kTileKeys + r_base + ROW_STEP * k;
+            tk[k] = (t < ntile && j < n) ? __ldg(ir + j) : -1;
+        }
+    };
+    const __nv_bfloat16* kcol = K + (b * ld_tokens * hkv + h) * D + c_col * 8;
+    const __nv_bfloat16* vcol = V + (b * ld_tokens * hkv + h) * D + c_col * 8;
+    auto load_tile = [&](int t, const int* tk) {
         const int st = t % kStages;
         const uint32_t kb = smem_u32(Ks + st * TILE_BYTES), vb = smem_u32(Vs + st * TILE_BYTES);
-        for (int e = tid; e < kTileKeys * CH; e += kAttThreads) {
-            const int r = e / CH, c = e % CH;
-            const int j = t * kTileKeys + r;
-            int tok = -1;
-            if (j < n) {
-                tok = ir[j];
-                if (tok < 0 || tok >= ld_tokens) { latch(err, kErrDevice); tok = -1; }
-            }
-            const int64_t off = tok >= 0 ? (((b * ld_tokens + tok) * hkv + h) * D + c * 8) : 0;
+#pragma unroll
+        for (int k = 0; k < RPT; ++k) {
+            const int r = r_base + ROW_STEP * k;
+            int tok = tk[k];
+            if (tok >= ld_tokens || tok < -1) { latch(err, kErrDevice); tok = -1; }
+            const int64_t off = tok >= 0 ? (int64_t)tok * hkv * D : 0;
             const int bytes = tok >= 0 ? 16 : 0;
-            cp_async16(kb + swz<D>(r, c), K + off, bytes);
-            cp_async16(vb + swz<D>(r, c), V + off, bytes);
-            if (c == 0) toks[st * kTileKeys + r] = tok;
+            cp_async16(kb + swz<D>(r, c_col), kcol + off, bytes);
+            cp_async16(vb + swz<D>(r, c_col), vcol + off, bytes);
+            if (c_col == 0) toks[st * kTileKeys + r] = tok;
         }
     };
 
+    int tk_next[RPT];
 #pragma unroll
     for (int t = 0; t < kStages - 1; ++t) {
-        if (t < ntile) load_tile(t);
+        fetch_tokens(t, tk_next);
+        if (t < ntile) load_tile(t, tk_next);
         cp_async_commit();
     }
+    fetch_tokens(kStages - 1, tk_next);
     __syncthreads();
 
     // Q fragments for every 16-wide k step
@@ -149,8 +164,9 @@ __global__ __launch_bounds__(kAttThreads) void attn_bf16_kernel(
     for (int t = 0; t < ntile; ++t) {
         cp_async_wait<kStages - 2>();
         __syncthreads();
-        if (t + kStages - 1 < ntile) load_tile(t + kStages - 1);
+        if (t + kStages - 1 < ntile) load_tile(t + kStages - 1, tk_next);
         cp_async_commit();
+        fetch_tokens(t + kStages, tk_next);
         const int st = t % kStages;
         const uint32_t kb = smem_u32(Ks + st * TILE_BYTES), vb = smem_u32(Vs + st * TILE_BYTES);
         const int key0 = warp * 16;  // this warp's 16 keys within the tile
