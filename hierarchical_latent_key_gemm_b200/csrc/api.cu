@@ -178,9 +178,14 @@ int alloc_index(const lsa_build_params* p, const float* W, cudaStream_t s, lsa_i
         ix->minpos[l] = A.alloc<int64_t>(U * nl);
         ix->parent[l] = A.alloc<int32_t>(U * nl);
         ix->objective[l] = A.alloc<double>((int64_t)p->lloyd_iters * U);
+        ix->ord_id[l] = A.alloc<int32_t>(U * nl);
+        ix->ord_pos[l] = A.alloc<int32_t>(U * nl);
+        ix->ord_cent[l] = A.alloc<float>(U * nl * r);
+        ix->ord_mp[l] = A.alloc<int64_t>(U * nl);
         if (l + 1 < p->levels) {
             ix->child_off[l] = A.alloc<int32_t>(U * nl + 1);
             ix->child_ids[l] = A.alloc<int32_t>(U * (int64_t)p->level_sizes[l + 1]);
+            ix->ord_coff[l] = A.alloc<int32_t>(U * nl + 1);
         }
     }
     ix->err = A.alloc<int32_t>(1);

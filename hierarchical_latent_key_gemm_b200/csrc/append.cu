@@ -27,6 +27,8 @@ struct AppArgs {
     int32_t* leaf_of_block;
     const float* cent_leaf;
     int64_t* minpos[LSA_MAX_LEVELS];
+    int64_t* ord_mp[LSA_MAX_LEVELS];
+    const int32_t* ord_pos[LSA_MAX_LEVELS];
     const int32_t* parent[LSA_MAX_LEVELS];
     int n_l[LSA_MAX_LEVELS];
     int levels, L, d, r, pool, sink, hkv, grid_log2;
@@ -117,6 +119,8 @@ __global__ __launch_bounds__(kAppThreads) void append_kernel(const T* __restrict
                     for (int l = a.levels - 1; l >= 0; --l) {
                         int64_t* mp = a.minpos[l] + (int64_t)u * a.n_l[l] + node;
                         if (start < *mp) *mp = start;
+                        int64_t* omp = a.ord_mp[l] + (int64_t)u * a.n_l[l] + a.ord_pos[l][(int64_t)u * a.n_l[l] + node];
+                        if (start < *omp) *omp = start;
                         if (l > 0) node = a.parent[l][(int64_t)u * a.n_l[l] + node];
                     }
                 }
@@ -150,6 +154,8 @@ int launch_append(lsa_index* ix, const void* K, int64_t first_block, int64_t n_n
     a.cent_leaf = ix->cent[p.levels - 1];
     for (int l = 0; l < p.levels; ++l) {
         a.minpos[l] = ix->minpos[l];
+        a.ord_mp[l] = ix->ord_mp[l];
+        a.ord_pos[l] = ix->ord_pos[l];
         a.parent[l] = ix->parent[l];
         a.n_l[l] = p.level_sizes[l];
     }

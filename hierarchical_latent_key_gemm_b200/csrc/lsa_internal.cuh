@@ -89,6 +89,13 @@ struct lsa_index {
     int32_t* child_off[LSA_MAX_LEVELS];  // [units*n_l + 1] into child_ids (l < levels-1)
     int32_t* child_ids[LSA_MAX_LEVELS];  // [units*n_{l+1}] child id within the unit
     double* objective[LSA_MAX_LEVELS];   // [iters][units]
+    // The same levels in tree order (children of a node contiguous), the
+    // layout the selection reads.  Position q of level l holds node ord_id[q].
+    int32_t* ord_id[LSA_MAX_LEVELS];     // [units*n_l] node id at each position
+    int32_t* ord_pos[LSA_MAX_LEVELS];    // [units*n_l] position of each node id
+    float* ord_cent[LSA_MAX_LEVELS];     // [units*n_l][r]
+    int64_t* ord_mp[LSA_MAX_LEVELS];     // [units*n_l] minpos by position
+    int32_t* ord_coff[LSA_MAX_LEVELS];   // [units*n_l + 1] global child positions (l < levels-1)
     int32_t* err;          // latched kernel error bits
     lsa::Arena* mem;       // owns every device allocation above
 };

@@ -11,27 +11,28 @@
 // Full scan (the "old indexer" of the wiki note's flowchart): the same top-K
 // over every candidate block, no tree.
 //
-// One CTA per (query, KV head).  Candidates stream through a shared-memory
-// buffer: scores are appended, and whenever the buffer holds more than k
-// items a block-wide radix select (on the order-preserving bit pattern of the
-// fp32 score, then on the id for ties) compacts it to the top k.  Order is
-// total: (score desc, id asc), so the result does not depend on the order in
-// which warps append.  Each score is a fp32 dot product of the fp32 latent
-// query with an fp32 latent row: sub-warp groups of r/8 lanes load one row
-// with two 16-byte loads per lane and reduce by xor shuffles.
+// One CTA per (query, KV head).  Every tree level is stored in tree order
+// (children of a node are contiguous), so a candidate's minpos, original id
+// and centroid row are independent loads; each sub-warp group of r/8 lanes
+// issues the loads of several candidates before it uses any of them.  Scores
+// stream through a shared-memory buffer; whenever it holds more than k items a
+// block-wide radix select (on the order-preserving bit pattern of the fp32
+// score, then on the original id for ties) compacts it to the top k.  The
+// order is total, (score desc, id asc), so the result does not depend on the
+// order in which warps append.
 #include "lsa_internal.cuh"
 
 namespace lsa {
 namespace {
 
 constexpr int kSelThreads = 128;
-constexpr int kMaxBeam = 1024;
+constexpr int kUnroll = 4;
 
 struct SelArgs {
-    const float* cent[LSA_MAX_LEVELS];
-    const int64_t* minpos[LSA_MAX_LEVELS];
-    const int32_t* child_off[LSA_MAX_LEVELS];
-    const int32_t* child_ids[LSA_MAX_LEVELS];
+    const float* ocent[LSA_MAX_LEVELS];     // [units*n_l][r], tree order
+    const int64_t* omp[LSA_MAX_LEVELS];     // [units*n_l] minpos, tree order
+    const int32_t* oid[LSA_MAX_LEVELS];     // [units*n_l] original id of each position
+    const int32_t* ocoff[LSA_MAX_LEVELS];   // [units*n_l + 1] child position ranges (global)
     int n_l[LSA_MAX_LEVELS];
     int levels;
     const float* Klp;
@@ -57,9 +58,6 @@ struct SelShared {
     int count;
     int count2;
     int nkept;
-    int kk[kMaxBeam];
-    int pre[kMaxBeam + 1];
-    int lo[kMaxBeam];
 };
 
 // Order-preserving map of a float onto uint32 (-0 and +0 map together).
@@ -72,7 +70,7 @@ __device__ __forceinline__ int warp_incl_scan(int v) {
     const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-        int t = __shfl_up_sync(0xffffffffu, v, o);
+        const int t = __shfl_up_sync(0xffffffffu, v, o);
         if (lane >= o) v += t;
     }
     return v;
@@ -80,15 +78,15 @@ __device__ __forceinline__ int warp_incl_scan(int v) {
 
 // k-th largest key among n items (1 <= k <= n).  mode 0: key = fkey(score);
 // mode 1: key = ~id, restricted to items with fkey(score) == tkey.
-// Returns the key; *need = how many items equal to it are in the top k,
-// *eq = how many items equal it.
+// Precondition: sh.hist is all zero; it is left all zero.  Two barriers per
+// 8-bit pass.  Returns the key; *need = how many items equal to it belong to
+// the top k, *eq = how many items equal it.  Also clears sh.count2.
 __device__ uint32_t block_kth(const float* s, const int* id, int n, int k, int mode, uint32_t tkey,
                               SelShared& sh, int* need, int* eq) {
     uint32_t prefix = 0, pmask = 0;
     int kk = k, eqc = 0;
+#pragma unroll 1
     for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int b = threadIdx.x; b < 256; b += blockDim.x) sh.hist[b] = 0;
-        __syncthreads();
         for (int i = threadIdx.x; i < n; i += blockDim.x) {
             uint32_t key;
             bool act;
@@ -108,6 +106,7 @@ __device__ uint32_t block_kth(const float* s, const int* id, int n, int k, int m
 #pragma unroll
             for (int t = 0; t < 8; ++t) {
                 c[t] = sh.hist[255 - lane * 8 - t];
+                sh.hist[255 - lane * 8 - t] = 0;
                 sum += c[t];
             }
             const int incl = warp_incl_scan(sum);
@@ -125,22 +124,22 @@ __device__ uint32_t block_kth(const float* s, const int* id, int n, int k, int m
                     run += c[t];
                 }
             }
+            if (lane == 0 && shift == 0) sh.count2 = 0;
         }
         __syncthreads();
-        const int dg = sh.bc[0];
+        prefix |= (uint32_t)sh.bc[0] << shift;
+        pmask |= 255u << shift;
         kk = sh.bc[1];
         eqc = sh.bc[2];
-        prefix |= (uint32_t)dg << shift;
-        pmask |= 255u << shift;
-        __syncthreads();
     }
     *need = kk;
     *eq = eqc;
     return prefix;
 }
 
-// Keep the top k of the n items in (s, id); result in (ds, di)[0..k).
-__device__ void topk_compact(const float* s, const int* id, int n, int k, float* ds, int* di, SelShared& sh) {
+// Keep the top k of the n items in (s, id, ps); result in (ds, di, dp)[0..k).
+__device__ void topk_compact(const float* s, const int* id, const int* ps, int n, int k, float* ds, int* di,
+                             int* dp, SelShared& sh) {
     int need, eq;
     const uint32_t T = block_kth(s, id, n, k, 0, 0u, sh, &need, &eq);
     const bool split = need < eq;
@@ -149,8 +148,6 @@ __device__ void topk_compact(const float* s, const int* id, int n, int k, float*
         int need2, eq2;
         T2 = block_kth(s, id, n, need, 1, T, sh, &need2, &eq2);
     }
-    if (threadIdx.x == 0) sh.count2 = 0;
-    __syncthreads();
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
         const uint32_t key = fkey(s[i]);
         const bool take = key > T || (key == T && (!split || ~(uint32_t)id[i] >= T2));
@@ -158,33 +155,34 @@ __device__ void topk_compact(const float* s, const int* id, int n, int k, float*
             const int p = atomicAdd(&sh.count2, 1);
             ds[p] = s[i];
             di[p] = id[i];
+            dp[p] = ps[i];
         }
     }
     __syncthreads();
 }
 
-// Exclusive scan of sh.pre[0..n) in place (values are counts), sh.pre[n] = total.
-__device__ void scan_pre(SelShared& sh, int n) {
+// Exclusive scan of pre[0..n) in place (values are counts), pre[n] = total.
+__device__ void scan_pre(int* pre, int n) {
     __syncthreads();
     if (threadIdx.x < 32) {
         const int lane = threadIdx.x;
         int carry = 0;
         for (int base = 0; base < n; base += 32) {
-            const int v = (base + lane < n) ? sh.pre[base + lane] : 0;
+            const int v = (base + lane < n) ? pre[base + lane] : 0;
             const int incl = warp_incl_scan(v);
-            if (base + lane < n) sh.pre[base + lane] = carry + incl - v;
+            if (base + lane < n) pre[base + lane] = carry + incl - v;
             carry += __shfl_sync(0xffffffffu, incl, 31);
         }
-        if (lane == 0) sh.pre[n] = carry;
+        if (lane == 0) pre[n] = carry;
     }
     __syncthreads();
 }
 
-__device__ __forceinline__ int find_owner(const SelShared& sh, int nk, int t) {
-    int lo = 0, hi = nk;  // sh.pre[lo] <= t < sh.pre[hi]
+__device__ __forceinline__ int find_owner(const int* pre, int nk, int t) {
+    int lo = 0, hi = nk;  // pre[lo] <= t < pre[hi]
     while (hi - lo > 1) {
         const int mid = (lo + hi) >> 1;
-        if (sh.pre[mid] <= t) lo = mid; else hi = mid;
+        if (pre[mid] <= t) lo = mid; else hi = mid;
     }
     return lo;
 }
@@ -195,10 +193,16 @@ __global__ __launch_bounds__(kSelThreads) void select_kernel(const SelArgs a) {
     __shared__ SelShared sh;
     float* bsb[2];
     int* bib[2];
+    int* bpb[2];
     bsb[0] = reinterpret_cast<float*>(dyn4);
     bib[0] = reinterpret_cast<int*>(bsb[0] + a.cap);
-    bsb[1] = reinterpret_cast<float*>(bib[0] + a.cap);
+    bpb[0] = bib[0] + a.cap;
+    bsb[1] = reinterpret_cast<float*>(bpb[0] + a.cap);
     bib[1] = reinterpret_cast<int*>(bsb[1] + a.cap);
+    bpb[1] = bib[1] + a.cap;
+    int* kk = bpb[1] + a.cap;        // kept positions [beam]
+    int* pre = kk + a.beam;          // [beam + 1]
+    int* lo = pre + a.beam + 1;      // [beam]
 
     constexpr int LPC = R / 8;              // lanes per candidate row
     constexpr int CPW = 32 / LPC;           // candidates per warp
@@ -224,9 +228,7 @@ __global__ __launch_bounds__(kSelThreads) void select_kernel(const SelArgs a) {
         qv[0] = x0.x; qv[1] = x0.y; qv[2] = x0.z; qv[3] = x0.w;
         qv[4] = x1.x; qv[5] = x1.y; qv[6] = x1.z; qv[7] = x1.w;
     }
-    auto dot = [&](const float* p) -> float {
-        const float4* v = reinterpret_cast<const float4*>(p + gl * 8);
-        const float4 y0 = __ldg(v), y1 = __ldg(v + 1);
+    auto dot = [&](const float4& y0, const float4& y1) -> float {
         float s = 0.f;
         s = __fmaf_rn(qv[0], y0.x, s); s = __fmaf_rn(qv[1], y0.y, s);
         s = __fmaf_rn(qv[2], y0.z, s); s = __fmaf_rn(qv[3], y0.w, s);
@@ -237,35 +239,49 @@ __global__ __launch_bounds__(kSelThreads) void select_kernel(const SelArgs a) {
         return s;
     };
 
-    int cur = 0;
+    for (int e = threadIdx.x; e < 256; e += blockDim.x) sh.hist[e] = 0;
     if (threadIdx.x == 0) { sh.count = 0; sh.nkept = 0; }
     __syncthreads();
 
+    int cur = 0;
     // Push candidates t in [0, total) through the buffer, keeping the top k.
-    // get(t, &id, &rowptr) returns false when t is not eligible.
-    auto stream_topk = [&](int total, int k, auto&& get) {
+    // fetch(t, &elig, &id, &p, &y0, &y1) issues the candidate's loads; the
+    // results are used only after every load of the batch is in flight.
+    auto stream_topk = [&](int total, int k, auto&& fetch) {
         if (k <= 0) return;  // nothing is kept; the buffer stays empty
         const int chunk = a.cap - k;
         for (int t0 = 0; t0 < total; t0 += chunk) {
             const int t1 = min(total, t0 + chunk);
             float* bs = bsb[cur];
             int* bi = bib[cur];
-            for (int t = t0 + gid; t < t1; t += NG) {
-                int id;
-                const float* rp;
-                if (get(t, &id, &rp)) {
-                    const float sc = dot(rp);
-                    if (gl == 0) {
-                        const int p = atomicAdd(&sh.count, 1);
-                        bs[p] = sc;
-                        bi[p] = id;
+            int* bp = bpb[cur];
+            for (int t = t0 + gid; t < t1; t += NG * kUnroll) {
+                float4 y0[kUnroll], y1[kUnroll];
+                int idv[kUnroll], pv[kUnroll];
+                bool ok[kUnroll];
+#pragma unroll
+                for (int v = 0; v < kUnroll; ++v) {
+                    const int tt = t + v * NG;
+                    ok[v] = tt < t1;
+                    if (ok[v]) fetch(tt, &ok[v], &idv[v], &pv[v], &y0[v], &y1[v]);
+                }
+#pragma unroll
+                for (int v = 0; v < kUnroll; ++v) {
+                    if (ok[v]) {
+                        const float sc = dot(y0[v], y1[v]);
+                        if (gl == 0) {
+                            const int p = atomicAdd(&sh.count, 1);
+                            bs[p] = sc;
+                            bi[p] = idv[v];
+                            bp[p] = pv[v];
+                        }
                     }
                 }
             }
             __syncthreads();
             const int n = sh.count;
             if (n > k) {
-                topk_compact(bs, bi, n, k, bsb[cur ^ 1], bib[cur ^ 1], sh);
+                topk_compact(bs, bi, bp, n, k, bsb[cur ^ 1], bib[cur ^ 1], bpb[cur ^ 1], sh);
                 cur ^= 1;
                 if (threadIdx.x == 0) sh.count = k;
             }
@@ -273,83 +289,93 @@ __global__ __launch_bounds__(kSelThreads) void select_kernel(const SelArgs a) {
         }
     };
 
-    int nsel;
     if (!FULL) {
         for (int l = 0; l < a.levels; ++l) {
             const int nl = a.n_l[l];
-            const float* cent = a.cent[l] + (int64_t)u * nl * R;
-            const int64_t* mp = a.minpos[l] + (int64_t)u * nl;
+            const float* cent = a.ocent[l] + (int64_t)u * nl * R;
+            const int64_t* mp = a.omp[l] + (int64_t)u * nl;
+            const int32_t* oid = a.oid[l] + (int64_t)u * nl;
             const int nk = sh.nkept;
-            const int total = (l == 0) ? nl : sh.pre[nk];
-            const int32_t* coff = l > 0 ? a.child_off[l - 1] + (int64_t)u * a.n_l[l - 1] : nullptr;
-            const int32_t* cids = l > 0 ? a.child_ids[l - 1] : nullptr;
+            const int total = (l == 0) ? nl : pre[nk];
             if (threadIdx.x == 0) sh.count = 0;
             __syncthreads();
-            stream_topk(total, a.beam, [&](int t, int* id, const float** rp) -> bool {
-                int node;
+            stream_topk(total, a.beam, [&](int t, bool* el, int* id, int* p, float4* y0, float4* y1) {
+                int q;
                 if (l == 0) {
-                    node = t;
+                    q = t;
                 } else {
-                    const int p = find_owner(sh, nk, t);
-                    node = cids[coff[sh.kk[p]] + (t - sh.pre[p])];
+                    const int o = find_owner(pre, nk, t);
+                    q = lo[o] + (t - pre[o]);
                 }
-                if (mp[node] > bound) return false;
-                *id = node;
-                *rp = cent + (int64_t)node * R;
-                return true;
+                const float4* rp = reinterpret_cast<const float4*>(cent + (int64_t)q * R + gl * 8);
+                *y0 = __ldg(rp);
+                *y1 = __ldg(rp + 1);
+                *id = __ldg(oid + q);
+                *p = q;
+                *el = __ldg(mp + q) <= bound;
             });
             const int n = sh.count;
-            for (int e = threadIdx.x; e < n; e += blockDim.x) sh.kk[e] = bib[cur][e];
+            for (int e = threadIdx.x; e < n; e += blockDim.x) kk[e] = bpb[cur][e];
             __syncthreads();
             if (threadIdx.x == 0) sh.nkept = n;
             if (l + 1 < a.levels) {
-                const int32_t* co = a.child_off[l] + (int64_t)u * nl;
+                // child positions of kept node q: [co[q], co[q+1]) minus the unit's base
+                const int32_t* co = a.ocoff[l] + (int64_t)u * nl;
+                const int child_base = u * a.n_l[l + 1];
                 for (int e = threadIdx.x; e < n; e += blockDim.x) {
-                    const int node = bib[cur][e];
-                    sh.pre[e] = co[node + 1] - co[node];
+                    const int q = kk[e];
+                    lo[e] = co[q] - child_base;
+                    pre[e] = co[q + 1] - co[q];
                 }
-                scan_pre(sh, n);
+                scan_pre(pre, n);
             }
             __syncthreads();
         }
         // candidate slot range of every kept leaf
         const int nk = sh.nkept;
         const int L = a.n_l[a.levels - 1];
+        const int32_t* oidl = a.oid[a.levels - 1] + (int64_t)u * L;
         for (int e = threadIdx.x; e < nk; e += blockDim.x) {
-            const int leaf = sh.kk[e];
+            const int leaf = oidl[kk[e]];
             const int64_t c = (int64_t)u * L + leaf;
             const int st = a.leaf_start[c];
             const int cntl = a.leaf_cnt[c];
             const int32_t* bl = a.blk + st;
-            int lo = 0, hi = cntl;  // first index with bl >= b_lo
-            while (lo < hi) { const int m = (lo + hi) >> 1; if (bl[m] < b_lo) lo = m + 1; else hi = m; }
-            int lo2 = lo, hi2 = cntl; // first index with bl > b_hi
+            int lo1 = 0, hi1 = cntl;  // first index with bl >= b_lo
+            while (lo1 < hi1) { const int m = (lo1 + hi1) >> 1; if (bl[m] < b_lo) lo1 = m + 1; else hi1 = m; }
+            int lo2 = lo1, hi2 = cntl; // first index with bl > b_hi
             while (lo2 < hi2) { const int m = (lo2 + hi2) >> 1; if (bl[m] <= b_hi) lo2 = m + 1; else hi2 = m; }
-            sh.lo[e] = st + lo;
-            sh.pre[e] = lo2 - lo;
+            lo[e] = st + lo1;
+            pre[e] = lo2 - lo1;
         }
-        scan_pre(sh, nk);
+        scan_pre(pre, nk);
         if (threadIdx.x == 0) sh.count = 0;
         __syncthreads();
-        stream_topk(sh.pre[nk], a.kb, [&](int t, int* id, const float** rp) -> bool {
-            const int p = find_owner(sh, nk, t);
-            const int64_t slot = sh.lo[p] + (t - sh.pre[p]);
-            *id = a.blk[slot];
-            *rp = a.Klp + slot * R;
-            return true;
+        stream_topk(pre[nk], a.kb, [&](int t, bool* el, int* id, int* p, float4* y0, float4* y1) {
+            const int o = find_owner(pre, nk, t);
+            const int64_t slot = lo[o] + (t - pre[o]);
+            const float4* rp = reinterpret_cast<const float4*>(a.Klp + slot * R + gl * 8);
+            *y0 = __ldg(rp);
+            *y1 = __ldg(rp + 1);
+            *id = __ldg(a.blk + slot);
+            *p = 0;
+            *el = true;
         });
     } else {
         const int64_t hi = min(a.nb - 1, b_hi);
         const int total = hi >= b_lo ? (int)(hi - b_lo + 1) : 0;
         const float* kl = a.Kl + (int64_t)u * a.nb_cap * R;
-        stream_topk(total, a.kb, [&](int t, int* id, const float** rp) -> bool {
+        stream_topk(total, a.kb, [&](int t, bool* el, int* id, int* p, float4* y0, float4* y1) {
             const int64_t b = b_lo + t;
+            const float4* rp = reinterpret_cast<const float4*>(kl + b * R + gl * 8);
+            *y0 = __ldg(rp);
+            *y1 = __ldg(rp + 1);
             *id = (int)b;
-            *rp = kl + b * R;
-            return true;
+            *p = 0;
+            *el = true;
         });
     }
-    nsel = sh.count;
+    const int nsel = sh.count;
 
     // ascending block ids (bitonic sort, padded to a power of two)
     int M = 1;
@@ -388,7 +414,7 @@ __global__ __launch_bounds__(kSelThreads) void select_kernel(const SelArgs a) {
 
 template <int R>
 int launch_select_r(const SelArgs& a, int64_t nq, int64_t units, bool fullscan, cudaStream_t s) {
-    const size_t smem = (size_t)a.cap * 16;
+    const size_t smem = (size_t)a.cap * 24 + (size_t)(3 * a.beam + 1) * 4;
     auto kern = fullscan ? select_kernel<R, true> : select_kernel<R, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_status(e);
@@ -404,13 +430,13 @@ int launch_select(const lsa_index* ix, const lsa_select_params* sp, const float*
                   const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt, int max_sel, bool fullscan,
                   cudaStream_t s) {
     const lsa_build_params& p = ix->p;
-    if (sp->beam > kMaxBeam) return LSA_ERR_INVALID_ARG;
+    if (sp->beam > 1024) return LSA_ERR_INVALID_ARG;
     SelArgs a{};
     for (int l = 0; l < p.levels; ++l) {
-        a.cent[l] = ix->cent[l];
-        a.minpos[l] = ix->minpos[l];
-        a.child_off[l] = ix->child_off[l];
-        a.child_ids[l] = ix->child_ids[l];
+        a.ocent[l] = ix->ord_cent[l];
+        a.omp[l] = ix->ord_mp[l];
+        a.oid[l] = ix->ord_id[l];
+        a.ocoff[l] = ix->ord_coff[l];
         a.n_l[l] = p.level_sizes[l];
     }
     a.levels = p.levels;
@@ -435,7 +461,7 @@ int launch_select(const lsa_index* ix, const lsa_select_params* sp, const float*
     a.cnt = cnt;
     a.max_sel = max_sel;
     const int kmax = a.kb > a.beam ? a.kb : a.beam;
-    int cap = 2048;
+    int cap = 1024;
     while (cap < 2 * kmax) cap <<= 1;
     a.cap = cap;
     if (nq <= 0) return LSA_OK;

@@ -70,6 +70,49 @@ __global__ void minpos_up_kernel(const int32_t* __restrict__ child_off, const in
     mp[c] = best;
 }
 
+// Tree order: level 0 keeps its ids; the children of the node at position q
+// of level l take the positions [coff[q], coff[q+1]) of level l+1, in
+// ascending child id.
+__global__ void order_identity_kernel(int32_t* __restrict__ ord_id, int64_t total, int n_l) {
+    const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e < total) ord_id[e] = (int32_t)(e % n_l);
+}
+
+__global__ void order_counts_kernel(const int32_t* __restrict__ ord_id, const int32_t* __restrict__ child_off,
+                                    int64_t total, int n_l, int32_t* __restrict__ cnt) {
+    const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= total) return;
+    const int64_t u = e / n_l;
+    const int64_t node = u * n_l + ord_id[e];
+    cnt[e] = child_off[node + 1] - child_off[node];
+}
+
+__global__ void order_children_kernel(const int32_t* __restrict__ ord_id, const int32_t* __restrict__ child_off,
+                                      const int32_t* __restrict__ child_ids, const int32_t* __restrict__ coff,
+                                      int64_t total, int n_l, int n_child, int32_t* __restrict__ ord_id_child) {
+    const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= total) return;
+    const int64_t u = e / n_l;
+    const int64_t node = u * n_l + ord_id[e];
+    const int32_t s = child_off[node], n = child_off[node + 1] - s;
+    for (int32_t k = 0; k < n; ++k) ord_id_child[coff[e] + k] = child_ids[s + k];
+}
+
+__global__ void order_gather_kernel(const int32_t* __restrict__ ord_id, int64_t total, int n_l, int r,
+                                    const float* __restrict__ cent, const int64_t* __restrict__ mp,
+                                    float* __restrict__ ocent, int64_t* __restrict__ omp, int32_t* __restrict__ opos) {
+    const int64_t e = ((int64_t)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int lane = threadIdx.x & 31;
+    if (e >= total) return;
+    const int64_t u = e / n_l;
+    const int64_t node = u * n_l + ord_id[e];
+    for (int c = lane; c < r; c += 32) ocent[e * r + c] = cent[node * r + c];
+    if (lane == 0) {
+        omp[e] = mp[node];
+        opos[node] = (int32_t)(e - u * n_l);
+    }
+}
+
 }  // namespace
 
 int finish_tree(lsa_index* ix, const int32_t* leaf_perm, const int32_t* leaf_off, const int32_t* const* up_perm,
@@ -101,6 +144,33 @@ int finish_tree(lsa_index* ix, const int32_t* leaf_perm, const int32_t* leaf_off
         minpos_up_kernel<<<(unsigned)((U * n_l + 255) / 256), 256, 0, s>>>(ix->child_off[l], ix->child_ids[l],
                                                                            U * n_l, n_l, n_child,
                                                                            ix->minpos[l + 1], ix->minpos[l]);
+    }
+    // tree order of every level
+    int32_t* ocnt = A.alloc<int32_t>(U * (int64_t)p.level_sizes[levels - 1]);
+    int32_t* osc = A.alloc<int32_t>(scan_scratch_elems(U * (int64_t)p.level_sizes[levels - 1]) + 1);
+    if (A.status != LSA_OK) return A.status;
+    {
+        const int64_t t0 = U * p.level_sizes[0];
+        note_launch();
+        order_identity_kernel<<<(unsigned)((t0 + 255) / 256), 256, 0, s>>>(ix->ord_id[0], t0, p.level_sizes[0]);
+    }
+    for (int l = 0; l + 1 < levels; ++l) {
+        const int n_l = p.level_sizes[l], n_child = p.level_sizes[l + 1];
+        const int64_t tot = U * n_l;
+        note_launch();
+        order_counts_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, s>>>(ix->ord_id[l], ix->child_off[l], tot, n_l,
+                                                                          ocnt);
+        scan_exclusive(ocnt, ix->ord_coff[l], tot, osc, s);
+        note_launch();
+        order_children_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, s>>>(
+            ix->ord_id[l], ix->child_off[l], ix->child_ids[l], ix->ord_coff[l], tot, n_l, n_child, ix->ord_id[l + 1]);
+    }
+    for (int l = 0; l < levels; ++l) {
+        const int64_t tot = U * p.level_sizes[l];
+        note_launch();
+        order_gather_kernel<<<(unsigned)((tot * 32 + 255) / 256), 256, 0, s>>>(
+            ix->ord_id[l], tot, p.level_sizes[l], p.r, ix->cent[l], ix->minpos[l], ix->ord_cent[l], ix->ord_mp[l],
+            ix->ord_pos[l]);
     }
     return cuda_status(cudaGetLastError());
 }
