@@ -14,12 +14,12 @@
 // One CTA per (query, KV head).  Every tree level is stored in tree order
 // (children of a node are contiguous), so a candidate's minpos, original id
 // and centroid row are independent loads; each sub-warp group of r/8 lanes
-// issues the loads of several candidates before it uses any of them.  Scores
-// stream through a shared-memory buffer; whenever it holds more than k items a
-// block-wide radix select (on the order-preserving bit pattern of the fp32
-// score, then on the original id for ties) compacts it to the top k.  The
-// order is total, (score desc, id asc), so the result does not depend on the
-// order in which warps append.
+// walks a contiguous run of candidates and issues the loads of several before
+// it uses any of them.  Scores stream through a shared-memory buffer;
+// whenever it holds more than k items a block-wide radix select (on the
+// order-preserving bit pattern of the fp32 score, then on the original id for
+// ties) compacts it to the top k.  The order is total, (score desc, id asc),
+// so the result does not depend on the order in which warps append.
 #include "lsa_internal.cuh"
 
 namespace lsa {
@@ -244,9 +244,14 @@ __global__ __launch_bounds__(kSelThreads) void select_kernel(const SelArgs a) {
     __syncthreads();
 
     int cur = 0;
+    uint32_t lt_mask;
+    asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt_mask));
     // Push candidates t in [0, total) through the buffer, keeping the top k.
-    // fetch(t, &elig, &id, &p, &y0, &y1) issues the candidate's loads; the
-    // results are used only after every load of the batch is in flight.
+    // Each group walks a contiguous run of candidates, kUnroll at a time:
+    // fetch(t, &state, &elig, &id, &p, &y0, &y1) issues the loads of
+    // candidate t (state carries the owning node across consecutive t), and
+    // the results are used only after every load of the batch is in flight.
+    // Appends are aggregated per warp: one shared-memory atomic per batch.
     auto stream_topk = [&](int total, int k, auto&& fetch) {
         if (k <= 0) return;  // nothing is kept; the buffer stays empty
         const int chunk = a.cap - k;
@@ -255,27 +260,41 @@ __global__ __launch_bounds__(kSelThreads) void select_kernel(const SelArgs a) {
             float* bs = bsb[cur];
             int* bi = bib[cur];
             int* bp = bpb[cur];
-            for (int t = t0 + gid; t < t1; t += NG * kUnroll) {
+            const int span = (t1 - t0 + NG - 1) / NG;
+            const int tb = t0 + gid * span;
+            const int te = min(t1, tb + span);
+            int state = -1;
+            for (int s0 = 0; s0 < span; s0 += kUnroll) {
                 float4 y0[kUnroll], y1[kUnroll];
                 int idv[kUnroll], pv[kUnroll];
                 bool ok[kUnroll];
 #pragma unroll
                 for (int v = 0; v < kUnroll; ++v) {
-                    const int tt = t + v * NG;
-                    ok[v] = tt < t1;
-                    if (ok[v]) fetch(tt, &ok[v], &idv[v], &pv[v], &y0[v], &y1[v]);
+                    const int tt = tb + s0 + v;
+                    ok[v] = tt < te;
+                    if (ok[v]) fetch(tt, &state, &ok[v], &idv[v], &pv[v], &y0[v], &y1[v]);
                 }
+                float sc[kUnroll];
+                uint32_t bal[kUnroll];
+                int nb_warp = 0;
 #pragma unroll
                 for (int v = 0; v < kUnroll; ++v) {
-                    if (ok[v]) {
-                        const float sc = dot(y0[v], y1[v]);
-                        if (gl == 0) {
-                            const int p = atomicAdd(&sh.count, 1);
-                            bs[p] = sc;
-                            bi[p] = idv[v];
-                            bp[p] = pv[v];
-                        }
+                    if (ok[v]) sc[v] = dot(y0[v], y1[v]);
+                    bal[v] = __ballot_sync(0xffffffffu, ok[v] && gl == 0);
+                    nb_warp += __popc(bal[v]);
+                }
+                int base = 0;
+                if (lane == 0 && nb_warp) base = atomicAdd(&sh.count, nb_warp);
+                base = __shfl_sync(0xffffffffu, base, 0);
+#pragma unroll
+                for (int v = 0; v < kUnroll; ++v) {
+                    if (ok[v] && gl == 0) {
+                        const int p = base + __popc(bal[v] & lt_mask);
+                        bs[p] = sc[v];
+                        bi[p] = idv[v];
+                        bp[p] = pv[v];
                     }
+                    base += __popc(bal[v]);
                 }
             }
             __syncthreads();
@@ -289,6 +308,16 @@ __global__ __launch_bounds__(kSelThreads) void select_kernel(const SelArgs a) {
         }
     };
 
+    // owner of candidate t among the nk kept nodes (ranges pre[o]..pre[o+1]),
+    // advanced from the previous candidate's owner
+    auto owner = [&](int t, int nk, int* state) -> int {
+        int o = *state;
+        if (o < 0) o = find_owner(pre, nk, t);
+        while (pre[o + 1] <= t) ++o;
+        *state = o;
+        return o;
+    };
+
     if (!FULL) {
         for (int l = 0; l < a.levels; ++l) {
             const int nl = a.n_l[l];
@@ -299,12 +328,12 @@ __global__ __launch_bounds__(kSelThreads) void select_kernel(const SelArgs a) {
             const int total = (l == 0) ? nl : pre[nk];
             if (threadIdx.x == 0) sh.count = 0;
             __syncthreads();
-            stream_topk(total, a.beam, [&](int t, bool* el, int* id, int* p, float4* y0, float4* y1) {
+            stream_topk(total, a.beam, [&](int t, int* state, bool* el, int* id, int* p, float4* y0, float4* y1) {
                 int q;
                 if (l == 0) {
                     q = t;
                 } else {
-                    const int o = find_owner(pre, nk, t);
+                    const int o = owner(t, nk, state);
                     q = lo[o] + (t - pre[o]);
                 }
                 const float4* rp = reinterpret_cast<const float4*>(cent + (int64_t)q * R + gl * 8);
@@ -351,8 +380,8 @@ __global__ __launch_bounds__(kSelThreads) void select_kernel(const SelArgs a) {
         scan_pre(pre, nk);
         if (threadIdx.x == 0) sh.count = 0;
         __syncthreads();
-        stream_topk(pre[nk], a.kb, [&](int t, bool* el, int* id, int* p, float4* y0, float4* y1) {
-            const int o = find_owner(pre, nk, t);
+        stream_topk(pre[nk], a.kb, [&](int t, int* state, bool* el, int* id, int* p, float4* y0, float4* y1) {
+            const int o = owner(t, nk, state);
             const int64_t slot = lo[o] + (t - pre[o]);
             const float4* rp = reinterpret_cast<const float4*>(a.Klp + slot * R + gl * 8);
             *y0 = __ldg(rp);
@@ -365,7 +394,8 @@ __global__ __launch_bounds__(kSelThreads) void select_kernel(const SelArgs a) {
         const int64_t hi = min(a.nb - 1, b_hi);
         const int total = hi >= b_lo ? (int)(hi - b_lo + 1) : 0;
         const float* kl = a.Kl + (int64_t)u * a.nb_cap * R;
-        stream_topk(total, a.kb, [&](int t, bool* el, int* id, int* p, float4* y0, float4* y1) {
+        stream_topk(total, a.kb, [&](int t, int* state, bool* el, int* id, int* p, float4* y0, float4* y1) {
+            (void)state;
             const int64_t b = b_lo + t;
             const float4* rp = reinterpret_cast<const float4*>(kl + b * R + gl * 8);
             *y0 = __ldg(rp);
