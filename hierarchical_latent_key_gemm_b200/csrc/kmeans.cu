@@ -7,8 +7,9 @@
 // an empty cluster keeps its centroid; optional integer grid (means rounded
 // half-to-even onto multiples of 2^-g, exact integer arithmetic).
 //
-// Assign (float): distance = ||c||^2 - 2 x.c (||x||^2 is common to a row),
-// a register-tiled fp32 product on CUDA cores with the running argmin kept in
+// Assign (float): distance = ||c||^2 - 2 x.c (||x||^2 is common to a row);
+// for r = 32 or 64 on the tensor cores (kmeans_tc.cu), otherwise a
+// register-tiled fp32 product on CUDA cores with the running argmin kept in
 // registers.  Assign (grid): exact int64 sum of squared grid differences.
 // Update: members are grouped by a stable sort, so each cluster sums its
 // points in ascending order (float64 accumulation): deterministic bits.
@@ -382,8 +383,10 @@ int run_kmeans(const float* X, int64_t ldx, int64_t units, int64_t n, int r, int
     const int64_t nc = units * (int64_t)k;
     const int64_t ldxt = (n + 3) / 4 * 4;
     const int64_t ldct = ((int64_t)k + 3) / 4 * 4;
-    float* XT = grid_log2 > 0 ? nullptr : A.alloc<float>(units * r * ldxt);
-    float* CT = grid_log2 > 0 ? nullptr : A.alloc<float>(units * r * ldct);
+    const bool tc = assign_tc_supported(r, grid_log2);
+    const bool simt = grid_log2 == 0 && !tc;
+    float* XT = simt ? A.alloc<float>(units * r * ldxt) : nullptr;
+    float* CT = simt ? A.alloc<float>(units * r * ldct) : nullptr;
     float* cc = A.alloc<float>(nc);
     float* Cb = A.alloc<float>(nc * r);
     double* cobj = A.alloc<double>(nc);
@@ -394,7 +397,12 @@ int run_kmeans(const float* X, int64_t ldx, int64_t units, int64_t n, int r, int
     const int64_t tot = nc * r;
     note_launch();
     init_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, s>>>(X, ldx, units, n, k, r, out.C);
-    if (!grid_log2) launch_transpose(X, units, n, ldx, r, XT, ldxt, s);
+    if (simt) launch_transpose(X, units, n, ldx, r, XT, ldxt, s);
+    void* tcw = nullptr;
+    if (tc) {
+        const int st = assign_tc_prepare_points(X, ldx, units, n, r, k, A, s, &tcw);
+        if (st != LSA_OK) return st;
+    }
     float* cur = out.C;
     float* nxt = Cb;
     int rc = LSA_OK;
@@ -407,6 +415,10 @@ int run_kmeans(const float* X, int64_t ldx, int64_t units, int64_t n, int r, int
             note_launch();
             assign_grid_kernel<<<grid, threads, smem, s>>>(X, ldx, n, r, cur, k, grid_log2, out.labels, ldl, err);
             rc = cuda_status(cudaGetLastError());
+        } else if (tc) {
+            note_launch();
+            cnorm_kernel<<<(unsigned)((nc + 255) / 256), 256, 0, s>>>(cur, nc, r, cc);
+            rc = assign_tc_run(tcw, cur, cc, units, n, r, k, out.labels, ldl, err, s);
         } else {
             launch_transpose(cur, units, k, k, r, CT, ldct, s);
             note_launch();
@@ -432,6 +444,7 @@ int run_kmeans(const float* X, int64_t ldx, int64_t units, int64_t n, int r, int
         float* t = cur; cur = nxt; nxt = t;
         rc = cuda_status(cudaGetLastError());
     }
+    if (tcw) assign_tc_release(tcw);
     if (rc == LSA_OK && cur != out.C)
         cudaMemcpyAsync(out.C, cur, tot * sizeof(float), cudaMemcpyDeviceToDevice, s);
     return rc != LSA_OK ? rc : cuda_status(cudaGetLastError());

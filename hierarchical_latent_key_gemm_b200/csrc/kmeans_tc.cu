@@ -1,0 +1,381 @@
+// k-means assign on the 5th-generation tensor cores (tcgen05).
+//
+// distance(x, c_j) = ||c_j||^2 - 2 x.c_j (||x||^2 is common to a row); the
+// x.c products of a 128-point tile against 256-centroid tiles are one dense
+// GEMM per tile.  Operands are fp32; each is split into two tf32 parts
+// (x = xb + xs, c = cb + cs) and the GEMM runs over K = 3r with
+// A = [xb | xb | xs], B = [cb | cs | cb], so the accumulator holds
+// xb.cb + xb.cs + xs.cb: the dropped xs.cs term and the tf32 roundings leave an
+// error near 2^-21 of |x||c|, i.e. fp32-like assignments.
+//
+// One CTA per 128 points, persistent over all centroid tiles of its unit:
+//   warp 0    TMA producer: the point tile once (6 K-chunks resident), then
+//             centroid K-chunks through a 3-stage ring (128B swizzle)
+//   warp 1    TMEM owner and MMA issuer (one thread): tcgen05.mma kind::tf32,
+//             M=128, N=256, K=8 per instruction, into one of two TMEM
+//             accumulators (2 x 256 columns)
+//   warps 2-5 epilogue: tcgen05.ld of the accumulator rows, running
+//             (distance, id) minimum per point, ties to the lower id
+// Every mbarrier wait is bounded; a timeout latches kErrTimeout and the CTA
+// winds down (TMEM is always released).
+#include <cuda.h>
+#include <cudaTypedefs.h>
+
+#include <mutex>
+#include <new>
+
+#include "lsa_internal.cuh"
+
+namespace lsa {
+namespace {
+
+constexpr int kTM = 128;          // points per CTA (UMMA M)
+constexpr int kTN = 256;          // centroids per tile (UMMA N)
+constexpr int kKC = 32;           // tf32 per K-chunk: one 128-byte swizzle row
+constexpr int kStagesB = 3;
+constexpr int kThreadsTC = 192;
+constexpr uint32_t kSpinLimit = 1u << 22;
+
+__device__ __forceinline__ uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
+}
+// Bounded wait for the phase with the given parity; false on timeout.
+__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
+    const uint32_t a = su32(b);
+    for (uint32_t it = 0; it < kSpinLimit; ++it) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(a), "r"(parity)
+            : "memory");
+        if (ok) return true;
+    }
+    return false;
+}
+__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
+        "[%2];" ::"r"(su32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(su32(bar)), "r"(x), "r"(y)
+        : "memory");
+}
+// K-major operand, 128-byte swizzle: 8-row x 128-byte atoms, 1024 bytes apart.
+__device__ __forceinline__ uint64_t umma_desc(const void* p) {
+    const uint64_t addr = su32(p);
+    uint64_t d = 0;
+    d |= (addr >> 4) & 0x3FFFull;          // start address
+    d |= (uint64_t)1 << 16;                // leading byte offset (unused for swizzled K-major)
+    d |= (uint64_t)(1024 >> 4) << 32;      // stride byte offset: next 8-row group
+    d |= (uint64_t)1 << 46;                // descriptor version
+    d |= (uint64_t)2 << 61;                // 128-byte swizzle
+    return d;
+}
+// kind::tf32, fp32 accumulate, K-major A and B, M = 128, N = 256.
+constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(kTN >> 3) << 17) |
+                            ((uint32_t)(kTM >> 4) << 24);
+
+__device__ __forceinline__ void umma_tf32(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(tmem_d),
+        "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate), "r"(0u));
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(bar))
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
+    uint32_t r[32];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
+        "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ float to_tf32(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return __uint_as_float(r);
+}
+
+// Xs[u*n_pad + p] = [tf32(x) | tf32(x) | tf32(x - tf32(x))], zero rows past n.
+__global__ void split_points_kernel(const float* __restrict__ X, int64_t ldx, int64_t n, int64_t n_pad, int r,
+                                    int64_t units, float* __restrict__ Xs) {
+    const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= units * n_pad * r) return;
+    const int c = (int)(e % r);
+    const int64_t row = e / r;
+    const int64_t u = row / n_pad, p = row % n_pad;
+    float x = 0.f;
+    if (p < n) x = X[(u * ldx + p) * r + c];
+    const float xb = to_tf32(x);
+    float* o = Xs + row * 3 * r;
+    o[c] = xb;
+    o[r + c] = xb;
+    o[2 * r + c] = to_tf32(x - xb);
+}
+
+// Cs[u*k_pad + j] = [tf32(c) | tf32(c - tf32(c)) | tf32(c)], zero rows past k.
+__global__ void split_centroids_kernel(const float* __restrict__ C, int k, int k_pad, int r, int64_t units,
+                                       float* __restrict__ Cs) {
+    const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= units * k_pad * r) return;
+    const int c = (int)(e % r);
+    const int64_t row = e / r;
+    const int64_t u = row / k_pad, j = row % k_pad;
+    float x = 0.f;
+    if (j < k) x = C[(u * k + j) * r + c];
+    const float xb = to_tf32(x);
+    float* o = Cs + row * 3 * r;
+    o[c] = xb;
+    o[r + c] = to_tf32(x - xb);
+    o[2 * r + c] = xb;
+}
+
+template <int R>
+__global__ void __launch_bounds__(kThreadsTC, 1)
+    assign_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_c,
+                     int64_t n, int64_t n_pad, int k, int k_pad, const float* __restrict__ cc,
+                     int32_t* __restrict__ labels, int64_t ldl, int32_t* err) {
+    constexpr int KS = 3 * R / kKC;                  // K-chunks
+    constexpr int A_CHUNK = kTM * 128;               // bytes per A chunk
+    constexpr int B_CHUNK = kTN * 128;               // bytes per B stage
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* smem = reinterpret_cast<unsigned char*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                                           ~uintptr_t(1023));
+    unsigned char* As = smem;                                    // KS x 16 KB
+    unsigned char* Bs = smem + KS * A_CHUNK;                     // kStagesB x 32 KB
+    uint64_t* bars = reinterpret_cast<uint64_t*>(Bs + kStagesB * B_CHUNK);
+    uint64_t* a_full = bars;                                     // 1
+    uint64_t* b_full = bars + 1;                                 // kStagesB
+    uint64_t* b_empty = b_full + kStagesB;                       // kStagesB
+    uint64_t* acc_full = b_empty + kStagesB;                     // 2
+    uint64_t* acc_empty = acc_full + 2;                          // 2
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(acc_empty + 2);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int u = blockIdx.y;
+    const int64_t p0 = (int64_t)blockIdx.x * kTM;
+    const int ntile = (k + kTN - 1) / kTN;
+
+    if (threadIdx.x == 0) {
+        mbar_init(a_full, 1);
+        for (int s = 0; s < kStagesB; ++s) {
+            mbar_init(b_full + s, 1);
+            mbar_init(b_empty + s, 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(acc_full + b, 1);
+            mbar_init(acc_empty + b, 128);
+        }
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    if (warp == 1) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], 512;" ::"r"(su32(tmem_slot)));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;");
+    const uint32_t tmem = *tmem_slot;
+
+    bool ok = true;
+    if (warp == 0) {
+        if (lane == 0) {
+            mbar_expect_tx(a_full, KS * A_CHUNK);
+            for (int c = 0; c < KS; ++c)
+                tma_load_2d(As + c * A_CHUNK, &map_x, a_full, c * kKC, (int)(u * n_pad + p0));
+            int issued = 0;
+            for (int t = 0; t < ntile && ok; ++t) {
+                for (int c = 0; c < KS && ok; ++c) {
+                    const int it = t * KS + c, s = it % kStagesB;
+                    const uint32_t ph = (uint32_t)(it / kStagesB) & 1u;
+                    if (!mbar_wait(b_empty + s, ph ^ 1u)) { ok = false; break; }
+                    mbar_expect_tx(b_full + s, B_CHUNK);
+                    tma_load_2d(Bs + s * B_CHUNK, &map_c, b_full + s, c * kKC, u * k_pad + t * kTN);
+                    ++issued;
+                }
+            }
+            if (!ok) {
+                latch(err, kErrTimeout);
+                // let the copies already issued land before the CTA exits
+                for (int it = 0; it < issued && it < kStagesB; ++it) {
+                    const int last = issued - 1 - it;
+                    mbar_wait(b_full + last % kStagesB, (uint32_t)(last / kStagesB) & 1u);
+                }
+                mbar_wait(a_full, 0);
+            }
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            if (!mbar_wait(a_full, 0)) ok = false;
+            for (int t = 0; t < ntile && ok; ++t) {
+                const int buf = t & 1;
+                if (!mbar_wait(acc_empty + buf, ((uint32_t)(t >> 1) & 1u) ^ 1u)) { ok = false; break; }
+                asm volatile("tcgen05.fence::after_thread_sync;");
+                const uint32_t d = tmem + buf * kTN;
+                for (int c = 0; c < KS; ++c) {
+                    const int it = t * KS + c, s = it % kStagesB;
+                    if (!mbar_wait(b_full + s, (uint32_t)(it / kStagesB) & 1u)) { ok = false; break; }
+                    asm volatile("tcgen05.fence::after_thread_sync;");
+#pragma unroll
+                    for (int kk = 0; kk < kKC / 8; ++kk) {
+                        const uint64_t da = umma_desc(As + c * A_CHUNK + kk * 32);
+                        const uint64_t db = umma_desc(Bs + s * B_CHUNK + kk * 32);
+                        umma_tf32(d, da, db, (c | kk) ? 1u : 0u);
+                    }
+                    umma_commit(b_empty + s);
+                }
+                if (!ok) break;
+                umma_commit(acc_full + buf);
+            }
+            if (!ok) latch(err, kErrTimeout);
+        }
+    } else {
+        // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31, one point per thread
+        const int q = warp & 3;
+        const int row = 32 * q + lane;
+        const int64_t p = p0 + row;
+        float best = INFINITY;
+        int bestj = 0;
+        const float* ccu = cc + (int64_t)u * k;
+        for (int t = 0; t < ntile; ++t) {
+            const int buf = t & 1;
+            if (!mbar_wait(acc_full + buf, (uint32_t)(t >> 1) & 1u)) { ok = false; latch(err, kErrTimeout); break; }
+            asm volatile("tcgen05.fence::after_thread_sync;");
+#pragma unroll 1
+            for (int cb = 0; cb < kTN / 32; ++cb) {
+                float v[32];
+                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + buf * kTN + cb * 32, v);
+                const int j0 = t * kTN + cb * 32;
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const int j = j0 + i;
+                    if (j < k) {
+                        const float dist = __fmaf_rn(-2.f, v[i], __ldg(ccu + j));
+                        if (dist < best) { best = dist; bestj = j; }
+                    }
+                }
+            }
+            asm volatile("tcgen05.fence::before_thread_sync;");
+            mbar_arrive(acc_empty + buf);
+        }
+        if (ok && p < n) labels[(int64_t)u * ldl + p] = bestj;
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;");
+    if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+    static std::once_flag once;
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    std::call_once(once, [] {
+        void* p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+        cudaGetLastError();
+    });
+    return fn;
+}
+
+// 2D fp32 tensor map: rows of `width` floats, boxes of 32 floats x box_rows.
+bool make_map(CUtensorMap* m, const float* base, int64_t rows, int width, int box_rows) {
+    auto fn = encode_fn();
+    if (!fn) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)width * sizeof(float)};
+    cuuint32_t box[2] = {(cuuint32_t)kKC, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int R>
+size_t tc_smem_bytes() {
+    return (size_t)(3 * R / kKC) * kTM * 128 + (size_t)kStagesB * kTN * 128 + 256 + 1024;
+}
+
+}  // namespace
+
+bool assign_tc_supported(int r, int grid_log2) { return (r == 32 || r == 64) && grid_log2 == 0 && encode_fn(); }
+
+// Scratch for the tensor-core assign of (units, n, k, r): split points and
+// split centroids.
+struct AssignTcWork {
+    float* Xs = nullptr;
+    float* Cs = nullptr;
+    int64_t n_pad = 0;
+    int k_pad = 0;
+};
+
+int assign_tc_prepare_points(const float* X, int64_t ldx, int64_t units, int64_t n, int r, int k, Arena& A,
+                             cudaStream_t s, void** work_out) {
+    AssignTcWork* w = new (std::nothrow) AssignTcWork();
+    if (!w) return LSA_ERR_OOM;
+    w->n_pad = (n + kTM - 1) / kTM * kTM;
+    w->k_pad = (k + kTN - 1) / kTN * kTN;
+    w->Xs = A.alloc<float>(units * w->n_pad * 3 * r);
+    w->Cs = A.alloc<float>(units * (int64_t)w->k_pad * 3 * r);
+    if (A.status != LSA_OK) { delete w; return A.status; }
+    const int64_t tot = units * w->n_pad * r;
+    note_launch();
+    split_points_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, s>>>(X, ldx, n, w->n_pad, r, units, w->Xs);
+    *work_out = w;
+    return cuda_status(cudaGetLastError());
+}
+
+void assign_tc_release(void* work) { delete static_cast<AssignTcWork*>(work); }
+
+int assign_tc_run(void* work, const float* C, const float* cc, int64_t units, int64_t n, int r, int k,
+                  int32_t* labels, int64_t ldl, int32_t* err, cudaStream_t s) {
+    AssignTcWork* w = static_cast<AssignTcWork*>(work);
+    const int64_t tot = units * (int64_t)w->k_pad * r;
+    note_launch();
+    split_centroids_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, s>>>(C, k, w->k_pad, r, units, w->Cs);
+    CUtensorMap mx, mc;
+    if (!make_map(&mx, w->Xs, units * w->n_pad, 3 * r, kTM) || !make_map(&mc, w->Cs, units * w->k_pad, 3 * r, kTN))
+        return LSA_ERR_CUDA;
+    dim3 grid((unsigned)(w->n_pad / kTM), (unsigned)units);
+    cudaError_t e;
+    if (r == 64) {
+        const size_t smem = tc_smem_bytes<64>();
+        e = cudaFuncSetAttribute(assign_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return cuda_status(e);
+        note_launch();
+        assign_tc_kernel<64><<<grid, kThreadsTC, smem, s>>>(mx, mc, n, w->n_pad, k, w->k_pad, cc, labels, ldl, err);
+    } else {
+        const size_t smem = tc_smem_bytes<32>();
+        e = cudaFuncSetAttribute(assign_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return cuda_status(e);
+        note_launch();
+        assign_tc_kernel<32><<<grid, kThreadsTC, smem, s>>>(mx, mc, n, w->n_pad, k, w->k_pad, cc, labels, ldl, err);
+    }
+    return cuda_status(cudaGetLastError());
+}
+
+}  // namespace lsa

@@ -145,6 +145,15 @@ GroupWork alloc_group_work(int64_t units, int64_t n, int k, Arena& A);
 int group_by_label(const int32_t* labels, int64_t ldl, int64_t units, int64_t n, int k, int32_t* perm,
                    int32_t* off, int32_t* err, cudaStream_t s, const GroupWork& w);
 
+// Tensor-core assign (kmeans_tc.cu): prepare the split points once per run,
+// then one call per Lloyd round.
+bool assign_tc_supported(int r, int grid_log2);
+int assign_tc_prepare_points(const float* X, int64_t ldx, int64_t units, int64_t n, int r, int k, Arena& A,
+                             cudaStream_t s, void** work_out);
+int assign_tc_run(void* work, const float* C, const float* cc, int64_t units, int64_t n, int r, int k,
+                  int32_t* labels, int64_t ldl, int32_t* err, cudaStream_t s);
+void assign_tc_release(void* work);
+
 // ---------------------------------------------------------------- latents
 int launch_project_pool(const void* K, const float* W, int64_t batch, int64_t n_blocks,
                         int64_t ld_tokens, int hkv, int d, int r, int pool, int dtype,
