@@ -18,13 +18,10 @@
 //             (distance, id) minimum per point, ties to the lower id
 // Every mbarrier wait is bounded; a timeout latches kErrTimeout and the CTA
 // winds down (TMEM is always released).
-#include <cuda.h>
-#include <cudaTypedefs.h>
-
 #include <mutex>
 #include <new>
 
-#include "lsa_internal.cuh"
+#include "tma_util.cuh"
 
 namespace lsa {
 namespace {
@@ -34,42 +31,6 @@ constexpr int kTN = 256;          // centroids per tile (UMMA N)
 constexpr int kKC = 32;           // tf32 per K-chunk: one 128-byte swizzle row
 constexpr int kStagesB = 3;
 constexpr int kThreadsTC = 192;
-constexpr uint32_t kSpinLimit = 1u << 22;
-
-__device__ __forceinline__ uint32_t su32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
-
-__device__ __forceinline__ void mbar_init(uint64_t* b, uint32_t count) {
-    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(su32(b)), "r"(count));
-}
-__device__ __forceinline__ void mbar_expect_tx(uint64_t* b, uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(su32(b)), "r"(bytes) : "memory");
-}
-__device__ __forceinline__ void mbar_arrive(uint64_t* b) {
-    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(su32(b)) : "memory");
-}
-// Bounded wait for the phase with the given parity; false on timeout.
-__device__ __forceinline__ bool mbar_wait(uint64_t* b, uint32_t parity) {
-    const uint32_t a = su32(b);
-    for (uint32_t it = 0; it < kSpinLimit; ++it) {
-        uint32_t ok;
-        asm volatile(
-            "{\n\t.reg .pred p;\n\t"
-            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-            "selp.u32 %0, 1, 0, p;\n\t}"
-            : "=r"(ok)
-            : "r"(a), "r"(parity)
-            : "memory");
-        if (ok) return true;
-    }
-    return false;
-}
-__device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], "
-        "[%2];" ::"r"(su32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(su32(bar)), "r"(x), "r"(y)
-        : "memory");
-}
 // K-major operand, 128-byte swizzle: 8-row x 128-byte atoms, 1024 bytes apart.
 __device__ __forceinline__ uint64_t umma_desc(const void* p) {
     const uint64_t addr = su32(p);
@@ -288,33 +249,6 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
     if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, 512;" ::"r"(tmem));
 }
 
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-    static std::once_flag once;
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    std::call_once(once, [] {
-        void* p = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-        cudaGetLastError();
-    });
-    return fn;
-}
-
-// 2D fp32 tensor map: rows of `width` floats, boxes of 32 floats x box_rows.
-bool make_map(CUtensorMap* m, const float* base, int64_t rows, int width, int box_rows) {
-    auto fn = encode_fn();
-    if (!fn) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)width * sizeof(float)};
-    cuuint32_t box[2] = {(cuuint32_t)kKC, (cuuint32_t)box_rows};
-    cuuint32_t estr[2] = {1, 1};
-    return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(base), dims, strides, box, estr,
-              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
 template <int R>
 size_t tc_smem_bytes() {
     return (size_t)(3 * R / kKC) * kTM * 128 + (size_t)kStagesB * kTN * 128 + 256 + 1024;
@@ -322,7 +256,7 @@ size_t tc_smem_bytes() {
 
 }  // namespace
 
-bool assign_tc_supported(int r, int grid_log2) { return (r == 32 || r == 64) && grid_log2 == 0 && encode_fn(); }
+bool assign_tc_supported(int r, int grid_log2) { return (r == 32 || r == 64) && grid_log2 == 0 && tma_available(); }
 
 // Scratch for the tensor-core assign of (units, n, k, r): split points and
 // split centroids.
@@ -358,7 +292,10 @@ int assign_tc_run(void* work, const float* C, const float* cc, int64_t units, in
     note_launch();
     split_centroids_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, s>>>(C, k, w->k_pad, r, units, w->Cs);
     CUtensorMap mx, mc;
-    if (!make_map(&mx, w->Xs, units * w->n_pad, 3 * r, kTM) || !make_map(&mc, w->Cs, units * w->k_pad, 3 * r, kTN))
+    if (!make_tensor_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->Xs, units * w->n_pad, 3 * r, 3 * r * 4, kKC,
+                            kTM) ||
+        !make_tensor_map_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->Cs, units * w->k_pad, 3 * r, 3 * r * 4, kKC,
+                            kTN))
         return LSA_ERR_CUDA;
     dim3 grid((unsigned)(w->n_pad / kTM), (unsigned)units);
     cudaError_t e;
