@@ -215,10 +215,13 @@ __global__ __launch_bounds__(kAttThreads) void attn_bf16_kernel(
         l1 = l1 * al1 + (p[0][2] + p[0][3] + p[1][2] + p[1][3]);
         m0 = mn0;
         m1 = mn1;
+        // rescale O only when some running maximum moved
+        if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
 #pragma unroll
-        for (int i = 0; i < D / 8; ++i) {
-            o[i][0] *= al0; o[i][1] *= al0;
-            o[i][2] *= al1; o[i][3] *= al1;
+            for (int i = 0; i < D / 8; ++i) {
+                o[i][0] *= al0; o[i][1] *= al0;
+                o[i][2] *= al1; o[i][3] *= al1;
+            }
         }
         // P = hi + lo, both bf16: the weights keep ~16 significant bits
         uint32_t pa[4], pl[4];

@@ -25,8 +25,16 @@
 namespace lsa {
 namespace {
 
+// 2 candidates in flight per group at 8 CTAs (32 warps) per SM measured
+// fastest on the 1M-token workload (4 in flight at 4 CTAs: 1.3x slower).
+#ifndef LSA_SELECT_UNROLL
+#define LSA_SELECT_UNROLL 2
+#endif
+#ifndef LSA_SELECT_MIN_BLOCKS
+#define LSA_SELECT_MIN_BLOCKS 8
+#endif
 constexpr int kSelThreads = 128;
-constexpr int kUnroll = 4;
+constexpr int kUnroll = LSA_SELECT_UNROLL;  // candidates in flight per group
 
 struct SelArgs {
     const float* ocent[LSA_MAX_LEVELS];     // [units*n_l][r], tree order
@@ -188,7 +196,7 @@ __device__ __forceinline__ int find_owner(const int* pre, int nk, int t) {
 }
 
 template <int R, bool FULL>
-__global__ __launch_bounds__(kSelThreads) void select_kernel(const SelArgs a) {
+__global__ __launch_bounds__(kSelThreads, LSA_SELECT_MIN_BLOCKS) void select_kernel(const SelArgs a) {
     extern __shared__ float4 dyn4[];
     __shared__ SelShared sh;
     float* bsb[2];

@@ -23,6 +23,7 @@ from __future__ import annotations
 import dataclasses
 from dataclasses import dataclass
 
+import numpy as np
 import torch
 
 
@@ -109,7 +110,7 @@ def torch_dtype(w: Workload):
 def make_map(w: Workload, seed: int = 0, device="cpu") -> torch.Tensor:
     """The seeded latent map W [d, r] (fp32).  Integer workload: every row has
     4 nonzeros in {-1, +1} at seeded positions.  Otherwise: orthonormal columns
-    (QR of a Gaussian matrix, signs fixed by the diagonal of R)."""
+    (Gram-Schmidt of a seeded Gaussian matrix)."""
     g = _gen("cpu", seed, _S_W)
     if w.kind == "int":
         Wm = torch.zeros(w.d, w.r, dtype=torch.float32)
@@ -119,35 +120,50 @@ def make_map(w: Workload, seed: int = 0, device="cpu") -> torch.Tensor:
             signs = torch.randint(0, 2, (nnz,), generator=g).float() * 2 - 1
             Wm[row, cols] = signs
     else:
-        A = torch.randn(w.d, w.r, generator=g, dtype=torch.float64)
-        Qm, Rm = torch.linalg.qr(A)
-        Wm = (Qm * torch.sign(torch.diagonal(Rm))[None, :]).to(torch.float32).contiguous()
+        # modified Gram-Schmidt in float64: the same bits on every host (a
+        # threaded LAPACK QR need not be bitwise reproducible)
+        A = torch.randn(w.d, w.r, generator=g, dtype=torch.float64).numpy()
+        Qm = np.zeros_like(A)
+        for j in range(w.r):
+            v = A[:, j].copy()
+            for i in range(j):
+                v -= float(np.dot(Qm[:, i], v)) * Qm[:, i]
+            Qm[:, j] = v / float(np.sqrt(np.dot(v, v)))
+        Wm = torch.from_numpy(Qm).to(torch.float32)
     return Wm.contiguous().to(device)
 
 
-def _segment_weights(w: Workload, n: int, seed: int, device) -> torch.Tensor | None:
-    """Mixture weights per drift segment: logits take a Gaussian random walk
-    (step 0.5) from one segment to the next.  None = uniform weights."""
+def _segment_cdfs(w: Workload, n: int, seed: int) -> np.ndarray | None:
+    """Cumulative mixture weights per drift segment (float64, CPU): logits
+    take a Gaussian random walk (step 0.5) from one segment to the next.
+    None = uniform weights."""
     if not w.drift_every:
         return None
     nseg = -(-n // w.drift_every)
-    g = _gen(device, seed, _S_DRIFT)
-    steps = torch.randn(nseg, w.components, generator=g, device=device) * 0.5
+    g = _gen("cpu", seed, _S_DRIFT)
+    steps = torch.randn(nseg, w.components, generator=g, dtype=torch.float64) * 0.5
     logits = torch.cumsum(steps, dim=0)
-    return torch.softmax(logits, dim=1)
+    weights = torch.softmax(logits, dim=1).numpy()
+    cdf = np.cumsum(weights, axis=1)
+    cdf[:, -1] = 1.0
+    return cdf
 
 
 def _components(w: Workload, n: int, count_per_pos: int, seed: int, stream: int, device) -> torch.Tensor:
-    """Mixture component per (position, slot): [n, count_per_pos] int64."""
+    """Mixture component per (position, slot): [n, count_per_pos] int64.
+    Drifting weights are sampled by inverse CDF (uniform draws located in the
+    segment's cumulative weights), which gives the same draws on any device."""
     g = _gen(device, seed, stream)
-    seg_w = _segment_weights(w, n, seed, device)
-    if seg_w is None:
+    cdfs = _segment_cdfs(w, n, seed)
+    if cdfs is None:
         return torch.randint(0, w.components, (n, count_per_pos), generator=g, device=device)
     out = torch.empty(n, count_per_pos, dtype=torch.int64, device=device)
-    for s in range(seg_w.shape[0]):
+    for s in range(cdfs.shape[0]):
         lo, hi = s * w.drift_every, min(n, (s + 1) * w.drift_every)
-        out[lo:hi] = torch.multinomial(seg_w[s], (hi - lo) * count_per_pos, replacement=True,
-                                       generator=g).view(hi - lo, count_per_pos)
+        cdf = torch.from_numpy(cdfs[s]).to(device)
+        u = torch.rand((hi - lo) * count_per_pos, generator=g, device=device, dtype=torch.float64)
+        c = torch.searchsorted(cdf, u, right=True).clamp_(max=w.components - 1)
+        out[lo:hi] = c.view(hi - lo, count_per_pos)
     return out
 
 

@@ -280,6 +280,29 @@ def test_select_three_levels_ragged_on_oracle_tree():
     _float_select_check(w, seed=3, sample=200)
 
 
+def test_select_and_attention_are_deterministic():
+    w = WORKLOADS["prefill_1m"].scaled(n_tokens=16384 + 9, level_sizes=(4, 32, 256), beam=16, topk=512,
+                                       window=256, needles=0, components=256, drift_every=4096)
+    inp = make_inputs(w, seed=21)
+    d = _dev(inp)
+    ix = lsa.lsa_build_index(TU.build_params(w), d["K"], d["W"])
+    sp = TU.select_params(w)
+    outs = []
+    for _ in range(3):
+        idx, cnt = lsa.lsa_select(ix, sp, d["Q"])
+        O_, lse = lsa.lsa_sparse_attn(d["Q"], d["K"], d["V"], idx, cnt, w.hkv)
+        outs.append((idx.clone(), cnt.clone(), O_.clone(), lse.clone()))
+    assert lsa.lsa_check(ix) == lsa.LSA_OK
+    for o in outs[1:]:
+        assert torch.equal(o[0], outs[0][0]) and torch.equal(o[1], outs[0][1])
+        assert torch.equal(o[2], outs[0][2]) and torch.equal(o[3], outs[0][3])
+    ix2 = lsa.lsa_build_index(TU.build_params(w), d["K"], d["W"])
+    for what in (lsa.LSA_GET_LEAF_OF_BLOCK, lsa.LSA_GET_CENTROIDS):
+        assert torch.equal(ix.get(what, 2), ix2.get(what, 2))
+    ix.free()
+    ix2.free()
+
+
 def test_full_beam_equals_fullscan_on_gpu():
     w = WORKLOADS["gqa_128k"].scaled(n_tokens=8192 + 3, level_sizes=(8, 64), needles=0, components=256)
     inp = make_inputs(w, seed=4)
