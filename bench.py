@@ -175,9 +175,9 @@ def run_ours(args):
     from hierarchical_latent_key_gemm_b200.workloads import WORKLOADS, describe, input_bytes, make_inputs
 
     w = WORKLOADS[args.workload]
-    if w.decode_steps:
-        raise SystemExit("bench.py times prefill workloads; decode is measured by its own tests")
     lsa.lib()
+    if w.decode_steps:
+        return run_decode(args, w, rank, world, dev)
     seed = args.seed + 1000 * rank
     inp = make_inputs(w, seed=seed, device=dev)
     Q, K, V, W = inp["Q"], inp["K"], inp["V"], inp["W"]
@@ -289,6 +289,71 @@ def run_ours(args):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def run_decode(args, w, rank, world, dev):
+    """Decode workload: build the index over every sequence's context (timed
+    once), then time decode steps: append the new token's key, select for the
+    new query, attend; one step covers all sequences of the batch."""
+    import torch
+    from hierarchical_latent_key_gemm_b200 import lsa
+    from hierarchical_latent_key_gemm_b200.workloads import describe, make_inputs
+    seed = args.seed + 1000 * rank
+    inp = make_inputs(w, seed=seed, device=dev)
+    K, V, Q, W = inp["K"], inp["V"], inp["Q"], inp["W"]
+    N = w.n_tokens
+    bp = lsa.make_build_params(w.batch, N, N + w.decode_steps, w.hkv, w.d, w.r, w.pool, lsa.LSA_BF16,
+                               w.level_sizes, w.lloyd_iters, w.grid_log2, w.sink, w.decode_steps)
+    sp = lsa.make_select_params(w.hq, w.beam, w.topk, w.sink, w.window)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    lsa.lsa_build_index(bp, K, W).free()  # warm-up build
+    torch.cuda.synchronize()
+    e0.record()
+    ix = lsa.lsa_build_index(bp, K, W)
+    e1.record()
+    torch.cuda.synchronize()
+    build_ms = e0.elapsed_time(e1)
+    idx = torch.empty((w.batch, 1, w.hkv, w.max_sel), dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.batch, 1, w.hkv), dtype=torch.int32, device=dev)
+    O = torch.empty((w.batch, 1, w.hq, w.d), dtype=torch.bfloat16, device=dev)
+    lse = torch.empty((w.batch, 1, w.hq), dtype=torch.float32, device=dev)
+    qs = [Q[:, s:s + 1].contiguous() for s in range(w.decode_steps)]
+
+    def step(s):
+        lsa.lsa_append(ix, K, 1)
+        lsa.lsa_select(ix, sp, qs[s], q_pos0=N + s, idx=idx, cnt=cnt, max_sel=w.max_sel)
+        lsa.lsa_sparse_attn(qs[s], K, V, idx, cnt, w.hkv, O=O, lse=lse)
+
+    warm = min(args.warmup, w.decode_steps // 4)
+    for s in range(warm):
+        step(s)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local_rank())
+    clocks.start()
+    launches0 = lsa.lsa_launch_count()
+    e0.record()
+    for s in range(warm, w.decode_steps):
+        step(s)
+    e1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    n_timed = w.decode_steps - warm
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / n_timed
+    st = lsa.lsa_check(ix)
+    info = ix.info()
+    ix.free()
+    if rank == 0:
+        print(json.dumps({
+            "metric": "LSA decode ms per step (append + select + attention, all sequences) at 10M context",
+            "value": ms, "unit": "ms/step", "n_gpus": world, "steps": n_timed, "warmup": warm,
+            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": {"workload": describe(w)}, "build_ms": build_ms,
+            "index_device_bytes": int(info.device_bytes), "gpu_launches": lsa.lsa_launch_count() - launches0,
+            "status": lsa.strerror(st), "clocks": clk}), flush=True)
+
+
+def local_rank() -> int:
+    return int(os.environ.get("LOCAL_RANK", "0"))
 
 
 def run_e2e(args, w, inp, bp, sp, idx, cnt, O, lse, dev, world):
