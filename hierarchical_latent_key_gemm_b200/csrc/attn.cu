@@ -14,6 +14,8 @@
 // 64-key tiles; each of the 4 warps owns 16 keys of every tile and the warps'
 // partial (max, sum, O) are merged at the end.
 // fp32 path: CUDA-core dot products, one warp per key, same merge.
+#include <algorithm>
+
 #include "lsa_internal.cuh"
 
 namespace lsa {
@@ -71,7 +73,8 @@ template <int D>
 __global__ __launch_bounds__(kAttThreads) void attn_bf16_kernel(
     const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V,
     const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt, int64_t nq, int hq, int hkv, int max_sel,
-    int64_t ld_tokens, __nv_bfloat16* __restrict__ O, float* __restrict__ lse, int32_t* err, float scale_log2) {
+    int64_t ld_tokens, __nv_bfloat16* __restrict__ O, float* __restrict__ lse, int32_t* err, float scale_log2,
+    int nsplit, float* __restrict__ part) {
     constexpr int CH = D / 8;                       // 16-byte chunks per row
     constexpr int TILE_BYTES = kTileKeys * D * 2;   // one K (or V) tile
     extern __shared__ __align__(128) unsigned char smem[];
@@ -102,7 +105,11 @@ __global__ __launch_bounds__(kAttThreads) void attn_bf16_kernel(
         *reinterpret_cast<uint4*>(Qs + swz<D>(r, c)) = v;
     }
 
-    const int ntile = (n + kTileKeys - 1) / kTileKeys;
+    // split-K: CTA z of nsplit takes a contiguous run of the row list's tiles
+    const int ntile_all = (n + kTileKeys - 1) / kTileKeys;
+    const int per_split = (ntile_all + nsplit - 1) / nsplit;
+    const int tile0 = blockIdx.z * per_split;
+    const int ntile = max(0, min(ntile_all, tile0 + per_split) - tile0);
     // Each thread gathers the same 16-byte column c of RPT rows of every tile;
     // its token ids are read one tile ahead into registers, so the gathers
     // never wait on an index load.
@@ -112,7 +119,7 @@ __global__ __launch_bounds__(kAttThreads) void attn_bf16_kernel(
     auto fetch_tokens = [&](int t, int* tk) {
 #pragma unroll
         for (int k = 0; k < RPT; ++k) {
-            const int j = t * kTileKeys + r_base + ROW_STEP * k;
+            const int j = (tile0 + t) * kTileKeys + r_base + ROW_STEP * k;
             tk[k] = (t < ntile && j < n) ? __ldg(ir + j) : -1;
         }
     };
@@ -283,9 +290,46 @@ __global__ __launch_bounds__(kAttThreads) void attn_bf16_kernel(
                 acc += f * Om[(w * 16 + r) * D + c];
             }
         }
+        if (part) {
+            // partial of this split: unnormalised sum, running max (log2 units), sum of weights
+            float* pp = part + ((row * nsplit + blockIdx.z) * G + r) * (D + 2);
+            pp[c] = acc;
+            if (c == 0) { pp[D] = M; pp[D + 1] = Ls; }
+            continue;
+        }
         const float outv = Ls > 0.f ? acc / Ls : 0.f;
         O[((b * nq + qi) * hq + (int64_t)h * G + r) * D + c] = __float2bfloat16_rn(outv);
         if (c == 0 && lse) lse[(b * nq + qi) * hq + (int64_t)h * G + r] = Ls > 0.f ? (M + log2f(Ls)) * 0.69314718055994531f : -INFINITY;
+    }
+}
+
+// Merge the nsplit partials of every (query, KV head) row list by their
+// maxima: O = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s.
+template <int D>
+__global__ __launch_bounds__(kAttThreads) void attn_combine_kernel(const float* __restrict__ part, int nsplit,
+                                                                    int64_t nq, int hq, int hkv,
+                                                                    __nv_bfloat16* __restrict__ O,
+                                                                    float* __restrict__ lse) {
+    const int G = hq / hkv;
+    const int64_t row = blockIdx.x;  // (b * nq + qi) * hkv + h
+    const int h = (int)(row % hkv);
+    const int64_t bq = row / hkv;    // b * nq + qi
+    for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
+        const int r = e / D, c = e % D;
+        const float* p0 = part + (row * nsplit * G + r) * (D + 2);
+        float M = -INFINITY;
+        for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, p0[(int64_t)sp * G * (D + 2) + D]);
+        float Ls = 0.f, acc = 0.f;
+        if (M != -INFINITY) {
+            for (int sp = 0; sp < nsplit; ++sp) {
+                const float* pp = p0 + (int64_t)sp * G * (D + 2);
+                const float f = exp2f(pp[D] - M);
+                Ls += f * pp[D + 1];
+                acc += f * pp[c];
+            }
+        }
+        O[(bq * hq + (int64_t)h * G + r) * D + c] = __float2bfloat16_rn(Ls > 0.f ? acc / Ls : 0.f);
+        if (c == 0 && lse) lse[bq * hq + (int64_t)h * G + r] = Ls > 0.f ? (M + log2f(Ls)) * 0.69314718055994531f : -INFINITY;
     }
 }
 
@@ -381,12 +425,38 @@ int launch_bf16(const void* Q, const void* K, const void* V, const int32_t* idx,
     cudaError_t e = cudaFuncSetAttribute(attn_bf16_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_status(e);
     const float scale_log2 = 1.4426950408889634f / sqrtf((float)D);
-    dim3 grid((unsigned)nq, (unsigned)(batch * hkv));
+    // few row lists (decode): split each across CTAs, then merge
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t rows_n = batch * nq * hkv;
+    int nsplit = 1;
+    if (rows_n < 2 * (int64_t)sms) {
+        const int64_t want = (4 * (int64_t)sms + rows_n - 1) / rows_n;
+        const int64_t tiles = ((int64_t)max_sel + kTileKeys - 1) / kTileKeys;
+        nsplit = (int)std::max<int64_t>(1, std::min<int64_t>({32, want, (tiles + 1) / 2}));
+    }
+    Arena scratch;
+    scratch.async = true;
+    scratch.stream = s;
+    float* part = nullptr;
+    if (nsplit > 1) {
+        part = scratch.alloc<float>(rows_n * nsplit * (hq / hkv) * (D + 2));
+        if (scratch.status != LSA_OK) return scratch.status;
+    }
+    dim3 grid((unsigned)nq, (unsigned)(batch * hkv), (unsigned)nsplit);
     note_launch();
     attn_bf16_kernel<D><<<grid, kAttThreads, smem, s>>>(
         (const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, idx, cnt, nq, hq, hkv, max_sel,
-        ld_tokens, (__nv_bfloat16*)O, lse, err, scale_log2);
-    return cuda_status(cudaGetLastError());
+        ld_tokens, (__nv_bfloat16*)O, lse, err, scale_log2, nsplit, part);
+    if (nsplit > 1) {
+        note_launch();
+        attn_combine_kernel<D><<<(unsigned)rows_n, kAttThreads, 0, s>>>(part, nsplit, nq, hq, hkv,
+                                                                       (__nv_bfloat16*)O, lse);
+    }
+    const int st = cuda_status(cudaGetLastError());
+    scratch.release();
+    return st;
 }
 
 template <int D>

@@ -195,8 +195,13 @@ __device__ __forceinline__ int find_owner(const int* pre, int nk, int t) {
     return lo;
 }
 
-template <int R, bool FULL>
-__global__ __launch_bounds__(kSelThreads, LSA_SELECT_MIN_BLOCKS) void select_kernel(const SelArgs a) {
+// THREADS = kSelThreads for large grids; small grids (decode: a few queries)
+// give each (query, KV head) kWideThreads so the few CTAs use more of the SM.
+constexpr int kWideThreads = 1024;
+
+template <int R, bool FULL, int THREADS>
+__global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BLOCKS : 1) void select_kernel(
+    const SelArgs a) {
     extern __shared__ float4 dyn4[];
     __shared__ SelShared sh;
     float* bsb[2];
@@ -214,7 +219,7 @@ __global__ __launch_bounds__(kSelThreads, LSA_SELECT_MIN_BLOCKS) void select_ker
 
     constexpr int LPC = R / 8;              // lanes per candidate row
     constexpr int CPW = 32 / LPC;           // candidates per warp
-    constexpr int NG = (kSelThreads / 32) * CPW;
+    constexpr int NG = (THREADS / 32) * CPW;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane / LPC, gl = lane % LPC, gid = warp * CPW + g;
     const unsigned gmask = (LPC == 32) ? 0xffffffffu : (((1u << LPC) - 1u) << (g * LPC));
@@ -450,16 +455,25 @@ __global__ __launch_bounds__(kSelThreads, LSA_SELECT_MIN_BLOCKS) void select_ker
     if (threadIdx.x == 0) a.cnt[row] = (int32_t)total;
 }
 
-template <int R>
-int launch_select_r(const SelArgs& a, int64_t nq, int64_t units, bool fullscan, cudaStream_t s) {
+template <int R, int THREADS>
+int launch_select_t(const SelArgs& a, int64_t nq, int64_t units, bool fullscan, cudaStream_t s) {
     const size_t smem = (size_t)a.cap * 24 + (size_t)(3 * a.beam + 1) * 4;
-    auto kern = fullscan ? select_kernel<R, true> : select_kernel<R, false>;
+    auto kern = fullscan ? select_kernel<R, true, THREADS> : select_kernel<R, false, THREADS>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_status(e);
     dim3 grid((unsigned)nq, (unsigned)units);
     note_launch();
-    kern<<<grid, kSelThreads, smem, s>>>(a);
+    kern<<<grid, THREADS, smem, s>>>(a);
     return cuda_status(cudaGetLastError());
+}
+
+template <int R>
+int launch_select_r(const SelArgs& a, int64_t nq, int64_t units, bool fullscan, cudaStream_t s) {
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (nq * units < 2 * (int64_t)sms) return launch_select_t<R, kWideThreads>(a, nq, units, fullscan, s);
+    return launch_select_t<R, kSelThreads>(a, nq, units, fullscan, s);
 }
 
 }  // namespace
