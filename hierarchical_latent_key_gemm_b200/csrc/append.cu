@@ -6,15 +6,20 @@
 // the build (same arithmetic order, so identical bits), placed in its nearest
 // leaf by squared distance over all leaves (frozen centroids, ties to the
 // lower id) at the end of that leaf's ascending member run, and the minpos of
-// the leaf and its ancestors is lowered.  One CTA per unit walks its new
-// blocks in order.  A full leaf latches kErrCapacity and leaves the block
-// unindexed.
+// the leaf and its ancestors is lowered.  A full leaf latches kErrCapacity
+// and leaves the block unindexed.
+//
+// Three launches: latents of the new blocks; the nearest-leaf scan spread over
+// many CTAs (each takes a chunk of leaves, one warp per leaf row, and folds its
+// best (distance, leaf) into one 64-bit key per block with atomicMin, so ties
+// go to the lower leaf); the ordered insertion, one CTA per unit.
 #include "latent_common.cuh"
 
 namespace lsa {
 namespace {
 
 constexpr int kAppThreads = 256;
+constexpr int kLeavesPerCta = 512;
 
 struct AppArgs {
     const float* W;
@@ -33,107 +38,122 @@ struct AppArgs {
     int n_l[LSA_MAX_LEVELS];
     int levels, L, d, r, pool, sink, hkv, grid_log2;
     int64_t nb_cap, ld_tokens, first_block, n_new;
+    unsigned long long* best;   // [units][n_new] packed (distance, leaf)
     int32_t* err;
 };
 
+// Latent of every new block: blockIdx.x = new block, blockIdx.y = unit.
 template <typename T>
-__global__ __launch_bounds__(kAppThreads) void append_kernel(const T* __restrict__ K, const AppArgs a) {
+__global__ __launch_bounds__(kAppThreads) void append_latent_kernel(const T* __restrict__ K, const AppArgs a) {
     extern __shared__ float sm[];
     float* Ws = sm;                     // [d][r]
     float* mean = Ws + a.d * a.r;       // [d]
-    float* x = mean + a.d;              // [r]
-    __shared__ float bd[kAppThreads];
-    __shared__ int bj[kAppThreads];
-    __shared__ int slot_sh;
-    const int u = blockIdx.x;
+    const int u = blockIdx.y;
+    const int64_t b = a.first_block + blockIdx.x;
     const int64_t bseq = u / a.hkv;
     const int h = u % a.hkv;
     for (int e = threadIdx.x; e < a.d * a.r; e += kAppThreads) Ws[e] = a.W[e];
+    for (int k = threadIdx.x; k < a.d; k += kAppThreads) {
+        const T* p = K + ((bseq * a.ld_tokens + b * a.pool) * a.hkv + h) * a.d + k;
+        mean[k] = mean_of_rows(p, (int64_t)a.hkv * a.d, a.pool);
+    }
+    __syncthreads();
+    for (int o = threadIdx.x; o < a.r; o += kAppThreads)
+        a.Kl[((int64_t)u * a.nb_cap + b) * a.r + o] = latent_dot(mean, Ws, a.d, a.r, o);
+}
+
+// Nearest leaf, one chunk of leaves per CTA: blockIdx.x = chunk, blockIdx.y =
+// unit.  One warp per leaf row (lanes split the dims, fixed reduction order).
+__global__ __launch_bounds__(kAppThreads) void append_nearest_kernel(const AppArgs a) {
+    extern __shared__ float xs[];       // [n_new][r] latents of the new blocks
+    const int u = blockIdx.y;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    for (int e = threadIdx.x; e < a.n_new * a.r; e += kAppThreads)
+        xs[e] = a.Kl[((int64_t)u * a.nb_cap + a.first_block + e / a.r) * a.r + e % a.r];
+    __syncthreads();
     const float* cl = a.cent_leaf + (int64_t)u * a.L * a.r;
     const float scale = a.grid_log2 > 0 ? (float)(1 << a.grid_log2) : 1.f;
-    for (int64_t t = 0; t < a.n_new; ++t) {
-        const int64_t b = a.first_block + t;
-        __syncthreads();
-        for (int k = threadIdx.x; k < a.d; k += kAppThreads) {
-            const T* p = K + ((bseq * a.ld_tokens + b * a.pool) * a.hkv + h) * a.d + k;
-            mean[k] = mean_of_rows(p, (int64_t)a.hkv * a.d, a.pool);
-        }
-        __syncthreads();
-        for (int o = threadIdx.x; o < a.r; o += kAppThreads) {
-            const float v = latent_dot(mean, Ws, a.d, a.r, o);
-            x[o] = v;
-            a.Kl[((int64_t)u * a.nb_cap + b) * a.r + o] = v;
-        }
-        __syncthreads();
-        float best = INFINITY;
-        int bestj = 0x7fffffff;
-        for (int j = threadIdx.x; j < a.L; j += kAppThreads) {
+    const int j0 = blockIdx.x * kLeavesPerCta;
+    const int j1 = min(a.L, j0 + kLeavesPerCta);
+    for (int64_t nb = 0; nb < a.n_new; ++nb) {
+        const float* x = xs + nb * a.r;
+        unsigned long long best = ~0ull;
+        for (int j = j0 + warp; j < j1; j += kAppThreads / 32) {
             const float* c = cl + (int64_t)j * a.r;
-            float dist;
+            unsigned long long key;
             if (a.grid_log2 > 0) {
                 long long s = 0;
-                for (int e = 0; e < a.r; ++e) {
+                for (int e = lane; e < a.r; e += 32) {
                     const long long dd = (long long)(x[e] * scale) - (long long)(c[e] * scale);
                     s += dd * dd;
                 }
-                dist = (float)s;  // exact ordering preserved below via integer compare
-                // keep exactness: compare in integers by encoding into the float only when small
-                if (s >= (1LL << 24)) latch(a.err, kErrInexact);
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+                if (s >= (1ll << 43)) latch(a.err, kErrInexact);
+                key = ((unsigned long long)s << 20) | (unsigned)j;
             } else {
                 float s = 0.f;
-                for (int e = 0; e < a.r; ++e) {
+                for (int e = lane; e < a.r; e += 32) {
                     const float dd = __fsub_rn(x[e], c[e]);
                     s = __fmaf_rn(dd, dd, s);
                 }
-                dist = s;
+#pragma unroll
+                for (int o = 16; o >= 1; o >>= 1) s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, o));
+                // distances are >= 0, so their bit patterns order like the values
+                key = ((unsigned long long)__float_as_uint(s) << 32) | (unsigned)j;
             }
-            if (dist < best) { best = dist; bestj = j; }
+            best = key < best ? key : best;
         }
-        bd[threadIdx.x] = best;
-        bj[threadIdx.x] = bestj;
-        __syncthreads();
-        for (int w = kAppThreads / 2; w >= 1; w >>= 1) {
-            if (threadIdx.x < w) {
-                const float od = bd[threadIdx.x + w];
-                const int oj = bj[threadIdx.x + w];
-                if (od < bd[threadIdx.x] || (od == bd[threadIdx.x] && oj < bj[threadIdx.x])) {
-                    bd[threadIdx.x] = od;
-                    bj[threadIdx.x] = oj;
-                }
-            }
-            __syncthreads();
-        }
+        if (lane == 0 && best != ~0ull) atomicMin(a.best + (int64_t)u * a.n_new + nb, best);
+    }
+}
+
+// Ordered insertion of the new blocks of one unit.
+__global__ __launch_bounds__(kAppThreads) void append_insert_kernel(const AppArgs a) {
+    __shared__ int slot_sh;
+    const int u = blockIdx.x;
+    for (int64_t t = 0; t < a.n_new; ++t) {
+        const int64_t b = a.first_block + t;
         if (threadIdx.x == 0) {
-            const int leaf = bj[0];
-            const int64_t c = (int64_t)u * a.L + leaf;
-            const int cnt = a.leaf_cnt[c];
+            const unsigned long long key = a.best[(int64_t)u * a.n_new + t];
+            const int leaf = a.grid_log2 > 0 ? (int)(key & 0xFFFFFull) : (int)(key & 0xFFFFFFFFull);
             int slot = -1;
-            if (cnt < a.leaf_cap[c]) {
-                slot = a.leaf_start[c] + cnt;
-                a.blk[slot] = (int32_t)b;
-                a.leaf_cnt[c] = cnt + 1;
-                a.leaf_of_block[(int64_t)u * a.nb_cap + b] = leaf;
-                const int64_t start = b * a.pool;
-                if (start >= a.sink) {
-                    int node = leaf;
-                    for (int l = a.levels - 1; l >= 0; --l) {
-                        int64_t* mp = a.minpos[l] + (int64_t)u * a.n_l[l] + node;
-                        if (start < *mp) *mp = start;
-                        int64_t* omp = a.ord_mp[l] + (int64_t)u * a.n_l[l] + a.ord_pos[l][(int64_t)u * a.n_l[l] + node];
-                        if (start < *omp) *omp = start;
-                        if (l > 0) node = a.parent[l][(int64_t)u * a.n_l[l] + node];
-                    }
-                }
-            } else {
-                latch(a.err, kErrCapacity);
+            if (key == ~0ull || leaf < 0 || leaf >= a.L) {
+                latch(a.err, kErrDevice);
                 a.leaf_of_block[(int64_t)u * a.nb_cap + b] = -1;
+            } else {
+                const int64_t c = (int64_t)u * a.L + leaf;
+                const int cnt = a.leaf_cnt[c];
+                if (cnt < a.leaf_cap[c]) {
+                    slot = a.leaf_start[c] + cnt;
+                    a.blk[slot] = (int32_t)b;
+                    a.leaf_cnt[c] = cnt + 1;
+                    a.leaf_of_block[(int64_t)u * a.nb_cap + b] = leaf;
+                    const int64_t start = b * a.pool;
+                    if (start >= a.sink) {
+                        int node = leaf;
+                        for (int l = a.levels - 1; l >= 0; --l) {
+                            const int64_t base = (int64_t)u * a.n_l[l];
+                            int64_t* mp = a.minpos[l] + base + node;
+                            if (start < *mp) *mp = start;
+                            int64_t* omp = a.ord_mp[l] + base + a.ord_pos[l][base + node];
+                            if (start < *omp) *omp = start;
+                            if (l > 0) node = a.parent[l][base + node];
+                        }
+                    }
+                } else {
+                    latch(a.err, kErrCapacity);
+                    a.leaf_of_block[(int64_t)u * a.nb_cap + b] = -1;
+                }
             }
             slot_sh = slot;
         }
         __syncthreads();
         const int slot = slot_sh;
         if (slot >= 0)
-            for (int o = threadIdx.x; o < a.r; o += kAppThreads) a.Klp[(int64_t)slot * a.r + o] = x[o];
+            for (int o = threadIdx.x; o < a.r; o += kAppThreads)
+                a.Klp[(int64_t)slot * a.r + o] = a.Kl[((int64_t)u * a.nb_cap + b) * a.r + o];
+        __syncthreads();
     }
 }
 
@@ -172,21 +192,40 @@ int launch_append(lsa_index* ix, const void* K, int64_t first_block, int64_t n_n
     a.first_block = first_block;
     a.n_new = n_new_blocks;
     a.err = ix->err;
-    const size_t smem = (size_t)(p.d * p.r + p.d + p.r) * sizeof(float);
+    const size_t smem_lat = (size_t)(p.d * p.r + p.d) * sizeof(float);
+    const size_t smem_near = (size_t)n_new_blocks * p.r * sizeof(float);
+    if (smem_near > 200 * 1024) return LSA_ERR_INVALID_ARG;
+    Arena scratch;
+    scratch.async = true;
+    scratch.stream = s;
+    a.best = scratch.alloc<unsigned long long>(ix->units * n_new_blocks);
+    if (scratch.status != LSA_OK) return scratch.status;
+    cudaMemsetAsync(a.best, 0xff, ix->units * n_new_blocks * sizeof(unsigned long long), s);
     cudaError_t e;
+    dim3 glat((unsigned)n_new_blocks, (unsigned)ix->units);
     if (p.dtype == LSA_F32) {
-        e = cudaFuncSetAttribute(append_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = cudaFuncSetAttribute(append_latent_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem_lat);
         if (e != cudaSuccess) return cuda_status(e);
         note_launch();
-        append_kernel<float><<<(unsigned)ix->units, kAppThreads, smem, s>>>((const float*)K, a);
+        append_latent_kernel<float><<<glat, kAppThreads, smem_lat, s>>>((const float*)K, a);
     } else {
-        e = cudaFuncSetAttribute(append_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem);
+        e = cudaFuncSetAttribute(append_latent_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem_lat);
         if (e != cudaSuccess) return cuda_status(e);
         note_launch();
-        append_kernel<__nv_bfloat16><<<(unsigned)ix->units, kAppThreads, smem, s>>>((const __nv_bfloat16*)K, a);
+        append_latent_kernel<__nv_bfloat16><<<glat, kAppThreads, smem_lat, s>>>((const __nv_bfloat16*)K, a);
     }
-    return cuda_status(cudaGetLastError());
+    e = cudaFuncSetAttribute(append_nearest_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_near);
+    if (e != cudaSuccess) return cuda_status(e);
+    dim3 gnear((unsigned)((ix->L + kLeavesPerCta - 1) / kLeavesPerCta), (unsigned)ix->units);
+    note_launch();
+    append_nearest_kernel<<<gnear, kAppThreads, smem_near, s>>>(a);
+    note_launch();
+    append_insert_kernel<<<(unsigned)ix->units, kAppThreads, 0, s>>>(a);
+    const int st = cuda_status(cudaGetLastError());
+    scratch.release();
+    return st;
 }
 
 }  // namespace lsa

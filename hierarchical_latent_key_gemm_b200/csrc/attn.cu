@@ -304,33 +304,40 @@ __global__ __launch_bounds__(kAttThreads) void attn_bf16_kernel(
 }
 
 // Merge the nsplit partials of every (query, KV head) row list by their
-// maxima: O = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s.
+// maxima: O = sum_s 2^(m_s - M) acc_s / sum_s 2^(m_s - M) l_s.  One CTA per
+// (row list, query head), one thread per output column.
 template <int D>
-__global__ __launch_bounds__(kAttThreads) void attn_combine_kernel(const float* __restrict__ part, int nsplit,
-                                                                    int64_t nq, int hq, int hkv,
-                                                                    __nv_bfloat16* __restrict__ O,
-                                                                    float* __restrict__ lse) {
-    const int G = hq / hkv;
-    const int64_t row = blockIdx.x;  // (b * nq + qi) * hkv + h
+__global__ __launch_bounds__(D) void attn_combine_kernel(const float* __restrict__ part, int nsplit, int G, int hq,
+                                                         int hkv, __nv_bfloat16* __restrict__ O,
+                                                         float* __restrict__ lse) {
+    __shared__ float wsp[32];
+    __shared__ float Msh, Lsh;
+    const int64_t row = blockIdx.x / G;  // (b * nq + qi) * hkv + h
+    const int r = blockIdx.x % G;
     const int h = (int)(row % hkv);
-    const int64_t bq = row / hkv;    // b * nq + qi
-    for (int e = threadIdx.x; e < G * D; e += blockDim.x) {
-        const int r = e / D, c = e % D;
-        const float* p0 = part + (row * nsplit * G + r) * (D + 2);
-        float M = -INFINITY;
-        for (int sp = 0; sp < nsplit; ++sp) M = fmaxf(M, p0[(int64_t)sp * G * (D + 2) + D]);
-        float Ls = 0.f, acc = 0.f;
-        if (M != -INFINITY) {
-            for (int sp = 0; sp < nsplit; ++sp) {
-                const float* pp = p0 + (int64_t)sp * G * (D + 2);
-                const float f = exp2f(pp[D] - M);
-                Ls += f * pp[D + 1];
-                acc += f * pp[c];
-            }
-        }
-        O[(bq * hq + (int64_t)h * G + r) * D + c] = __float2bfloat16_rn(Ls > 0.f ? acc / Ls : 0.f);
-        if (c == 0 && lse) lse[bq * hq + (int64_t)h * G + r] = Ls > 0.f ? (M + log2f(Ls)) * 0.69314718055994531f : -INFINITY;
+    const int64_t bq = row / hkv;        // b * nq + qi
+    const int64_t stride = (int64_t)G * (D + 2);
+    const float* p0 = part + (row * nsplit * G + r) * (D + 2);
+    if (threadIdx.x < 32) {
+        const int sp = threadIdx.x;
+        const float m = sp < nsplit ? p0[sp * stride + D] : -INFINITY;
+        float M = m;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+        const float w = (M == -INFINITY || sp >= nsplit) ? 0.f : exp2f(m - M);
+        float L = sp < nsplit ? w * p0[sp * stride + D + 1] : 0.f;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+        wsp[sp] = w;
+        if (sp == 0) { Msh = M; Lsh = L; }
     }
+    __syncthreads();
+    const int c = threadIdx.x;
+    float acc = 0.f;
+    for (int sp = 0; sp < nsplit; ++sp) acc += wsp[sp] * p0[sp * stride + c];
+    const float Ls = Lsh;
+    O[(bq * hq + (int64_t)h * G + r) * D + c] = __float2bfloat16_rn(Ls > 0.f ? acc / Ls : 0.f);
+    if (c == 0 && lse) lse[bq * hq + (int64_t)h * G + r] = Ls > 0.f ? (Msh + log2f(Ls)) * 0.69314718055994531f : -INFINITY;
 }
 
 template <int D, int GMAX>
@@ -451,8 +458,8 @@ int launch_bf16(const void* Q, const void* K, const void* V, const int32_t* idx,
         ld_tokens, (__nv_bfloat16*)O, lse, err, scale_log2, nsplit, part);
     if (nsplit > 1) {
         note_launch();
-        attn_combine_kernel<D><<<(unsigned)rows_n, kAttThreads, 0, s>>>(part, nsplit, nq, hq, hkv,
-                                                                       (__nv_bfloat16*)O, lse);
+        attn_combine_kernel<D><<<(unsigned)(rows_n * (hq / hkv)), D, 0, s>>>(part, nsplit, hq / hkv, hq, hkv,
+                                                                             (__nv_bfloat16*)O, lse);
     }
     const int st = cuda_status(cudaGetLastError());
     scratch.release();

@@ -198,6 +198,7 @@ __device__ __forceinline__ int find_owner(const int* pre, int nk, int t) {
 // THREADS = kSelThreads for large grids; small grids (decode: a few queries)
 // give each (query, KV head) kWideThreads so the few CTAs use more of the SM.
 constexpr int kWideThreads = 1024;
+constexpr int kWideCap = 8192;
 
 template <int R, bool FULL, int THREADS>
 __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BLOCKS : 1) void select_kernel(
@@ -420,22 +421,35 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
     }
     const int nsel = sh.count;
 
-    // ascending block ids (bitonic sort, padded to a power of two)
-    int M = 1;
-    while (M < nsel) M <<= 1;
+    // ascending block ids
     int* arr = bib[cur ^ 1];
-    for (int e = threadIdx.x; e < M; e += blockDim.x) arr[e] = e < nsel ? bib[cur][e] : INT32_MAX;
-    __syncthreads();
-    for (int size = 2; size <= M; size <<= 1) {
-        for (int stride = size >> 1; stride > 0; stride >>= 1) {
-            for (int t = threadIdx.x; t < (M >> 1); t += blockDim.x) {
-                const int i = 2 * stride * (t / stride) + (t % stride);
-                const int j = i + stride;
-                const bool asc = (i & size) == 0;
-                const int x = arr[i], y = arr[j];
-                if ((x > y) == asc) { arr[i] = y; arr[j] = x; }
+    if (THREADS >= 512) {
+        // wide CTAs: rank sort (each id counts the smaller ones), one barrier
+        const int* src = bib[cur];
+        for (int e = threadIdx.x; e < nsel; e += THREADS) {
+            const int x = src[e];
+            int rank = 0;
+            for (int j = 0; j < nsel; ++j) rank += src[j] < x;
+            arr[rank] = x;
+        }
+        __syncthreads();
+    } else {
+        // bitonic sort, padded to a power of two
+        int M = 1;
+        while (M < nsel) M <<= 1;
+        for (int e = threadIdx.x; e < M; e += blockDim.x) arr[e] = e < nsel ? bib[cur][e] : INT32_MAX;
+        __syncthreads();
+        for (int size = 2; size <= M; size <<= 1) {
+            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                for (int t = threadIdx.x; t < (M >> 1); t += blockDim.x) {
+                    const int i = 2 * stride * (t / stride) + (t % stride);
+                    const int j = i + stride;
+                    const bool asc = (i & size) == 0;
+                    const int x = arr[i], y = arr[j];
+                    if ((x > y) == asc) { arr[i] = y; arr[j] = x; }
+                }
+                __syncthreads();
             }
-            __syncthreads();
         }
     }
 
@@ -472,7 +486,13 @@ int launch_select_r(const SelArgs& a, int64_t nq, int64_t units, bool fullscan, 
     int dev = 0, sms = 148;
     cudaGetDevice(&dev);
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    if (nq * units < 2 * (int64_t)sms) return launch_select_t<R, kWideThreads>(a, nq, units, fullscan, s);
+    if (nq * units < 2 * (int64_t)sms) {
+        // one CTA per SM at most: a buffer that holds a whole level (fewer
+        // compaction rounds), within the 227 KB a CTA may use
+        SelArgs w = a;
+        while (w.cap < kWideCap && (size_t)(2 * w.cap) * 24 + (size_t)(3 * w.beam + 1) * 4 <= 200 * 1024) w.cap *= 2;
+        return launch_select_t<R, kWideThreads>(w, nq, units, fullscan, s);
+    }
     return launch_select_t<R, kSelThreads>(a, nq, units, fullscan, s);
 }
 
