@@ -207,7 +207,7 @@ def run_ours(args):
         lsa.lsa_select(ix, sp, Q, idx=idx, cnt=cnt, max_sel=max_sel, q_pos0=q0)
         if ev:
             ev[2].record()
-        lsa.lsa_sparse_attn(Q, K, V, idx, cnt, w.hkv, O=O, lse=lse)
+        lsa.lsa_sparse_attn_banded(Q, K, V, idx, cnt, w.hkv, w.sink, w.window, q_pos0=q0, O=O, lse=lse)
         if ev:
             ev[3].record()
         return ix
@@ -375,7 +375,7 @@ def run_e2e(args, w, inp, bp, sp, idx, cnt, O, lse, dev, world):
         dW.copy_(hW, non_blocking=True)
         ix = lsa.lsa_build_index(bp, dK, dW)
         lsa.lsa_select(ix, sp, dQ, idx=idx, cnt=cnt, max_sel=idx.shape[-1])
-        lsa.lsa_sparse_attn(dQ, dK, dV, idx, cnt, w.hkv, O=O, lse=lse)
+        lsa.lsa_sparse_attn_banded(dQ, dK, dV, idx, cnt, w.hkv, w.sink, w.window, O=O, lse=lse)
         hO.copy_(O, non_blocking=True)
         return ix
 

@@ -399,6 +399,28 @@ int lsa_sparse_attn(const void* Q, const void* K, const void* V, const int32_t* 
                               global_err_word(), as_stream(stream));
 }
 
+int lsa_sparse_attn_banded(const void* Q, const void* K, const void* V, const int32_t* idx, const int32_t* cnt,
+                           int64_t batch, int64_t nq, int64_t q_pos0, int32_t hq, int32_t hkv, int32_t d,
+                           int32_t dtype, int32_t max_sel, int64_t ld_tokens, int32_t sink, int32_t window, void* O,
+                           float* lse, void* stream) {
+    if (batch < 1 || nq < 0 || hkv < 1 || hq < hkv || hq % hkv || !valid_d(d) || max_sel < 1 || ld_tokens < 1)
+        return LSA_ERR_INVALID_ARG;
+    if (dtype != LSA_F32 && dtype != LSA_BF16) return LSA_ERR_INVALID_ARG;
+    if (batch * hkv > 65535 || nq > INT32_MAX) return LSA_ERR_INVALID_ARG;
+    if (q_pos0 < 0 || q_pos0 + nq > ld_tokens || sink < 0 || window < 1) return LSA_ERR_INVALID_ARG;
+    if (nq == 0) return LSA_OK;
+    if (!is_device_ptr(Q) || !is_device_ptr(K) || !is_device_ptr(V) || !is_device_ptr(idx) || !is_device_ptr(cnt) ||
+        !is_device_ptr(O))
+        return LSA_ERR_INVALID_ARG;
+    if (lse && !is_device_ptr(lse)) return LSA_ERR_INVALID_ARG;
+    const int G = hq / hkv;
+    if (dtype == LSA_BF16 && (G == 1 || G == 2 || G == 4 || G == 8 || G == 16))
+        return launch_banded_attn(Q, K, V, idx, cnt, batch, nq, q_pos0, hq, hkv, d, max_sel, ld_tokens, sink, window,
+                                  O, lse, global_err_word(), as_stream(stream));
+    return launch_sparse_attn(Q, K, V, idx, cnt, batch, nq, hq, hkv, d, dtype, max_sel, ld_tokens, O, lse,
+                              global_err_word(), as_stream(stream));
+}
+
 int lsa_append(lsa_index* index, const void* K, int64_t n_new, void* stream) {
     if (!live(index) || n_new < 0) return LSA_ERR_INVALID_ARG;
     const lsa_build_params& p = index->p;

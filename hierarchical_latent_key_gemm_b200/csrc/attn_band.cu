@@ -1,0 +1,561 @@
+// Exact softmax attention over the selection, split by where the rows come
+// from.  The selection of query i is the union of the attention sink
+// [0, min(S, i+1)), the chosen long-range blocks, and the local window
+// [max(0, i-W+1), i] (LSA explainer, "How does LSA work?" step 3: the kept
+// long-range keys plus the sink and a local window; the attention kernel itself
+// is unchanged).  Sink and window rows are the same for neighbouring queries,
+// so they are read once per tile of consecutive queries instead of once per
+// query:
+//
+//   attn_band_kernel    dense tiles: 128 (query, head) rows per CTA against the
+//                       contiguous key band [0, S) and [i0-W+1, i1], with the
+//                       per-row mask j <= i && (j < S || j >= i-W+1); writes an
+//                       unnormalised partial (acc, running max, sum of weights).
+//   attn_gather_kernel  one warp per (query, KV head): the long-range entries of
+//                       the row list only, starting from the band partial, and
+//                       writes the normalised output.
+//
+// Both parts are the same softmax over disjoint key sets, merged by their
+// maxima, so the result equals attention over the whole list up to rounding.
+// A row list that does not have the selection form (checked in O(1) per row:
+// rows are ascending without repeats, the first min(S, i+1) entries are the
+// sink, the last ones the window) is processed whole by the gather kernel
+// with the band partial ignored, so any ascending list gives exact attention.
+//
+// Gather kernel tensor-core layout: keys on the M side (16 per slice), the G
+// heads of the group on N (n8 tiles), so no head padding to 16 rows:
+// S^T = K_slice Q^T, then O^T += V^T P^T with P^T moved into B-operand order by
+// movmatrix.  P is split into two bf16 terms (hi + lo) as in the other paths.
+#include <algorithm>
+
+#include "lsa_internal.cuh"
+#include "warp_mma.cuh"
+
+namespace lsa {
+namespace {
+
+constexpr int kBandThreads = 256;   // 8 warps x 16 rows
+constexpr int kBandRows = 128;      // (query, head) rows per CTA
+constexpr int kBandTile = 64;       // keys per pipeline stage
+constexpr int kBandStages = 3;
+
+constexpr int kGatWarps = 4;        // queries per CTA (one warp each)
+constexpr int kGatSlice = 16;       // keys per slice
+constexpr int kGatStages = 3;
+
+struct BandArgs {
+    const __nv_bfloat16* Q;
+    const __nv_bfloat16* K;
+    const __nv_bfloat16* V;
+    int64_t nq, q_pos0, ld_tokens;
+    int hq, hkv, sink, window;
+    float scale_log2;
+    float* part_o;    // [batch*nq*hq][D] unnormalised sum of p * v
+    float2* part_ml;  // [batch*nq*hq] (running max in log2 units, sum of weights)
+};
+
+template <int D, int G>
+__global__ __launch_bounds__(kBandThreads, 1) void attn_band_kernel(const BandArgs a) {
+    constexpr int CH = D / 8;
+    constexpr int QT = kBandRows / G;   // queries per CTA
+    constexpr int QW = 16 / G;          // queries per warp
+    constexpr int TILE_BYTES = kBandTile * D * 2;
+    extern __shared__ __align__(128) unsigned char smem[];
+    unsigned char* Ks = smem;                                  // [stages][64][D]
+    unsigned char* Vs = smem + kBandStages * TILE_BYTES;       // [stages][64][D]
+    unsigned char* Qs = smem + 2 * kBandStages * TILE_BYTES;   // [128][D]
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int u = blockIdx.y;
+    const int64_t b = u / a.hkv;
+    const int h = u % a.hkv;
+    const int64_t q0 = (int64_t)blockIdx.x * QT;
+    const int64_t qlast = min(a.nq, q0 + QT) - 1;
+    const int64_t i0 = a.q_pos0 + q0, i1 = a.q_pos0 + qlast;
+    // key segments: sink [0, s_end) and window [w_beg, w_end)
+    const int64_t s_end = min((int64_t)a.sink, i1 + 1);
+    const int64_t w_beg = max((int64_t)a.sink, i0 - a.window + 1);
+    const int64_t w_end = i1 + 1;
+    const int nt_s = (int)((s_end + kBandTile - 1) / kBandTile);
+    const int nt_w = w_end > w_beg ? (int)((w_end - w_beg + kBandTile - 1) / kBandTile) : 0;
+    const int ntile = nt_s + nt_w;
+    auto tile_range = [&](int t, int64_t& jb, int64_t& je) {
+        if (t < nt_s) {
+            jb = (int64_t)t * kBandTile;
+            je = min(jb + kBandTile, s_end);
+        } else {
+            jb = w_beg + (int64_t)(t - nt_s) * kBandTile;
+            je = min(jb + kBandTile, w_end);
+        }
+    };
+
+    // Q rows: row r = (query q0 + r / G, head r % G); rows past nq are zero
+    const uint32_t qsb = smem_u32(Qs);
+    for (int e = tid; e < kBandRows * CH; e += kBandThreads) {
+        const int r = e / CH, c = e % CH;
+        const int64_t q = q0 + r / G;
+        const bool ok = q < a.nq;
+        const __nv_bfloat16* src = a.Q + (((b * a.nq + (ok ? q : 0)) * a.hq + (int64_t)h * G + r % G) * D + c * 8);
+        cp_async16(qsb + swz<D>(r, c), src, ok ? 16 : 0);
+    }
+    cp_async_commit();
+
+    const __nv_bfloat16* kbase = a.K + (b * a.ld_tokens * a.hkv + h) * D;
+    const __nv_bfloat16* vbase = a.V + (b * a.ld_tokens * a.hkv + h) * D;
+    auto load_tile = [&](int t) {
+        int64_t jb, je;
+        tile_range(t, jb, je);
+        const int st = t % kBandStages;
+        const uint32_t kb = smem_u32(Ks + st * TILE_BYTES), vb = smem_u32(Vs + st * TILE_BYTES);
+        for (int e = tid; e < kBandTile * CH; e += kBandThreads) {
+            const int r = e / CH, c = e % CH;
+            const int64_t j = jb + r;
+            const bool ok = j < je;
+            const int64_t off = (ok ? j : 0) * a.hkv * D + c * 8;
+            cp_async16(kb + swz<D>(r, c), kbase + off, ok ? 16 : 0);
+            cp_async16(vb + swz<D>(r, c), vbase + off, ok ? 16 : 0);
+        }
+    };
+#pragma unroll
+    for (int t = 0; t < kBandStages - 1; ++t) {
+        if (t < ntile) load_tile(t);
+        cp_async_commit();
+    }
+    cp_async_wait<kBandStages - 1>();   // the Q group
+    __syncthreads();
+
+    uint32_t qa[D / 16][4];
+    {
+        const int r = warp * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+        for (int kt = 0; kt < D / 16; ++kt) ldsm_x4(qsb + swz<D>(r, 2 * kt + (lane >> 4)), qa[kt][0], qa[kt][1], qa[kt][2], qa[kt][3]);
+    }
+    // this thread's two rows and their query positions
+    const int r0 = warp * 16 + (lane >> 2), r1 = r0 + 8;
+    const int64_t pa = i0 + r0 / G, pb = i0 + r1 / G;
+    const bool va = q0 + r0 / G <= qlast, vb_ = q0 + r1 / G <= qlast;
+    const int64_t wlo = i0 + warp * QW, whi = min(i0 + warp * QW + QW - 1, i1);
+    const bool warp_live = q0 + warp * QW <= qlast;
+
+    float o[D / 8][4];
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+
+    for (int t = 0; t < ntile; ++t) {
+        cp_async_wait<kBandStages - 2>();
+        __syncthreads();
+        if (t + kBandStages - 1 < ntile) load_tile(t + kBandStages - 1);
+        cp_async_commit();
+        int64_t jb, je;
+        tile_range(t, jb, je);
+        const bool sink_tile = t < nt_s;
+        // does any (row, key) of this warp survive the mask?
+        const bool live = warp_live && jb <= whi && (sink_tile || je - 1 >= wlo - a.window + 1);
+        if (!live) continue;
+        const bool full = je - jb == kBandTile && je - 1 <= wlo && (sink_tile || jb >= whi - a.window + 1) &&
+                          q0 + warp * QW + QW - 1 <= qlast;
+        const int st = t % kBandStages;
+        const uint32_t kb = smem_u32(Ks + st * TILE_BYTES), vb = smem_u32(Vs + st * TILE_BYTES);
+        float s[8][4];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
+#pragma unroll
+        for (int np = 0; np < 4; ++np) {
+            const int kr = np * 16 + (lane & 7) + 8 * (lane >> 4);
+#pragma unroll
+            for (int kt = 0; kt < D / 16; ++kt) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4(kb + swz<D>(kr, 2 * kt + ((lane >> 3) & 1)), b0, b1, b2, b3);
+                mma_bf16(s[2 * np], qa[kt], b0, b1);
+                mma_bf16(s[2 * np + 1], qa[kt], b2, b3);
+            }
+        }
+        // scale and mask: key j = jb + 8 * nt + 2 * (lane & 3) + (e & 1)
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                float x = s[nt][e] * a.scale_log2;
+                if (!full) {
+                    const int64_t j = jb + 8 * nt + 2 * (lane & 3) + (e & 1);
+                    const int64_t i = e < 2 ? pa : pb;
+                    const bool ok = (e < 2 ? va : vb_) && j < je && j <= i && (sink_tile || j >= i - a.window + 1);
+                    x = ok ? x : -INFINITY;
+                }
+                s[nt][e] = x;
+            }
+        }
+        float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            mx0 = fmaxf(mx0, fmaxf(s[nt][0], s[nt][1]));
+            mx1 = fmaxf(mx1, fmaxf(s[nt][2], s[nt][3]));
+        }
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
+        const float al0 = (mn0 == -INFINITY) ? 1.f : exp2f(m0 - mn0);
+        const float al1 = (mn1 == -INFINITY) ? 1.f : exp2f(m1 - mn1);
+        float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+        for (int nt = 0; nt < 8; ++nt) {
+            s[nt][0] = (mn0 == -INFINITY) ? 0.f : exp2f(s[nt][0] - mn0);
+            s[nt][1] = (mn0 == -INFINITY) ? 0.f : exp2f(s[nt][1] - mn0);
+            s[nt][2] = (mn1 == -INFINITY) ? 0.f : exp2f(s[nt][2] - mn1);
+            s[nt][3] = (mn1 == -INFINITY) ? 0.f : exp2f(s[nt][3] - mn1);
+            ls0 += s[nt][0] + s[nt][1];
+            ls1 += s[nt][2] + s[nt][3];
+        }
+        l0 = l0 * al0 + ls0;
+        l1 = l1 * al1 + ls1;
+        m0 = mn0;
+        m1 = mn1;
+        if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) {
+                o[i][0] *= al0; o[i][1] *= al0;
+                o[i][2] *= al1; o[i][3] *= al1;
+            }
+        }
+        // O += P V, 16 keys per k step, P = hi + lo
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) {
+            uint32_t ph[4], pl[4];
+            split_pack(s[2 * kk][0], s[2 * kk][1], ph[0], pl[0]);
+            split_pack(s[2 * kk][2], s[2 * kk][3], ph[1], pl[1]);
+            split_pack(s[2 * kk + 1][0], s[2 * kk + 1][1], ph[2], pl[2]);
+            split_pack(s[2 * kk + 1][2], s[2 * kk + 1][3], ph[3], pl[3]);
+            const int vr = kk * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+            for (int nt = 0; nt < D / 8; nt += 2) {
+                uint32_t b0, b1, b2, b3;
+                ldsm_x4_t(vb + swz<D>(vr, nt + (lane >> 4)), b0, b1, b2, b3);
+                mma_bf16(o[nt], ph, b0, b1);
+                mma_bf16(o[nt + 1], ph, b2, b3);
+                mma_bf16(o[nt], pl, b0, b1);
+                mma_bf16(o[nt + 1], pl, b2, b3);
+            }
+        }
+    }
+    cp_async_wait<0>();
+
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    const int64_t ga = ((b * a.nq + q0 + r0 / G) * a.hq + (int64_t)h * G + r0 % G);
+    const int64_t gb = ((b * a.nq + q0 + r1 / G) * a.hq + (int64_t)h * G + r1 % G);
+#pragma unroll
+    for (int nt = 0; nt < D / 8; ++nt) {
+        const int c = nt * 8 + 2 * (lane & 3);
+        if (va) *reinterpret_cast<float2*>(a.part_o + ga * D + c) = make_float2(o[nt][0], o[nt][1]);
+        if (vb_) *reinterpret_cast<float2*>(a.part_o + gb * D + c) = make_float2(o[nt][2], o[nt][3]);
+    }
+    if ((lane & 3) == 0) {
+        if (va) a.part_ml[ga] = make_float2(m0, l0);
+        if (vb_) a.part_ml[gb] = make_float2(m1, l1);
+    }
+}
+
+struct GatherArgs {
+    const __nv_bfloat16* Q;
+    const __nv_bfloat16* K;
+    const __nv_bfloat16* V;
+    const int32_t* idx;
+    const int32_t* cnt;
+    int64_t nq, q_pos0, ld_tokens;
+    int hq, hkv, max_sel, sink, window;
+    float scale_log2;
+    const float* part_o;
+    const float2* part_ml;
+    __nv_bfloat16* O;
+    float* lse;
+    int32_t* err;
+};
+
+// NT = n8 tiles of heads (G <= 8 * NT; heads past G are zero and dropped)
+template <int D, int NT>
+__global__ __launch_bounds__(kGatWarps * 32) void attn_gather_kernel(const GatherArgs a) {
+    constexpr int CH = D / 8;
+    constexpr int SLICE_BYTES = kGatSlice * D * 2;
+    constexpr int RPL = kGatSlice * CH / 32;   // rows of a slice each lane copies
+    constexpr int RSTEP = 32 / CH;
+    extern __shared__ __align__(128) unsigned char smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    unsigned char* Ks = smem + warp * (2 * kGatStages * SLICE_BYTES);   // [stages][16][D]
+    unsigned char* Vs = Ks + kGatStages * SLICE_BYTES;
+    // per stage: bit k set when key k of the slice is a real token
+    uint32_t* vmask = reinterpret_cast<uint32_t*>(smem + kGatWarps * 2 * kGatStages * SLICE_BYTES) + warp * kGatStages;
+    const int G = a.hq / a.hkv;
+    const int u = blockIdx.y;
+    const int64_t b = u / a.hkv;
+    const int h = u % a.hkv;
+    const int64_t qi = (int64_t)blockIdx.x * kGatWarps + warp;
+    if (qi >= a.nq) return;   // warp-uniform; the kernel has no CTA barrier
+    const int64_t i = a.q_pos0 + qi;
+    const int64_t row = (b * a.nq + qi) * a.hkv + h;
+    int n = a.cnt[row];
+    if (n < 0 || n > a.max_sel) {
+        if (lane == 0) latch(a.err, kErrDevice);
+        n = n < 0 ? 0 : a.max_sel;
+    }
+    const int32_t* ir = a.idx + row * a.max_sel;
+
+    // does the row have the selection form?
+    const int ns = (int)min((int64_t)a.sink, i + 1);
+    const int nw = i >= a.sink ? (int)min(i - a.sink + 1, (int64_t)a.window) : 0;
+    bool form = n >= ns + nw;
+    if (form && ns > 0) form = __ldg(ir) == 0 && __ldg(ir + ns - 1) == ns - 1;
+    if (form && nw > 0) form = __ldg(ir + n - 1) == i && __ldg(ir + n - nw) == i - nw + 1;
+    if (form && n - nw > ns) form = __ldg(ir + ns) >= a.sink && __ldg(ir + n - nw - 1) <= i - a.window;
+    const int pbeg = form ? ns : 0, pend = form ? n - nw : n;
+
+    // Q^T as B fragments: head = 8 nt + lane/4, dims 16 kt + 2 (lane%4) (+8)
+    const int64_t qrow0 = (b * a.nq + qi) * a.hq + (int64_t)h * G;
+    uint32_t qb[D / 16][NT][2];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+        const int hh = nt * 8 + (lane >> 2);
+        const uint32_t* qp = reinterpret_cast<const uint32_t*>(a.Q + (qrow0 + (hh < G ? hh : 0)) * D);
+#pragma unroll
+        for (int kt = 0; kt < D / 16; ++kt) {
+            const int dd = 16 * kt + 2 * (lane & 3);
+            qb[kt][nt][0] = hh < G ? __ldg(qp + dd / 2) : 0u;
+            qb[kt][nt][1] = hh < G ? __ldg(qp + dd / 2 + 4) : 0u;
+        }
+    }
+
+    // state: this thread's heads hA = 8 nt + 2 (lane%4), hB = hA + 1; O^T rows
+    // (dims) 16 mt + lane/4 and + 8
+    float m[NT][2], l[NT][2], ot[D / 16][NT][4];
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            const int hh = nt * 8 + 2 * (lane & 3) + c;
+            float mm = -INFINITY, ll = 0.f;
+            if (form && hh < G) {
+                const float2 ml = a.part_ml[qrow0 + hh];
+                mm = ml.x;
+                ll = lane < 4 ? ml.y : 0.f;   // summed over the 8 key lanes at the end
+            }
+            m[nt][c] = mm;
+            l[nt][c] = ll;
+#pragma unroll
+            for (int mt = 0; mt < D / 16; ++mt) {
+                float v0 = 0.f, v1 = 0.f;
+                if (form && hh < G) {
+                    const float* po = a.part_o + (qrow0 + hh) * D + 16 * mt + (lane >> 2);
+                    v0 = po[0];
+                    v1 = po[8];
+                }
+                ot[mt][nt][c] = v0;
+                ot[mt][nt][2 + c] = v1;
+            }
+        }
+    }
+
+    const int nslice = (pend - pbeg + kGatSlice - 1) / kGatSlice;
+    const __nv_bfloat16* kbase = a.K + (b * a.ld_tokens * a.hkv + h) * D;
+    const __nv_bfloat16* vbase = a.V + (b * a.ld_tokens * a.hkv + h) * D;
+    auto fetch_tok = [&](int s) -> int {
+        const int p = pbeg + s * kGatSlice + lane;
+        return (lane < kGatSlice && s < nslice && p < pend) ? __ldg(ir + p) : -1;
+    };
+    auto load_slice = [&](int s, int tok_l) {
+        const int st = s % kGatStages;
+        const uint32_t kb = smem_u32(Ks + st * SLICE_BYTES), vb = smem_u32(Vs + st * SLICE_BYTES);
+        const int c = lane % CH;
+        const uint32_t live = __ballot_sync(0xffffffffu, tok_l >= 0 && tok_l < a.ld_tokens);
+        if (lane == 0) vmask[st] = live & 0xffffu;
+#pragma unroll
+        for (int k = 0; k < RPL; ++k) {
+            const int r = lane / CH + RSTEP * k;
+            int tok = __shfl_sync(0xffffffffu, tok_l, r);
+            if (tok >= a.ld_tokens || tok < -1) { latch(a.err, kErrDevice); tok = -1; }
+            const int64_t off = tok >= 0 ? (int64_t)tok * a.hkv * D + c * 8 : 0;
+            cp_async16(kb + swz<D>(r, c), kbase + off, tok >= 0 ? 16 : 0);
+            cp_async16(vb + swz<D>(r, c), vbase + off, tok >= 0 ? 16 : 0);
+        }
+    };
+    int tok_next = fetch_tok(0);
+#pragma unroll
+    for (int s = 0; s < kGatStages - 1; ++s) {
+        if (s < nslice) load_slice(s, tok_next);
+        cp_async_commit();
+        tok_next = fetch_tok(s + 1);
+    }
+
+    for (int s = 0; s < nslice; ++s) {
+        cp_async_wait<kGatStages - 2>();
+        __syncwarp();
+        if (s + kGatStages - 1 < nslice) load_slice(s + kGatStages - 1, tok_next);
+        cp_async_commit();
+        tok_next = fetch_tok(s + kGatStages);
+        const int st = s % kGatStages;
+        const uint32_t kb = smem_u32(Ks + st * SLICE_BYTES), vb = smem_u32(Vs + st * SLICE_BYTES);
+        // S^T = K_slice Q^T: rows = 16 keys, cols = heads
+        float sc[NT][4];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+        {
+            const int kr = (lane & 7) + 8 * ((lane >> 3) & 1);
+#pragma unroll
+            for (int kt = 0; kt < D / 16; ++kt) {
+                uint32_t ka[4];
+                ldsm_x4(kb + swz<D>(kr, 2 * kt + (lane >> 4)), ka[0], ka[1], ka[2], ka[3]);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma_bf16(sc[nt], ka, qb[kt][nt][0], qb[kt][nt][1]);
+            }
+        }
+        // keys lane/4 and lane/4 + 8 of the slice
+        const uint32_t vm = vmask[st];
+        const bool k0 = (vm >> (lane >> 2)) & 1u, k1 = (vm >> ((lane >> 2) + 8)) & 1u;
+        uint32_t bh[NT][2], bl[NT][2];
+#pragma unroll
+        for (int nt = 0; nt < NT; ++nt) {
+            const float x0 = k0 ? sc[nt][0] * a.scale_log2 : -INFINITY;   // (key, hA)
+            const float x1 = k0 ? sc[nt][1] * a.scale_log2 : -INFINITY;   // (key, hB)
+            const float x2 = k1 ? sc[nt][2] * a.scale_log2 : -INFINITY;   // (key+8, hA)
+            const float x3 = k1 ? sc[nt][3] * a.scale_log2 : -INFINITY;   // (key+8, hB)
+            float mA = fmaxf(x0, x2), mB = fmaxf(x1, x3);
+#pragma unroll
+            for (int o = 4; o <= 16; o <<= 1) {
+                mA = fmaxf(mA, __shfl_xor_sync(0xffffffffu, mA, o));
+                mB = fmaxf(mB, __shfl_xor_sync(0xffffffffu, mB, o));
+            }
+            const float nA = fmaxf(m[nt][0], mA), nB = fmaxf(m[nt][1], mB);
+            const float aA = (nA == -INFINITY) ? 1.f : exp2f(m[nt][0] - nA);
+            const float aB = (nB == -INFINITY) ? 1.f : exp2f(m[nt][1] - nB);
+            const float p0 = (nA == -INFINITY) ? 0.f : exp2f(x0 - nA);
+            const float p2 = (nA == -INFINITY) ? 0.f : exp2f(x2 - nA);
+            const float p1 = (nB == -INFINITY) ? 0.f : exp2f(x1 - nB);
+            const float p3 = (nB == -INFINITY) ? 0.f : exp2f(x3 - nB);
+            l[nt][0] = l[nt][0] * aA + (p0 + p2);
+            l[nt][1] = l[nt][1] * aB + (p1 + p3);
+            m[nt][0] = nA;
+            m[nt][1] = nB;
+            uint32_t h01, l01, h23, l23;
+            split_pack(p0, p1, h01, l01);   // row = key lane/4, cols = (hA, hB)
+            split_pack(p2, p3, h23, l23);   // row = key lane/4 + 8
+            bh[nt][0] = movmatrix_t(h01);
+            bh[nt][1] = movmatrix_t(h23);
+            bl[nt][0] = movmatrix_t(l01);
+            bl[nt][1] = movmatrix_t(l23);
+            if (__any_sync(0xffffffffu, aA != 1.f || aB != 1.f)) {
+#pragma unroll
+                for (int mt = 0; mt < D / 16; ++mt) {
+                    ot[mt][nt][0] *= aA; ot[mt][nt][1] *= aB;
+                    ot[mt][nt][2] *= aA; ot[mt][nt][3] *= aB;
+                }
+            }
+        }
+        // O^T += V^T P^T: rows = dims (16 per m tile), k = 16 keys
+        {
+            const int vr = (lane & 7) + 8 * (lane >> 4);
+#pragma unroll
+            for (int mt = 0; mt < D / 16; ++mt) {
+                uint32_t va[4];
+                ldsm_x4_t(vb + swz<D>(vr, 2 * mt + ((lane >> 3) & 1)), va[0], va[1], va[2], va[3]);
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    mma_bf16(ot[mt][nt], va, bh[nt][0], bh[nt][1]);
+                    mma_bf16(ot[mt][nt], va, bl[nt][0], bl[nt][1]);
+                }
+            }
+        }
+    }
+    cp_async_wait<0>();
+    __syncwarp();
+
+    // normalise and write: stage [G][D] bf16 in this warp's ring, then 16-byte stores
+    __nv_bfloat16* stage = reinterpret_cast<__nv_bfloat16*>(Ks);
+#pragma unroll
+    for (int nt = 0; nt < NT; ++nt) {
+#pragma unroll
+        for (int c = 0; c < 2; ++c) {
+            float ll = l[nt][c];
+#pragma unroll
+            for (int o = 4; o <= 16; o <<= 1) ll += __shfl_xor_sync(0xffffffffu, ll, o);
+            const int hh = nt * 8 + 2 * (lane & 3) + c;
+            const float inv = ll > 0.f ? 1.f / ll : 0.f;
+            if (hh < G) {
+#pragma unroll
+                for (int mt = 0; mt < D / 16; ++mt) {
+                    const int dd = 16 * mt + (lane >> 2);
+                    stage[hh * D + dd] = __float2bfloat16_rn(ot[mt][nt][c] * inv);
+                    stage[hh * D + dd + 8] = __float2bfloat16_rn(ot[mt][nt][2 + c] * inv);
+                }
+                if (lane < 4 && a.lse)
+                    a.lse[qrow0 + hh] = ll > 0.f ? (m[nt][c] + log2f(ll)) * 0.69314718055994531f : -INFINITY;
+            }
+        }
+    }
+    __syncwarp();
+    uint4* dst = reinterpret_cast<uint4*>(a.O + qrow0 * D);
+    const uint4* srcv = reinterpret_cast<const uint4*>(stage);
+    for (int e = lane; e < G * D / 8; e += 32) dst[e] = srcv[e];
+}
+
+template <int D, int G>
+int launch_band_g(const BandArgs& ba, const GatherArgs& ga, int64_t batch, cudaStream_t s) {
+    const size_t smem_band = (size_t)2 * kBandStages * kBandTile * D * 2 + (size_t)kBandRows * D * 2;
+    cudaError_t e = cudaFuncSetAttribute(attn_band_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem_band);
+    if (e != cudaSuccess) return cuda_status(e);
+    constexpr int NT = (G + 7) / 8;
+    const size_t smem_gat = (size_t)kGatWarps * 2 * kGatStages * kGatSlice * D * 2 + kGatWarps * kGatStages * 4;
+    e = cudaFuncSetAttribute(attn_gather_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_gat);
+    if (e != cudaSuccess) return cuda_status(e);
+    constexpr int QT = kBandRows / G;
+    const unsigned units = (unsigned)(batch * ba.hkv);
+    note_launch();
+    attn_band_kernel<D, G><<<dim3((unsigned)((ba.nq + QT - 1) / QT), units), kBandThreads, smem_band, s>>>(ba);
+    note_launch();
+    attn_gather_kernel<D, NT><<<dim3((unsigned)((ga.nq + kGatWarps - 1) / kGatWarps), units), kGatWarps * 32,
+                                 smem_gat, s>>>(ga);
+    return cuda_status(cudaGetLastError());
+}
+
+template <int D>
+int launch_band_d(int G, const BandArgs& ba, const GatherArgs& ga, int64_t batch, cudaStream_t s) {
+    switch (G) {
+        case 1: return launch_band_g<D, 1>(ba, ga, batch, s);
+        case 2: return launch_band_g<D, 2>(ba, ga, batch, s);
+        case 4: return launch_band_g<D, 4>(ba, ga, batch, s);
+        case 8: return launch_band_g<D, 8>(ba, ga, batch, s);
+        case 16: return launch_band_g<D, 16>(ba, ga, batch, s);
+        default: return LSA_ERR_INVALID_ARG;
+    }
+}
+
+}  // namespace
+
+int launch_banded_attn(const void* Q, const void* K, const void* V, const int32_t* idx, const int32_t* cnt,
+                       int64_t batch, int64_t nq, int64_t q_pos0, int hq, int hkv, int d, int max_sel,
+                       int64_t ld_tokens, int sink, int window, void* O, float* lse, int32_t* err, cudaStream_t s) {
+    if (nq <= 0 || batch <= 0) return LSA_OK;
+    const int G = hq / hkv;
+    const int64_t rows = batch * nq * hq;
+    Arena scratch;
+    scratch.async = true;
+    scratch.stream = s;
+    float* part_o = scratch.alloc<float>(rows * d);
+    float2* part_ml = scratch.alloc<float2>(rows);
+    if (scratch.status != LSA_OK) return scratch.status;
+    BandArgs ba{(const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, nq, q_pos0, ld_tokens,
+                hq, hkv, sink, window, 1.4426950408889634f / sqrtf((float)d), part_o, part_ml};
+    GatherArgs ga{(const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, idx, cnt, nq, q_pos0,
+                  ld_tokens, hq, hkv, max_sel, sink, window, ba.scale_log2, part_o, part_ml,
+                  (__nv_bfloat16*)O, lse, err};
+    int st = LSA_ERR_INVALID_ARG;
+    if (d == 128) st = launch_band_d<128>(G, ba, ga, batch, s);
+    else if (d == 64) st = launch_band_d<64>(G, ba, ga, batch, s);
+    scratch.release();
+    return st;
+}
+
+}  // namespace lsa

@@ -171,6 +171,9 @@ int launch_sparse_attn(const void* Q, const void* K, const void* V, const int32_
                        const int32_t* cnt, int64_t batch, int64_t nq, int hq, int hkv, int d,
                        int dtype, int max_sel, int64_t ld_tokens, void* O, float* lse,
                        int32_t* err, cudaStream_t s);
+int launch_banded_attn(const void* Q, const void* K, const void* V, const int32_t* idx, const int32_t* cnt,
+                       int64_t batch, int64_t nq, int64_t q_pos0, int hq, int hkv, int d, int max_sel,
+                       int64_t ld_tokens, int sink, int window, void* O, float* lse, int32_t* err, cudaStream_t s);
 
 // ---------------------------------------------------------------- append
 int launch_append(lsa_index* ix, const void* K, int64_t first_block, int64_t n_new_blocks,

@@ -60,6 +60,8 @@ _SIGS = {
     "lsa_select_noalloc": (_i32, [_vp, C.POINTER(SelectParams), _vp, _i64, _vp, _i64, _vp, _vp, _i32, _vp]),
     "lsa_sparse_attn": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _i64, _vp, _vp,
                                _vp]),
+    "lsa_sparse_attn_banded": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _i32, _i32,
+                                      _i64, _i32, _i32, _vp, _vp, _vp]),
     "lsa_append": (_i32, [_vp, _vp, _i64, _vp]),
     "lsa_project_pool": (_i32, [_vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
     "lsa_query_latent": (_i32, [_vp, _vp, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
@@ -264,6 +266,22 @@ def lsa_sparse_attn(Q, K, V, idx, cnt, hkv, O=None, lse=None, want_lse=True, str
                                int(d), dtype_code(Q), int(max_sel), int(ld_tokens), _ptr(O), _ptr(lse),
                                _stream(stream))
     _ok(st, "lsa_sparse_attn")
+    return O, lse
+
+
+def lsa_sparse_attn_banded(Q, K, V, idx, cnt, hkv, sink, window, q_pos0=0, O=None, lse=None, want_lse=True,
+                           stream=None):
+    B, nq, hq, d = Q.shape
+    ld_tokens = K.shape[1]
+    max_sel = idx.shape[-1]
+    if O is None:
+        O = torch.empty_like(Q)
+    if lse is None and want_lse:
+        lse = torch.empty((B, nq, hq), dtype=torch.float32, device=Q.device)
+    st = lib().lsa_sparse_attn_banded(_ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(cnt), int(B), int(nq), int(q_pos0),
+                                      int(hq), int(hkv), int(d), dtype_code(Q), int(max_sel), int(ld_tokens),
+                                      int(sink), int(window), _ptr(O), _ptr(lse), _stream(stream))
+    _ok(st, "lsa_sparse_attn_banded")
     return O, lse
 
 

@@ -212,6 +212,30 @@ int lsa_sparse_attn(const void* Q, const void* K, const void* V, const int32_t* 
                     int32_t d, int32_t dtype, int32_t max_sel, int64_t ld_tokens,
                     void* O, float* lse, void* stream);
 
+/* The same attention for a run of consecutive query positions, faster when
+ * each row list is a selection as lsa_select writes it: query qi sits at
+ * position i = q_pos0 + qi and its row is the sink [0, min(sink, i+1)), then
+ * long-range tokens in [sink, i-window], then the window
+ * [max(sink, i-window+1), i], ascending without repeats.  The sink and window
+ * rows are read once per tile of consecutive queries (a dense band, masked per
+ * query) and only the long-range entries are gathered per query; the two
+ * softmax parts are merged by their maxima, so the result is the attention of
+ * lsa_sparse_attn over the same row up to fp32 rounding order.
+ *  - Arguments as lsa_sparse_attn, plus q_pos0 (>= 0, q_pos0 + nq <=
+ *    ld_tokens), sink (>= 0) and window (>= 1), the values lsa_select used.
+ *  - A row that is ascending but not of that form is attended whole from the
+ *    list, with the same result; rows must be ascending without repeats.
+ *  - bf16 with hq/hkv in {1, 2, 4, 8, 16} takes the band path; other cases
+ *    run the lsa_sparse_attn kernels.
+ *  - Needs batch*nq*hq*(d+2) floats of stream-ordered scratch (pool memory).
+ * [p5 step 3 "selected long-range keys plus the attention sink and a local
+ * window"; the kernel is unchanged] */
+int lsa_sparse_attn_banded(const void* Q, const void* K, const void* V, const int32_t* idx,
+                           const int32_t* cnt, int64_t batch, int64_t nq, int64_t q_pos0,
+                           int32_t hq, int32_t hkv, int32_t d, int32_t dtype, int32_t max_sel,
+                           int64_t ld_tokens, int32_t sink, int32_t window,
+                           void* O, float* lse, void* stream);
+
 /* Decode: index tokens [n_tokens, n_tokens + n_new) that the caller has
  * already written into K (same layout and ld_tokens as the build).  Every
  * block this completes is pooled, mapped, and placed in its nearest leaf
