@@ -470,11 +470,13 @@ def cpu_cores() -> int:
     return os.cpu_count() or 1
 
 
-def cpu_oracle_estimate(w, inp, sample_queries: int) -> dict:
+def cpu_oracle_estimate(w, inp, sample_queries: int, lloyd_stride: int = 8) -> dict:
     """Time the oracle, as it stands, on a bounded sample of the workload and
-    scale to one whole layer: latents of every block; one full-size Lloyd
-    round of one KV head (x rounds x heads); the upper tree levels in full;
-    select + attention on sampled queries (x all queries x heads)."""
+    scale to one whole layer: latents of every block; one Lloyd round of one
+    KV head over every lloyd_stride-th block against all leaf centroids
+    (x lloyd_stride x rounds x heads: assignment cost is linear in the
+    points); the upper tree levels in full; select + attention on sampled
+    queries (x all queries x heads)."""
     import numpy as np
     import oracle as O
     K = inp["K"]
@@ -492,12 +494,18 @@ def cpu_oracle_estimate(w, inp, sample_queries: int) -> dict:
         Kh.append(kh)
         Kls.append(O.project_pool(kh, Wm, w.pool))
     t_lat = time.perf_counter() - t
-    # one Lloyd round of head 0 at full size
-    t = time.perf_counter()
+    # one Lloyd round of head 0 on a strided sample of the blocks
     C0 = O.kmeans_init(Kls[0], w.level_sizes[-1])
-    lab, _ = O.kmeans_assign(Kls[0], C0)
+    Xs = Kls[0][::lloyd_stride]
+    t = time.perf_counter()
+    lab_s, _ = O.kmeans_assign(Xs, C0)
+    O.kmeans_update(Xs, lab_s, C0, w.grid_log2)
+    t_round = (time.perf_counter() - t) * (Kls[0].shape[0] / Xs.shape[0])
+    # the tree the query sample runs on: every block takes the label of its
+    # stride group's sampled block (same bucket sizes as a real round, at no
+    # extra assignment cost; not timed)
+    lab = np.repeat(lab_s, lloyd_stride)[: Kls[0].shape[0]]
     C1 = O.kmeans_update(Kls[0], lab, C0, w.grid_log2)
-    t_round = time.perf_counter() - t
     # upper levels in full, on the leaf centroids of that round
     t = time.perf_counter()
     cents = [None] * len(w.level_sizes)
@@ -527,9 +535,11 @@ def cpu_oracle_estimate(w, inp, sample_queries: int) -> dict:
     wall = time.perf_counter() - t_start
     return {"value": N * w.batch / est, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
             "sample": (f"numpy fp64 oracle: latents of all {w.hkv} KV heads in full ({t_lat:.1f} s); one full-size "
-                       f"Lloyd round of one KV head ({t_round:.1f} s) x {w.lloyd_iters} rounds x {w.hkv} heads; "
+                       f"Lloyd round of one KV head, timed on every {lloyd_stride}th block and scaled "
+                       f"({t_round:.1f} s) x {w.lloyd_iters} rounds x {w.hkv} heads; "
                        f"upper levels in full ({t_upper:.1f} s) x {w.hkv}; select+attention on {len(rows)} "
-                       f"sampled queries ({t_query * 1e3:.1f} ms each) x {N} queries x {w.hkv} heads; "
+                       f"sampled queries over a tree whose leaves take the sampled labels "
+                       f"({t_query * 1e3:.1f} ms each) x {N} queries x {w.hkv} heads; "
                        f"estimated layer time {est:.0f} s from {wall:.0f} s of CPU work"),
             "estimated_layer_s": est}
 
@@ -546,7 +556,7 @@ def run_reference(args):
     vals = []
     cpu = None
     for k in range(args.warmup + args.steps):
-        r = cpu_oracle_estimate(w, inp, max(8, args.cpu_sample_queries // 4))
+        r = cpu_oracle_estimate(w, inp, max(8, args.cpu_sample_queries // 4), lloyd_stride=32)
         if k >= args.warmup:
             vals.append(r["value"])
             cpu = r

@@ -39,9 +39,15 @@ constexpr int kBandRows = 128;      // (query, head) rows per CTA
 constexpr int kBandTile = 64;       // keys per pipeline stage
 constexpr int kBandStages = 3;
 
-constexpr int kGatWarps = 4;        // queries per CTA (one warp each)
-constexpr int kGatSlice = 16;       // keys per slice
-constexpr int kGatStages = 3;
+#ifndef LSA_GAT_WARPS
+#define LSA_GAT_WARPS 2
+#endif
+#ifndef LSA_GAT_STAGES
+#define LSA_GAT_STAGES 2
+#endif
+constexpr int kGatWarps = LSA_GAT_WARPS;    // queries per CTA (one warp each)
+constexpr int kGatSlice = 16;               // keys per slice
+constexpr int kGatStages = LSA_GAT_STAGES;  // slices in each warp's ring
 
 struct BandArgs {
     const __nv_bfloat16* Q;
@@ -124,12 +130,8 @@ __global__ __launch_bounds__(kBandThreads, 1) void attn_band_kernel(const BandAr
     cp_async_wait<kBandStages - 1>();   // the Q group
     __syncthreads();
 
-    uint32_t qa[D / 16][4];
-    {
-        const int r = warp * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
-#pragma unroll
-        for (int kt = 0; kt < D / 16; ++kt) ldsm_x4(qsb + swz<D>(r, 2 * kt + (lane >> 4)), qa[kt][0], qa[kt][1], qa[kt][2], qa[kt][3]);
-    }
+    // A-fragment row of this lane in the warp's 16 Q rows (re-read per k step)
+    const int qrow = warp * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
     // this thread's two rows and their query positions
     const int r0 = warp * 16 + (lane >> 2), r1 = r0 + 8;
     const int64_t pa = i0 + r0 / G, pb = i0 + r1 / G;
@@ -157,18 +159,22 @@ __global__ __launch_bounds__(kBandThreads, 1) void attn_band_kernel(const BandAr
                           q0 + warp * QW + QW - 1 <= qlast;
         const int st = t % kBandStages;
         const uint32_t kb = smem_u32(Ks + st * TILE_BYTES), vb = smem_u32(Vs + st * TILE_BYTES);
+        // S = Q K^T over 64 keys: k steps outermost, so the 8 accumulators
+        // are 8 independent chains
         float s[8][4];
 #pragma unroll
         for (int j = 0; j < 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
 #pragma unroll
-        for (int np = 0; np < 4; ++np) {
-            const int kr = np * 16 + (lane & 7) + 8 * (lane >> 4);
+        for (int kt = 0; kt < D / 16; ++kt) {
+            uint32_t qa[4];
+            ldsm_x4(qsb + swz<D>(qrow, 2 * kt + (lane >> 4)), qa[0], qa[1], qa[2], qa[3]);
 #pragma unroll
-            for (int kt = 0; kt < D / 16; ++kt) {
+            for (int np = 0; np < 4; ++np) {
                 uint32_t b0, b1, b2, b3;
-                ldsm_x4(kb + swz<D>(kr, 2 * kt + ((lane >> 3) & 1)), b0, b1, b2, b3);
-                mma_bf16(s[2 * np], qa[kt], b0, b1);
-                mma_bf16(s[2 * np + 1], qa[kt], b2, b3);
+                ldsm_x4(kb + swz<D>(np * 16 + (lane & 7) + 8 * (lane >> 4), 2 * kt + ((lane >> 3) & 1)), b0, b1,
+                        b2, b3);
+                mma_bf16(s[2 * np], qa, b0, b1);
+                mma_bf16(s[2 * np + 1], qa, b2, b3);
             }
         }
         // scale and mask: key j = jb + 8 * nt + 2 * (lane & 3) + (e & 1)
@@ -229,14 +235,24 @@ __global__ __launch_bounds__(kBandThreads, 1) void attn_band_kernel(const BandAr
             split_pack(s[2 * kk + 1][0], s[2 * kk + 1][1], ph[2], pl[2]);
             split_pack(s[2 * kk + 1][2], s[2 * kk + 1][3], ph[3], pl[3]);
             const int vr = kk * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
+            // per half of the d columns: fragments first, then the hi and the
+            // lo pass (8 MMAs apart on each accumulator)
 #pragma unroll
-            for (int nt = 0; nt < D / 8; nt += 2) {
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4_t(vb + swz<D>(vr, nt + (lane >> 4)), b0, b1, b2, b3);
-                mma_bf16(o[nt], ph, b0, b1);
-                mma_bf16(o[nt + 1], ph, b2, b3);
-                mma_bf16(o[nt], pl, b0, b1);
-                mma_bf16(o[nt + 1], pl, b2, b3);
+            for (int hf = 0; hf < D / 64; ++hf) {
+                uint32_t vf[4][4];
+#pragma unroll
+                for (int j = 0; j < 4; ++j)
+                    ldsm_x4_t(vb + swz<D>(vr, hf * 8 + 2 * j + (lane >> 4)), vf[j][0], vf[j][1], vf[j][2], vf[j][3]);
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    mma_bf16(o[hf * 8 + 2 * j], ph, vf[j][0], vf[j][1]);
+                    mma_bf16(o[hf * 8 + 2 * j + 1], ph, vf[j][2], vf[j][3]);
+                }
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    mma_bf16(o[hf * 8 + 2 * j], pl, vf[j][0], vf[j][1]);
+                    mma_bf16(o[hf * 8 + 2 * j + 1], pl, vf[j][2], vf[j][3]);
+                }
             }
         }
     }
@@ -361,24 +377,37 @@ __global__ __launch_bounds__(kGatWarps * 32) void attn_gather_kernel(const Gathe
     const int nslice = (pend - pbeg + kGatSlice - 1) / kGatSlice;
     const __nv_bfloat16* kbase = a.K + (b * a.ld_tokens * a.hkv + h) * D;
     const __nv_bfloat16* vbase = a.V + (b * a.ld_tokens * a.hkv + h) * D;
+    // token of key `lane` of slice s (lanes < 16); a bad index is latched and skipped
     auto fetch_tok = [&](int s) -> int {
         const int p = pbeg + s * kGatSlice + lane;
-        return (lane < kGatSlice && s < nslice && p < pend) ? __ldg(ir + p) : -1;
+        int t = (lane < kGatSlice && s < nslice && p < pend) ? __ldg(ir + p) : -1;
+        if (t >= a.ld_tokens || t < -1) {
+            latch(a.err, kErrDevice);
+            t = -1;
+        }
+        return t;
     };
+    // each lane copies 16-byte column c of rows lane/CH + RSTEP*k; the shared
+    // offsets of those rows and the column's source offset are fixed
+    const int c_col = lane % CH;
+    uint32_t dsto[RPL];
+#pragma unroll
+    for (int k = 0; k < RPL; ++k) dsto[k] = swz<D>(lane / CH + RSTEP * k, c_col);
+    const char* ksrc = reinterpret_cast<const char*>(kbase + c_col * 8);
+    const int64_t vk = reinterpret_cast<const char*>(vbase) - reinterpret_cast<const char*>(kbase);
+    const int64_t rs = (int64_t)a.hkv * D * 2;
     auto load_slice = [&](int s, int tok_l) {
         const int st = s % kGatStages;
         const uint32_t kb = smem_u32(Ks + st * SLICE_BYTES), vb = smem_u32(Vs + st * SLICE_BYTES);
-        const int c = lane % CH;
-        const uint32_t live = __ballot_sync(0xffffffffu, tok_l >= 0 && tok_l < a.ld_tokens);
+        const uint32_t live = __ballot_sync(0xffffffffu, tok_l >= 0);
         if (lane == 0) vmask[st] = live & 0xffffu;
 #pragma unroll
         for (int k = 0; k < RPL; ++k) {
-            const int r = lane / CH + RSTEP * k;
-            int tok = __shfl_sync(0xffffffffu, tok_l, r);
-            if (tok >= a.ld_tokens || tok < -1) { latch(a.err, kErrDevice); tok = -1; }
-            const int64_t off = tok >= 0 ? (int64_t)tok * a.hkv * D + c * 8 : 0;
-            cp_async16(kb + swz<D>(r, c), kbase + off, tok >= 0 ? 16 : 0);
-            cp_async16(vb + swz<D>(r, c), vbase + off, tok >= 0 ? 16 : 0);
+            const int tok = __shfl_sync(0xffffffffu, tok_l, lane / CH + RSTEP * k);
+            const char* src = ksrc + (tok >= 0 ? (int64_t)tok * rs : 0);
+            const int nbytes = tok >= 0 ? 16 : 0;
+            cp_async16(kb + dsto[k], src, nbytes);
+            cp_async16(vb + dsto[k], src + vk, nbytes);
         }
     };
     int tok_next = fetch_tok(0);
@@ -398,18 +427,31 @@ __global__ __launch_bounds__(kGatWarps * 32) void attn_gather_kernel(const Gathe
         const int st = s % kGatStages;
         const uint32_t kb = smem_u32(Ks + st * SLICE_BYTES), vb = smem_u32(Vs + st * SLICE_BYTES);
         // S^T = K_slice Q^T: rows = 16 keys, cols = heads
-        float sc[NT][4];
+        // (all fragments first, then two independent accumulation chains)
+        float sc[NT][4], sc2[NT][4];
 #pragma unroll
-        for (int nt = 0; nt < NT; ++nt) sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+        for (int nt = 0; nt < NT; ++nt) {
+            sc[nt][0] = sc[nt][1] = sc[nt][2] = sc[nt][3] = 0.f;
+            sc2[nt][0] = sc2[nt][1] = sc2[nt][2] = sc2[nt][3] = 0.f;
+        }
         {
             const int kr = (lane & 7) + 8 * ((lane >> 3) & 1);
+            uint32_t ka[D / 16][4];
 #pragma unroll
-            for (int kt = 0; kt < D / 16; ++kt) {
-                uint32_t ka[4];
-                ldsm_x4(kb + swz<D>(kr, 2 * kt + (lane >> 4)), ka[0], ka[1], ka[2], ka[3]);
+            for (int kt = 0; kt < D / 16; ++kt)
+                ldsm_x4(kb + swz<D>(kr, 2 * kt + (lane >> 4)), ka[kt][0], ka[kt][1], ka[kt][2], ka[kt][3]);
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) mma_bf16(sc[nt], ka, qb[kt][nt][0], qb[kt][nt][1]);
+            for (int kt = 0; kt < D / 16; kt += 2) {
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) {
+                    mma_bf16(sc[nt], ka[kt], qb[kt][nt][0], qb[kt][nt][1]);
+                    mma_bf16(sc2[nt], ka[kt + 1], qb[kt + 1][nt][0], qb[kt + 1][nt][1]);
+                }
             }
+#pragma unroll
+            for (int nt = 0; nt < NT; ++nt)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) sc[nt][e] += sc2[nt][e];
         }
         // keys lane/4 and lane/4 + 8 of the slice
         const uint32_t vm = vmask[st];
@@ -454,18 +496,22 @@ __global__ __launch_bounds__(kGatWarps * 32) void attn_gather_kernel(const Gathe
             }
         }
         // O^T += V^T P^T: rows = dims (16 per m tile), k = 16 keys
+        // (all fragments first; the hi pass over every m tile, then the lo pass,
+        // so no two consecutive MMAs share an accumulator)
         {
             const int vr = (lane & 7) + 8 * (lane >> 4);
+            uint32_t va[D / 16][4];
 #pragma unroll
-            for (int mt = 0; mt < D / 16; ++mt) {
-                uint32_t va[4];
-                ldsm_x4_t(vb + swz<D>(vr, 2 * mt + ((lane >> 3) & 1)), va[0], va[1], va[2], va[3]);
+            for (int mt = 0; mt < D / 16; ++mt)
+                ldsm_x4_t(vb + swz<D>(vr, 2 * mt + ((lane >> 3) & 1)), va[mt][0], va[mt][1], va[mt][2], va[mt][3]);
 #pragma unroll
-                for (int nt = 0; nt < NT; ++nt) {
-                    mma_bf16(ot[mt][nt], va, bh[nt][0], bh[nt][1]);
-                    mma_bf16(ot[mt][nt], va, bl[nt][0], bl[nt][1]);
-                }
-            }
+            for (int mt = 0; mt < D / 16; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma_bf16(ot[mt][nt], va[mt], bh[nt][0], bh[nt][1]);
+#pragma unroll
+            for (int mt = 0; mt < D / 16; ++mt)
+#pragma unroll
+                for (int nt = 0; nt < NT; ++nt) mma_bf16(ot[mt][nt], va[mt], bl[nt][0], bl[nt][1]);
         }
     }
     cp_async_wait<0>();

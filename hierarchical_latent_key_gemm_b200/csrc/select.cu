@@ -13,9 +13,8 @@
 //
 // One CTA per (query, KV head).  Every tree level is stored in tree order
 // (children of a node are contiguous), so a candidate's minpos, original id
-// and centroid row are independent loads; each sub-warp group of r/8 lanes
-// walks a contiguous run of candidates and issues the loads of several before
-// it uses any of them.  Scores stream through a shared-memory buffer;
+// and centroid row are independent loads; each sub-warp group of r/16 lanes
+// (16 floats of the row per lane) walks a contiguous run of candidates.  Scores stream through a shared-memory buffer;
 // whenever it holds more than k items a block-wide radix select (on the
 // order-preserving bit pattern of the fp32 score, then on the original id for
 // ties) compacts it to the top k.  The order is total, (score desc, id asc),
@@ -25,10 +24,11 @@
 namespace lsa {
 namespace {
 
-// 2 candidates in flight per group at 8 CTAs (32 warps) per SM measured
-// fastest on the 1M-token workload (4 in flight at 4 CTAs: 1.3x slower).
+// One candidate in flight per group at 8 CTAs (32 warps) per SM measured
+// fastest on the 1M-token workload (194 ms; 2 in flight at 6 CTAs: 209 ms,
+// at 4 CTAs: 249 ms).
 #ifndef LSA_SELECT_UNROLL
-#define LSA_SELECT_UNROLL 2
+#define LSA_SELECT_UNROLL 1
 #endif
 #ifndef LSA_SELECT_MIN_BLOCKS
 #define LSA_SELECT_MIN_BLOCKS 8
@@ -66,6 +66,7 @@ struct SelShared {
     int count;
     int count2;
     int nkept;
+    uint32_t thr;   // key of the k-th best item after the last compaction (0: none yet)
 };
 
 // Order-preserving map of a float onto uint32 (-0 and +0 map together).
@@ -156,6 +157,7 @@ __device__ void topk_compact(const float* s, const int* id, const int* ps, int n
         int need2, eq2;
         T2 = block_kth(s, id, n, need, 1, T, sh, &need2, &eq2);
     }
+    if (threadIdx.x == 0) sh.thr = T;
     for (int i = threadIdx.x; i < n; i += blockDim.x) {
         const uint32_t key = fkey(s[i]);
         const bool take = key > T || (key == T && (!split || ~(uint32_t)id[i] >= T2));
@@ -205,20 +207,18 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
     const SelArgs a) {
     extern __shared__ float4 dyn4[];
     __shared__ SelShared sh;
-    float* bsb[2];
-    int* bib[2];
-    int* bpb[2];
-    bsb[0] = reinterpret_cast<float*>(dyn4);
-    bib[0] = reinterpret_cast<int*>(bsb[0] + a.cap);
-    bpb[0] = bib[0] + a.cap;
-    bsb[1] = reinterpret_cast<float*>(bpb[0] + a.cap);
-    bib[1] = reinterpret_cast<int*>(bsb[1] + a.cap);
-    bpb[1] = bib[1] + a.cap;
-    int* kk = bpb[1] + a.cap;        // kept positions [beam]
+    // two buffers of (score, id, position) x cap, selected by `cur`
+    // (pointer arithmetic, not an indexed array, so nothing lives in local memory)
+    float* const buf0 = reinterpret_cast<float*>(dyn4);
+    const int bstride = 3 * a.cap;
+    auto bsb = [&](int c) { return buf0 + c * bstride; };
+    auto bib = [&](int c) { return reinterpret_cast<int*>(buf0 + c * bstride + a.cap); };
+    auto bpb = [&](int c) { return reinterpret_cast<int*>(buf0 + c * bstride + 2 * a.cap); };
+    int* kk = reinterpret_cast<int*>(buf0 + 2 * bstride);   // kept positions [beam]
     int* pre = kk + a.beam;          // [beam + 1]
     int* lo = pre + a.beam + 1;      // [beam]
 
-    constexpr int LPC = R / 8;              // lanes per candidate row
+    constexpr int LPC = R / 16;             // lanes per candidate row (16 floats each)
     constexpr int CPW = 32 / LPC;           // candidates per warp
     constexpr int NG = (THREADS / 32) * CPW;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -235,26 +235,36 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
     const int64_t b_lo = (a.sink + a.pool - 1) / a.pool;
     const int64_t b_hi = bound >= 0 ? bound / a.pool : -1;
 
-    float qv[8];
+    // lane gl of a group holds float4 chunks gl, gl + LPC, gl + 2 LPC, gl + 3 LPC
+    // of a row: each load instruction reads LPC * 16 contiguous bytes per row
+    float4 qv[4];
     {
-        const float4* qp = reinterpret_cast<const float4*>(a.qbar + row * R + gl * 8);
-        const float4 x0 = qp[0], x1 = qp[1];
-        qv[0] = x0.x; qv[1] = x0.y; qv[2] = x0.z; qv[3] = x0.w;
-        qv[4] = x1.x; qv[5] = x1.y; qv[6] = x1.z; qv[7] = x1.w;
+        const float4* qp = reinterpret_cast<const float4*>(a.qbar + row * R) + gl;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) qv[j] = qp[j * LPC];
     }
-    auto dot = [&](const float4& y0, const float4& y1) -> float {
-        float s = 0.f;
-        s = __fmaf_rn(qv[0], y0.x, s); s = __fmaf_rn(qv[1], y0.y, s);
-        s = __fmaf_rn(qv[2], y0.z, s); s = __fmaf_rn(qv[3], y0.w, s);
-        s = __fmaf_rn(qv[4], y1.x, s); s = __fmaf_rn(qv[5], y1.y, s);
-        s = __fmaf_rn(qv[6], y1.z, s); s = __fmaf_rn(qv[7], y1.w, s);
+    auto dot = [&](const float4* y) -> float {
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int j = 0; j < 4; j += 2) {
+            s0 = __fmaf_rn(qv[j].x, y[j].x, s0); s0 = __fmaf_rn(qv[j].y, y[j].y, s0);
+            s0 = __fmaf_rn(qv[j].z, y[j].z, s0); s0 = __fmaf_rn(qv[j].w, y[j].w, s0);
+            s1 = __fmaf_rn(qv[j + 1].x, y[j + 1].x, s1); s1 = __fmaf_rn(qv[j + 1].y, y[j + 1].y, s1);
+            s1 = __fmaf_rn(qv[j + 1].z, y[j + 1].z, s1); s1 = __fmaf_rn(qv[j + 1].w, y[j + 1].w, s1);
+        }
+        float s = __fadd_rn(s0, s1);
 #pragma unroll
         for (int o = LPC / 2; o >= 1; o >>= 1) s = __fadd_rn(s, __shfl_xor_sync(gmask, s, o));
         return s;
     };
+    auto load_row = [&](const float* rowp, float4* y) {
+        const float4* rp = reinterpret_cast<const float4*>(rowp) + gl;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) y[j] = __ldg(rp + j * LPC);
+    };
 
     for (int e = threadIdx.x; e < 256; e += blockDim.x) sh.hist[e] = 0;
-    if (threadIdx.x == 0) { sh.count = 0; sh.nkept = 0; }
+    if (threadIdx.x == 0) { sh.count = 0; sh.nkept = 0; sh.thr = 0u; }
     __syncthreads();
 
     int cur = 0;
@@ -262,38 +272,48 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt_mask));
     // Push candidates t in [0, total) through the buffer, keeping the top k.
     // Each group walks a contiguous run of candidates, kUnroll at a time:
-    // fetch(t, &state, &elig, &id, &p, &y0, &y1) issues the loads of
-    // candidate t (state carries the owning node across consecutive t), and
-    // the results are used only after every load of the batch is in flight.
-    // Appends are aggregated per warp: one shared-memory atomic per batch.
+    // fetch(t, &state, &elig, &id, &p, y) issues the loads of candidate t
+    // (state carries the owning node across consecutive t), and the results
+    // are used only after every load of the batch is in flight.  Once the
+    // buffer has been compacted, a candidate whose key is below the k-th kept
+    // key cannot enter the top k and is not appended.  The buffer is compacted
+    // only when the next chunk might not fit, and at the end.  Appends are
+    // aggregated per warp: one shared-memory atomic per batch.
     auto stream_topk = [&](int total, int k, auto&& fetch) {
         if (k <= 0) return;  // nothing is kept; the buffer stays empty
-        const int chunk = a.cap - k;
-        for (int t0 = 0; t0 < total; t0 += chunk) {
-            const int t1 = min(total, t0 + chunk);
-            float* bs = bsb[cur];
-            int* bi = bib[cur];
-            int* bp = bpb[cur];
+        // entered with an empty buffer; nbuf mirrors sh.count between chunks
+        if (threadIdx.x == 0) sh.thr = 0u;
+        __syncthreads();
+        int t0 = 0, nbuf = 0;
+        while (t0 < total) {
+            const uint32_t thr = sh.thr;
+            const int t1 = min(total, t0 + (a.cap - nbuf));
+            float* bs = bsb(cur);
+            int* bi = bib(cur);
+            int* bp = bpb(cur);
             const int span = (t1 - t0 + NG - 1) / NG;
             const int tb = t0 + gid * span;
             const int te = min(t1, tb + span);
             int state = -1;
             for (int s0 = 0; s0 < span; s0 += kUnroll) {
-                float4 y0[kUnroll], y1[kUnroll];
+                float4 y[kUnroll][4];
                 int idv[kUnroll], pv[kUnroll];
                 bool ok[kUnroll];
 #pragma unroll
                 for (int v = 0; v < kUnroll; ++v) {
                     const int tt = tb + s0 + v;
                     ok[v] = tt < te;
-                    if (ok[v]) fetch(tt, &state, &ok[v], &idv[v], &pv[v], &y0[v], &y1[v]);
+                    if (ok[v]) fetch(tt, &state, &ok[v], &idv[v], &pv[v], y[v]);
                 }
                 float sc[kUnroll];
                 uint32_t bal[kUnroll];
                 int nb_warp = 0;
 #pragma unroll
                 for (int v = 0; v < kUnroll; ++v) {
-                    if (ok[v]) sc[v] = dot(y0[v], y1[v]);
+                    if (ok[v]) {
+                        sc[v] = dot(y[v]);
+                        ok[v] = fkey(sc[v]) >= thr;
+                    }
                     bal[v] = __ballot_sync(0xffffffffu, ok[v] && gl == 0);
                     nb_warp += __popc(bal[v]);
                 }
@@ -311,12 +331,17 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
                     base += __popc(bal[v]);
                 }
             }
+            t0 = t1;
             __syncthreads();
             const int n = sh.count;
-            if (n > k) {
-                topk_compact(bs, bi, bp, n, k, bsb[cur ^ 1], bib[cur ^ 1], bpb[cur ^ 1], sh);
+            // compact when done, or when less than a quarter of the buffer is free
+            if (n > k && (t0 >= total || a.cap - n < a.cap / 4)) {
+                topk_compact(bs, bi, bp, n, k, bsb(cur ^ 1), bib(cur ^ 1), bpb(cur ^ 1), sh);
                 cur ^= 1;
                 if (threadIdx.x == 0) sh.count = k;
+                nbuf = k;
+            } else {
+                nbuf = n;
             }
             __syncthreads();
         }
@@ -342,7 +367,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
             const int total = (l == 0) ? nl : pre[nk];
             if (threadIdx.x == 0) sh.count = 0;
             __syncthreads();
-            stream_topk(total, a.beam, [&](int t, int* state, bool* el, int* id, int* p, float4* y0, float4* y1) {
+            stream_topk(total, a.beam, [&](int t, int* state, bool* el, int* id, int* p, float4* y) {
                 int q;
                 if (l == 0) {
                     q = t;
@@ -350,15 +375,13 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
                     const int o = owner(t, nk, state);
                     q = lo[o] + (t - pre[o]);
                 }
-                const float4* rp = reinterpret_cast<const float4*>(cent + (int64_t)q * R + gl * 8);
-                *y0 = __ldg(rp);
-                *y1 = __ldg(rp + 1);
+                load_row(cent + (int64_t)q * R, y);
                 *id = __ldg(oid + q);
                 *p = q;
                 *el = __ldg(mp + q) <= bound;
             });
             const int n = sh.count;
-            for (int e = threadIdx.x; e < n; e += blockDim.x) kk[e] = bpb[cur][e];
+            for (int e = threadIdx.x; e < n; e += blockDim.x) kk[e] = bpb(cur)[e];
             __syncthreads();
             if (threadIdx.x == 0) sh.nkept = n;
             if (l + 1 < a.levels) {
@@ -394,12 +417,10 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
         scan_pre(pre, nk);
         if (threadIdx.x == 0) sh.count = 0;
         __syncthreads();
-        stream_topk(pre[nk], a.kb, [&](int t, int* state, bool* el, int* id, int* p, float4* y0, float4* y1) {
+        stream_topk(pre[nk], a.kb, [&](int t, int* state, bool* el, int* id, int* p, float4* y) {
             const int o = owner(t, nk, state);
             const int64_t slot = lo[o] + (t - pre[o]);
-            const float4* rp = reinterpret_cast<const float4*>(a.Klp + slot * R + gl * 8);
-            *y0 = __ldg(rp);
-            *y1 = __ldg(rp + 1);
+            load_row(a.Klp + slot * R, y);
             *id = __ldg(a.blk + slot);
             *p = 0;
             *el = true;
@@ -408,12 +429,10 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
         const int64_t hi = min(a.nb - 1, b_hi);
         const int total = hi >= b_lo ? (int)(hi - b_lo + 1) : 0;
         const float* kl = a.Kl + (int64_t)u * a.nb_cap * R;
-        stream_topk(total, a.kb, [&](int t, int* state, bool* el, int* id, int* p, float4* y0, float4* y1) {
+        stream_topk(total, a.kb, [&](int t, int* state, bool* el, int* id, int* p, float4* y) {
             (void)state;
             const int64_t b = b_lo + t;
-            const float4* rp = reinterpret_cast<const float4*>(kl + b * R + gl * 8);
-            *y0 = __ldg(rp);
-            *y1 = __ldg(rp + 1);
+            load_row(kl + b * R, y);
             *id = (int)b;
             *p = 0;
             *el = true;
@@ -422,10 +441,10 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
     const int nsel = sh.count;
 
     // ascending block ids
-    int* arr = bib[cur ^ 1];
+    int* arr = bib(cur ^ 1);
     if (THREADS >= 512) {
         // wide CTAs: rank sort (each id counts the smaller ones), one barrier
-        const int* src = bib[cur];
+        const int* src = bib(cur);
         for (int e = threadIdx.x; e < nsel; e += THREADS) {
             const int x = src[e];
             int rank = 0;
@@ -437,7 +456,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
         // bitonic sort, padded to a power of two
         int M = 1;
         while (M < nsel) M <<= 1;
-        for (int e = threadIdx.x; e < M; e += blockDim.x) arr[e] = e < nsel ? bib[cur][e] : INT32_MAX;
+        for (int e = threadIdx.x; e < M; e += blockDim.x) arr[e] = e < nsel ? bib(cur)[e] : INT32_MAX;
         __syncthreads();
         for (int size = 2; size <= M; size <<= 1) {
             for (int stride = size >> 1; stride > 0; stride >>= 1) {
