@@ -69,6 +69,13 @@ struct SelShared {
     uint32_t thr;   // key of the k-th best item after the last compaction (0: none yet)
 };
 
+// 32 bytes from global memory in one 256-bit read-only load (32-byte aligned).
+__device__ __forceinline__ void ldg256(const float* p, float* v) {
+    asm volatile("ld.global.nc.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
+                 : "l"(p));
+}
+
 // Order-preserving map of a float onto uint32 (-0 and +0 map together).
 __device__ __forceinline__ uint32_t fkey(float f) {
     const uint32_t u = __float_as_uint(__fadd_rn(f, 0.0f));
@@ -235,32 +242,33 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
     const int64_t b_lo = (a.sink + a.pool - 1) / a.pool;
     const int64_t b_hi = bound >= 0 ? bound / a.pool : -1;
 
-    // lane gl of a group holds float4 chunks gl, gl + LPC, gl + 2 LPC, gl + 3 LPC
-    // of a row: each load instruction reads LPC * 16 contiguous bytes per row
-    float4 qv[4];
+    // lane gl of a group holds 32-byte pieces gl and gl + LPC of a row: each
+    // 256-bit load instruction reads LPC * 32 contiguous bytes (whole 128-byte
+    // lines) of every row it touches
+    float qv[16];
     {
-        const float4* qp = reinterpret_cast<const float4*>(a.qbar + row * R) + gl;
+        const float* qp = a.qbar + row * R + gl * 8;
 #pragma unroll
-        for (int j = 0; j < 4; ++j) qv[j] = qp[j * LPC];
+        for (int j = 0; j < 8; ++j) {
+            qv[j] = qp[j];
+            qv[8 + j] = qp[LPC * 8 + j];
+        }
     }
-    auto dot = [&](const float4* y) -> float {
+    auto dot = [&](const float* y) -> float {
         float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-        for (int j = 0; j < 4; j += 2) {
-            s0 = __fmaf_rn(qv[j].x, y[j].x, s0); s0 = __fmaf_rn(qv[j].y, y[j].y, s0);
-            s0 = __fmaf_rn(qv[j].z, y[j].z, s0); s0 = __fmaf_rn(qv[j].w, y[j].w, s0);
-            s1 = __fmaf_rn(qv[j + 1].x, y[j + 1].x, s1); s1 = __fmaf_rn(qv[j + 1].y, y[j + 1].y, s1);
-            s1 = __fmaf_rn(qv[j + 1].z, y[j + 1].z, s1); s1 = __fmaf_rn(qv[j + 1].w, y[j + 1].w, s1);
+        for (int j = 0; j < 8; ++j) {
+            s0 = __fmaf_rn(qv[j], y[j], s0);
+            s1 = __fmaf_rn(qv[8 + j], y[8 + j], s1);
         }
         float s = __fadd_rn(s0, s1);
 #pragma unroll
         for (int o = LPC / 2; o >= 1; o >>= 1) s = __fadd_rn(s, __shfl_xor_sync(gmask, s, o));
         return s;
     };
-    auto load_row = [&](const float* rowp, float4* y) {
-        const float4* rp = reinterpret_cast<const float4*>(rowp) + gl;
-#pragma unroll
-        for (int j = 0; j < 4; ++j) y[j] = __ldg(rp + j * LPC);
+    auto load_row = [&](const float* rowp, float* y) {
+        ldg256(rowp + gl * 8, y);
+        ldg256(rowp + (LPC + gl) * 8, y + 8);
     };
 
     for (int e = threadIdx.x; e < 256; e += blockDim.x) sh.hist[e] = 0;
@@ -296,7 +304,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
             const int te = min(t1, tb + span);
             int state = -1;
             for (int s0 = 0; s0 < span; s0 += kUnroll) {
-                float4 y[kUnroll][4];
+                float y[kUnroll][16];
                 int idv[kUnroll], pv[kUnroll];
                 bool ok[kUnroll];
 #pragma unroll
@@ -367,7 +375,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
             const int total = (l == 0) ? nl : pre[nk];
             if (threadIdx.x == 0) sh.count = 0;
             __syncthreads();
-            stream_topk(total, a.beam, [&](int t, int* state, bool* el, int* id, int* p, float4* y) {
+            stream_topk(total, a.beam, [&](int t, int* state, bool* el, int* id, int* p, float* y) {
                 int q;
                 if (l == 0) {
                     q = t;
@@ -417,7 +425,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
         scan_pre(pre, nk);
         if (threadIdx.x == 0) sh.count = 0;
         __syncthreads();
-        stream_topk(pre[nk], a.kb, [&](int t, int* state, bool* el, int* id, int* p, float4* y) {
+        stream_topk(pre[nk], a.kb, [&](int t, int* state, bool* el, int* id, int* p, float* y) {
             const int o = owner(t, nk, state);
             const int64_t slot = lo[o] + (t - pre[o]);
             load_row(a.Klp + slot * R, y);
@@ -429,7 +437,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
         const int64_t hi = min(a.nb - 1, b_hi);
         const int total = hi >= b_lo ? (int)(hi - b_lo + 1) : 0;
         const float* kl = a.Kl + (int64_t)u * a.nb_cap * R;
-        stream_topk(total, a.kb, [&](int t, int* state, bool* el, int* id, int* p, float4* y) {
+        stream_topk(total, a.kb, [&](int t, int* state, bool* el, int* id, int* p, float* y) {
             (void)state;
             const int64_t b = b_lo + t;
             load_row(kl + b * R, y);
@@ -451,6 +459,67 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
             for (int j = 0; j < nsel; ++j) rank += src[j] < x;
             arr[rank] = x;
         }
+        __syncthreads();
+    } else if (nsel <= 4 * THREADS) {
+        // bitonic sort of 4 * THREADS items (padded with INT32_MAX), 4 per
+        // thread in registers: item i = 4 tid + k; strides 1-2 inside a
+        // thread, 4-64 across lanes by shuffles, 128 and up through shared
+        // memory
+        constexpr int M = 4 * THREADS;
+        int v[4];
+        const int* src = bib(cur);
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+            const int i = 4 * threadIdx.x + k;
+            v[k] = i < nsel ? src[i] : INT32_MAX;
+        }
+        __syncthreads();   // src and arr may be read and written below
+        for (int size = 2; size <= M; size <<= 1) {
+            for (int stride = size >> 1; stride > 0; stride >>= 1) {
+                if (stride >= 128) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) arr[4 * threadIdx.x + k] = v[k];
+                    __syncthreads();
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int i = 4 * threadIdx.x + k;
+                        const int y = arr[i ^ stride];
+                        const bool asc = (i & size) == 0;
+                        const bool lower = (i & stride) == 0;
+                        v[k] = (lower == asc) ? min(v[k], y) : max(v[k], y);
+                    }
+                    __syncthreads();
+                } else if (stride >= 4) {
+#pragma unroll
+                    for (int k = 0; k < 4; ++k) {
+                        const int i = 4 * threadIdx.x + k;
+                        const int y = __shfl_xor_sync(0xffffffffu, v[k], stride >> 2);
+                        const bool asc = (i & size) == 0;
+                        const bool lower = (i & stride) == 0;
+                        v[k] = (lower == asc) ? min(v[k], y) : max(v[k], y);
+                    }
+                } else {
+                    // pairs (0, s), (1, 1 + s) ... inside the thread; written out
+                    // per stride so every register index is a constant
+                    // (direction of the pair starting at item k: ((4 tid + k) & size) == 0)
+                    auto cx = [&](int k, int& x, int& y) {
+                        const bool asc = ((4 * (int)threadIdx.x + k) & size) == 0;
+                        const int lo = min(x, y), hi = max(x, y);
+                        x = asc ? lo : hi;
+                        y = asc ? hi : lo;
+                    };
+                    if (stride == 2) {
+                        cx(0, v[0], v[2]);
+                        cx(1, v[1], v[3]);
+                    } else {
+                        cx(0, v[0], v[1]);
+                        cx(2, v[2], v[3]);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) arr[4 * threadIdx.x + k] = v[k];
         __syncthreads();
     } else {
         // bitonic sort, padded to a power of two
