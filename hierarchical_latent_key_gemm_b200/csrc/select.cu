@@ -60,13 +60,17 @@ struct SelArgs {
     int cap;
 };
 
+constexpr int kResolveCap = 256;   // most items of the threshold bin ranked pairwise
+
 struct SelShared {
     int hist[256];
     int bc[4];
     int count;
     int count2;
     int nkept;
-    uint32_t thr;   // key of the k-th best item after the last compaction (0: none yet)
+    uint32_t thr;   // no item below this key can be in the current top k (0: none yet)
+    uint32_t wmin[32], wmax[32];
+    int nres;
 };
 
 // 32 bytes from global memory in one 256-bit read-only load (32-byte aligned).
@@ -153,9 +157,125 @@ __device__ uint32_t block_kth(const float* s, const int* id, int n, int k, int m
     return prefix;
 }
 
-// Keep the top k of the n items in (s, id, ps); result in (ds, di, dp)[0..k).
+// Keep the top k of the n items in (s, id, ps) by (score desc, id asc), k < n;
+// result in (ds, di, dp)[0..k) in no particular order.  The keys are binned by
+// their offset from the smallest key, shifted so that at most 256 bins are
+// used (monotone in the key); bins above the one that holds the k-th item are
+// taken whole, and that bin's items are ranked exactly by (key, id).  If that
+// bin holds more than kResolveCap items (or all keys are equal), the general
+// radix select below runs instead.
+__device__ void topk_compact_radix(const float* s, const int* id, const int* ps, int n, int k, float* ds, int* di,
+                                   int* dp, SelShared& sh);
+
 __device__ void topk_compact(const float* s, const int* id, const int* ps, int n, int k, float* ds, int* di,
                              int* dp, SelShared& sh) {
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
+    uint32_t kmn = 0xffffffffu, kmx = 0u;
+    for (int i = tid; i < n; i += blockDim.x) {
+        const uint32_t key = fkey(s[i]);
+        kmn = min(kmn, key);
+        kmx = max(kmx, key);
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+        kmn = min(kmn, __shfl_xor_sync(0xffffffffu, kmn, o));
+        kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, o));
+    }
+    if (lane == 0) { sh.wmin[warp] = kmn; sh.wmax[warp] = kmx; }
+    if (tid == 0) { sh.count2 = 0; sh.nres = 0; }
+    __syncthreads();
+    kmn = sh.wmin[0];
+    kmx = sh.wmax[0];
+    for (int w = 1; w < nw; ++w) {
+        kmn = min(kmn, sh.wmin[w]);
+        kmx = max(kmx, sh.wmax[w]);
+    }
+    if (kmn == kmx) {
+        topk_compact_radix(s, id, ps, n, k, ds, di, dp, sh);
+        return;
+    }
+    const int shift = max(0, 24 - __clz(kmx - kmn));   // (kmx - kmn) >> shift <= 255
+    for (int i = tid; i < n; i += blockDim.x) atomicAdd(&sh.hist[(fkey(s[i]) - kmn) >> shift], 1);
+    __syncthreads();
+    if (warp == 0) {
+        int c[8], sum = 0;
+#pragma unroll
+        for (int t = 0; t < 8; ++t) {
+            c[t] = sh.hist[255 - lane * 8 - t];
+            sh.hist[255 - lane * 8 - t] = 0;
+            sum += c[t];
+        }
+        const int incl = warp_incl_scan(sum);
+        const int excl = incl - sum;
+        if (excl < k && k <= incl) {
+            int run = excl;
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+                if (run + c[t] >= k) {
+                    sh.bc[0] = 255 - lane * 8 - t;   // bin B of the k-th item
+                    sh.bc[1] = k - run;              // items of B in the top k
+                    sh.bc[2] = c[t];                 // items in B
+                    break;
+                }
+                run += c[t];
+            }
+        }
+    }
+    __syncthreads();
+    const uint32_t B = (uint32_t)sh.bc[0];
+    const int need = sh.bc[1], cntB = sh.bc[2];
+    const bool all_b = need == cntB;
+    // bin B's items wait in the free tail [k, k + cntB) of the destination
+    // (the caller's buffers hold at least 2k items): key, id, source index
+    uint32_t* rk = reinterpret_cast<uint32_t*>(ds + k);
+    int* rid = di + k;
+    int* rsrc = dp + k;
+    if (!all_b && cntB > min(kResolveCap, k)) {
+        topk_compact_radix(s, id, ps, n, k, ds, di, dp, sh);
+        return;
+    }
+    for (int i = tid; i < n; i += blockDim.x) {
+        const uint32_t key = fkey(s[i]);
+        const uint32_t b = (key - kmn) >> shift;
+        if (b > B || (b == B && all_b)) {
+            const int p = atomicAdd(&sh.count2, 1);
+            ds[p] = s[i];
+            di[p] = id[i];
+            dp[p] = ps[i];
+        } else if (b == B) {
+            const int r = atomicAdd(&sh.nres, 1);
+            rk[r] = key;
+            rid[r] = id[i];
+            rsrc[r] = i;
+        }
+    }
+    if (tid == 0) sh.thr = kmn + (B << shift);   // smallest key that falls in bin B
+    __syncthreads();
+    if (!all_b) {
+        // rank of each item of bin B among them (keys are distinct: ids are)
+        for (int r = tid; r < cntB; r += blockDim.x) {
+            const uint32_t xk = rk[r];
+            const int xi = rid[r];
+            int rank = 0;
+            for (int j = 0; j < cntB; ++j) {
+                const uint32_t yk = rk[j];
+                rank += yk > xk || (yk == xk && rid[j] < xi);
+            }
+            if (rank < need) {
+                const int i = rsrc[r];
+                const int p = atomicAdd(&sh.count2, 1);
+                ds[p] = s[i];
+                di[p] = id[i];
+                dp[p] = ps[i];
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// General form: exact k-th key by 8-bit radix passes, then ties by id.
+__device__ void topk_compact_radix(const float* s, const int* id, const int* ps, int n, int k, float* ds, int* di,
+                                   int* dp, SelShared& sh) {
     int need, eq;
     const uint32_t T = block_kth(s, id, n, k, 0, 0u, sh, &need, &eq);
     const bool split = need < eq;
