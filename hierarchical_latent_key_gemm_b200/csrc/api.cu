@@ -340,7 +340,8 @@ int check_select(const lsa_index* ix, const lsa_select_params* sp, const void* Q
 }
 
 int do_select(const lsa_index* ix, const lsa_select_params* sp, const void* Q, int64_t nq, const int64_t* q_pos,
-              int64_t q_pos0, int32_t* idx, int32_t* cnt, int32_t max_sel, void* stream, bool fullscan) {
+              int64_t q_pos0, int32_t* idx, int32_t* cnt, int32_t max_sel, void* stream, bool fullscan,
+              unsigned long long* work = nullptr) {
     int st = check_select(ix, sp, Q, nq, q_pos, q_pos0, idx, cnt, max_sel);
     if (st != LSA_OK || nq == 0) return st;
     cudaStream_t s = as_stream(stream);
@@ -352,9 +353,16 @@ int do_select(const lsa_index* ix, const lsa_select_params* sp, const void* Q, i
     float* qbar = scratch.alloc<float>(p.batch * nq * p.hkv * p.r);
     if (scratch.status != LSA_OK) return scratch.status;
     st = launch_query_latent(Q, ix->W, p.batch, nq, sp->hq, p.hkv, p.d, p.r, p.dtype, qbar, s);
-    if (st == LSA_OK) st = launch_select(ix, sp, qbar, nq, q_pos, q_pos0, idx, cnt, max_sel, fullscan, s);
+    if (st == LSA_OK) st = launch_select(ix, sp, qbar, nq, q_pos, q_pos0, idx, cnt, max_sel, fullscan, s, work);
     scratch.release();
     return st;
+}
+
+// bf16 attention reads Q, K, V rows and writes O in 16-byte pieces
+bool attn_aligned(int dtype, const void* Q, const void* K, const void* V, const void* O) {
+    if (dtype != LSA_BF16) return true;
+    return ((reinterpret_cast<uintptr_t>(Q) | reinterpret_cast<uintptr_t>(K) | reinterpret_cast<uintptr_t>(V) |
+             reinterpret_cast<uintptr_t>(O)) & 15u) == 0;
 }
 
 }  // namespace
@@ -377,6 +385,13 @@ int lsa_select(const lsa_index* index, const lsa_select_params* params, const vo
     return do_select(index, params, Q, nq, q_pos, q_pos0, idx, cnt, max_sel, stream, false);
 }
 
+int lsa_select_work(const lsa_index* index, const lsa_select_params* params, const void* Q, int64_t nq,
+                    const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt, int32_t max_sel,
+                    unsigned long long* scored, void* stream) {
+    if (!scored || !is_device_ptr(scored)) return LSA_ERR_INVALID_ARG;
+    return do_select(index, params, Q, nq, q_pos, q_pos0, idx, cnt, max_sel, stream, false, scored);
+}
+
 int lsa_fullscan_select(const lsa_index* index, const lsa_select_params* params, const void* Q, int64_t nq,
                         const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt, int32_t max_sel,
                         void* stream) {
@@ -395,6 +410,7 @@ int lsa_sparse_attn(const void* Q, const void* K, const void* V, const int32_t* 
         !is_device_ptr(O))
         return LSA_ERR_INVALID_ARG;
     if (lse && !is_device_ptr(lse)) return LSA_ERR_INVALID_ARG;
+    if (!attn_aligned(dtype, Q, K, V, O)) return LSA_ERR_INVALID_ARG;
     return launch_sparse_attn(Q, K, V, idx, cnt, batch, nq, hq, hkv, d, dtype, max_sel, ld_tokens, O, lse,
                               global_err_word(), as_stream(stream));
 }
@@ -413,6 +429,7 @@ int lsa_sparse_attn_banded(const void* Q, const void* K, const void* V, const in
         !is_device_ptr(O))
         return LSA_ERR_INVALID_ARG;
     if (lse && !is_device_ptr(lse)) return LSA_ERR_INVALID_ARG;
+    if (!attn_aligned(dtype, Q, K, V, O)) return LSA_ERR_INVALID_ARG;
     const int G = hq / hkv;
     if (dtype == LSA_BF16 && (G == 1 || G == 2 || G == 4 || G == 8 || G == 16))
         return launch_banded_attn(Q, K, V, idx, cnt, batch, nq, q_pos0, hq, hkv, d, max_sel, ld_tokens, sink, window,

@@ -29,6 +29,7 @@
 #include <algorithm>
 
 #include "lsa_internal.cuh"
+#include "tma_util.cuh"
 #include "warp_mma.cuh"
 
 namespace lsa {
@@ -558,8 +559,20 @@ int launch_band_g(const BandArgs& ba, const GatherArgs& ga, int64_t batch, cudaS
     if (e != cudaSuccess) return cuda_status(e);
     constexpr int QT = kBandRows / G;
     const unsigned units = (unsigned)(batch * ba.hkv);
-    note_launch();
-    attn_band_kernel<D, G><<<dim3((unsigned)((ba.nq + QT - 1) / QT), units), kBandThreads, smem_band, s>>>(ba);
+#ifndef LSA_BAND_MMA_SYNC
+    // tensor-core (tcgen05) band when TMA is usable and every TMA coordinate fits in int32
+    const bool aligned = ((reinterpret_cast<uintptr_t>(ba.Q) | reinterpret_cast<uintptr_t>(ba.K) |
+                           reinterpret_cast<uintptr_t>(ba.V)) & 15u) == 0;
+    if (aligned && batch * ba.nq < INT32_MAX && batch * ba.ld_tokens < INT32_MAX && tma_available()) {
+        const int st = launch_band_tc(ba.Q, ba.K, ba.V, batch, ba.nq, ba.q_pos0, ba.hq, ba.hkv, D, ba.ld_tokens,
+                                      ba.sink, ba.window, ba.part_o, ba.part_ml, ga.err, s);
+        if (st != LSA_OK) return st;
+    } else
+#endif
+    {
+        note_launch();
+        attn_band_kernel<D, G><<<dim3((unsigned)((ba.nq + QT - 1) / QT), units), kBandThreads, smem_band, s>>>(ba);
+    }
     note_launch();
     attn_gather_kernel<D, NT><<<dim3((unsigned)((ga.nq + kGatWarps - 1) / kGatWarps), units), kGatWarps * 32,
                                  smem_gat, s>>>(ga);

@@ -164,7 +164,7 @@ int launch_query_latent(const void* Q, const float* W, int64_t batch, int64_t nq
 // ---------------------------------------------------------------- select
 int launch_select(const lsa_index* ix, const lsa_select_params* sp, const float* qbar, int64_t nq,
                   const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt, int max_sel,
-                  bool fullscan, cudaStream_t s);
+                  bool fullscan, cudaStream_t s, unsigned long long* work = nullptr);
 
 // ---------------------------------------------------------------- attention
 int launch_sparse_attn(const void* Q, const void* K, const void* V, const int32_t* idx,
@@ -174,6 +174,10 @@ int launch_sparse_attn(const void* Q, const void* K, const void* V, const int32_
 int launch_banded_attn(const void* Q, const void* K, const void* V, const int32_t* idx, const int32_t* cnt,
                        int64_t batch, int64_t nq, int64_t q_pos0, int hq, int hkv, int d, int max_sel,
                        int64_t ld_tokens, int sink, int window, void* O, float* lse, int32_t* err, cudaStream_t s);
+// tensor-core band of the banded attention (attn_band_tc.cu): partials as the mma.sync band kernel writes them
+int launch_band_tc(const void* Q, const void* K, const void* V, int64_t batch, int64_t nq, int64_t q_pos0, int hq,
+                   int hkv, int d, int64_t ld_tokens, int sink, int window, float* part_o, float2* part_ml,
+                   int32_t* err, cudaStream_t s);
 
 // ---------------------------------------------------------------- append
 int launch_append(lsa_index* ix, const void* K, int64_t first_block, int64_t n_new_blocks,

@@ -30,6 +30,9 @@ namespace {
 #ifndef LSA_SELECT_UNROLL
 #define LSA_SELECT_UNROLL 1
 #endif
+#ifndef LSA_SELECT_LEAF_SCAN
+#define LSA_SELECT_LEAF_SCAN 1
+#endif
 #ifndef LSA_SELECT_MIN_BLOCKS
 #define LSA_SELECT_MIN_BLOCKS 8
 #endif
@@ -58,6 +61,7 @@ struct SelArgs {
     int32_t* cnt;
     int max_sel;
     int cap;
+    unsigned long long* work;   // optional: += eligible nodes and blocks scored
 };
 
 constexpr int kResolveCap = 256;   // most items of the threshold bin ranked pairwise
@@ -329,7 +333,9 @@ __device__ __forceinline__ int find_owner(const int* pre, int nk, int t) {
 constexpr int kWideThreads = 1024;
 constexpr int kWideCap = 8192;
 
-template <int R, bool FULL, int THREADS>
+// COUNT: also add the number of eligible rows scored to *a.work (a separate
+// instantiation, so the counting costs the timed path nothing)
+template <int R, bool FULL, int THREADS, bool COUNT>
 __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BLOCKS : 1) void select_kernel(
     const SelArgs a) {
     extern __shared__ float4 dyn4[];
@@ -396,6 +402,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
     __syncthreads();
 
     int cur = 0;
+    unsigned nscored = 0;   // eligible candidates this thread's group scored (leader lanes)
     uint32_t lt_mask;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt_mask));
     // Push candidates t in [0, total) through the buffer, keeping the top k.
@@ -440,6 +447,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
                 for (int v = 0; v < kUnroll; ++v) {
                     if (ok[v]) {
                         sc[v] = dot(y[v]);
+                        if (COUNT) nscored += (gl == 0);
                         ok[v] = fkey(sc[v]) >= thr;
                     }
                     bal[v] = __ballot_sync(0xffffffffu, ok[v] && gl == 0);
@@ -526,21 +534,41 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
             __syncthreads();
         }
         // candidate slot range of every kept leaf
+        // (the kept leaves' original ids are still in the buffer; a leaf's
+        // block ids ascend, so its candidates are the run between the counts
+        // of ids below b_lo and of ids up to b_hi, read 16 at a time so the
+        // loads of a leaf are in flight together)
         const int nk = sh.nkept;
         const int L = a.n_l[a.levels - 1];
-        const int32_t* oidl = a.oid[a.levels - 1] + (int64_t)u * L;
+        const int* kept_id = bib(cur);
         for (int e = threadIdx.x; e < nk; e += blockDim.x) {
-            const int leaf = oidl[kk[e]];
-            const int64_t c = (int64_t)u * L + leaf;
+            const int64_t c = (int64_t)u * L + kept_id[e];
             const int st = a.leaf_start[c];
             const int cntl = a.leaf_cnt[c];
             const int32_t* bl = a.blk + st;
-            int lo1 = 0, hi1 = cntl;  // first index with bl >= b_lo
-            while (lo1 < hi1) { const int m = (lo1 + hi1) >> 1; if (bl[m] < b_lo) lo1 = m + 1; else hi1 = m; }
-            int lo2 = lo1, hi2 = cntl; // first index with bl > b_hi
-            while (lo2 < hi2) { const int m = (lo2 + hi2) >> 1; if (bl[m] <= b_hi) lo2 = m + 1; else hi2 = m; }
-            lo[e] = st + lo1;
-            pre[e] = lo2 - lo1;
+            int nlo = 0, nle = 0;
+#if LSA_SELECT_LEAF_SCAN
+            for (int j0 = 0; j0 < cntl; j0 += 16) {
+                int v[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) v[j] = j0 + j < cntl ? __ldg(bl + j0 + j) : INT32_MAX;
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                    nlo += v[j] < b_lo;
+                    nle += v[j] <= b_hi;
+                }
+            }
+#else
+            {
+                int hi = cntl;   // first index with bl >= b_lo
+                while (nlo < hi) { const int m = (nlo + hi) >> 1; if (bl[m] < b_lo) nlo = m + 1; else hi = m; }
+                nle = nlo;
+                hi = cntl;       // first index with bl > b_hi
+                while (nle < hi) { const int m = (nle + hi) >> 1; if (bl[m] <= b_hi) nle = m + 1; else hi = m; }
+            }
+#endif
+            lo[e] = st + nlo;
+            pre[e] = max(0, nle - nlo);
         }
         scan_pre(pre, nk);
         if (threadIdx.x == 0) sh.count = 0;
@@ -661,26 +689,44 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
         }
     }
 
-    const int64_t lo_w = max((int64_t)0, pos - a.window + 1);
-    const int64_t ns = min((int64_t)a.sink, lo_w);
-    const int64_t nblk_tok = (int64_t)nsel * a.pool;
-    const int64_t total = ns + nblk_tok + (pos - lo_w + 1);
+    // row = sink [0, ns) | blocks (P tokens each, ascending) | window [lo_w, pos] | -1 padding;
+    // positions fit in int32 (checked by the caller), so no 64-bit division here
+    const int lo_w = (int)max((int64_t)0, pos - a.window + 1);
+    const int ns = min(a.sink, lo_w);
+    const int nblk_tok = nsel * a.pool;
+    const int total = ns + nblk_tok + ((int)pos - lo_w + 1);
     int32_t* out = a.idx + row * a.max_sel;
+    // (consecutive threads write consecutive entries: the row is written coalesced)
+    const unsigned P = (unsigned)a.pool;
     for (int e = threadIdx.x; e < a.max_sel; e += blockDim.x) {
-        int64_t v;
-        if (e < ns) v = e;
-        else if (e < ns + nblk_tok) { const int64_t t = e - ns; v = (int64_t)arr[t / a.pool] * a.pool + t % a.pool; }
-        else if (e < total) v = lo_w + (e - ns - nblk_tok);
-        else v = -1;
-        out[e] = (int32_t)v;
+        int v;
+        if (e < ns) {
+            v = e;
+        } else if (e < ns + nblk_tok) {
+            const unsigned t = (unsigned)(e - ns);
+            const unsigned j = t / P;
+            v = arr[j] * a.pool + (int)(t - j * P);
+        } else if (e < total) {
+            v = lo_w + (e - ns - nblk_tok);
+        } else {
+            v = -1;
+        }
+        out[e] = v;
     }
     if (threadIdx.x == 0) a.cnt[row] = (int32_t)total;
+    if (COUNT) {
+        unsigned long long w = nscored;
+#pragma unroll
+        for (int o = 16; o >= 1; o >>= 1) w += __shfl_xor_sync(0xffffffffu, w, o);
+        if (lane == 0) atomicAdd(a.work, w);
+    }
 }
 
 template <int R, int THREADS>
 int launch_select_t(const SelArgs& a, int64_t nq, int64_t units, bool fullscan, cudaStream_t s) {
     const size_t smem = (size_t)a.cap * 24 + (size_t)(3 * a.beam + 1) * 4;
-    auto kern = fullscan ? select_kernel<R, true, THREADS> : select_kernel<R, false, THREADS>;
+    auto kern = fullscan ? select_kernel<R, true, THREADS, false>
+                         : (a.work ? select_kernel<R, false, THREADS, true> : select_kernel<R, false, THREADS, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_status(e);
     dim3 grid((unsigned)nq, (unsigned)units);
@@ -708,7 +754,7 @@ int launch_select_r(const SelArgs& a, int64_t nq, int64_t units, bool fullscan, 
 
 int launch_select(const lsa_index* ix, const lsa_select_params* sp, const float* qbar, int64_t nq,
                   const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt, int max_sel, bool fullscan,
-                  cudaStream_t s) {
+                  cudaStream_t s, unsigned long long* work) {
     const lsa_build_params& p = ix->p;
     if (sp->beam > 1024) return LSA_ERR_INVALID_ARG;
     SelArgs a{};
@@ -740,6 +786,7 @@ int launch_select(const lsa_index* ix, const lsa_select_params* sp, const float*
     a.idx = idx;
     a.cnt = cnt;
     a.max_sel = max_sel;
+    a.work = work;
     const int kmax = a.kb > a.beam ? a.kb : a.beam;
     int cap = 1024;
     while (cap < 2 * kmax) cap <<= 1;

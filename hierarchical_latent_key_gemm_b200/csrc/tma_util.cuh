@@ -59,5 +59,17 @@ __device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, u
 bool tma_available();
 bool make_tensor_map_2d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, int64_t rows, int64_t width,
                         int64_t row_stride_bytes, int box_w, int box_h);
+// 3D map, 128-byte swizzle: dims[0] innermost (contiguous), strides of dims 1
+// and 2 in bytes, box extents per dimension.
+bool make_tensor_map_3d(CUtensorMap* m, CUtensorMapDataType dt, const void* base, const int64_t dims[3],
+                        const int64_t strides_bytes[2], const int box[3]);
+
+__device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y, int z) {
+    asm volatile(
+        "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4, %5}], "
+        "[%2];" ::"r"(su32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(su32(bar)), "r"(x), "r"(y), "r"(z)
+        : "memory");
+}
 
 }  // namespace lsa

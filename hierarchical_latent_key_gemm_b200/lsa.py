@@ -57,6 +57,7 @@ _SIGS = {
                                          _vp, C.POINTER(_vp)]),
     "lsa_select": (_i32, [_vp, C.POINTER(SelectParams), _vp, _i64, _vp, _i64, _vp, _vp, _i32, _vp]),
     "lsa_fullscan_select": (_i32, [_vp, C.POINTER(SelectParams), _vp, _i64, _vp, _i64, _vp, _vp, _i32, _vp]),
+    "lsa_select_work": (_i32, [_vp, C.POINTER(SelectParams), _vp, _i64, _vp, _i64, _vp, _vp, _i32, _vp, _vp]),
     "lsa_select_noalloc": (_i32, [_vp, C.POINTER(SelectParams), _vp, _i64, _vp, _i64, _vp, _vp, _i32, _vp]),
     "lsa_sparse_attn": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _i64, _vp, _vp,
                                _vp]),
@@ -248,6 +249,19 @@ def lsa_select_noalloc(index, sp, Q, idx, cnt, q_pos=None, q_pos0=0, stream=None
                                   _ptr(idx), _ptr(cnt), int(idx.shape[-1]), _stream(stream))
     _ok(st, "lsa_select_noalloc")
     return idx, cnt
+
+
+def lsa_select_work(index, sp, Q, q_pos=None, q_pos0=0, idx=None, cnt=None, max_sel=None, stream=None):
+    """lsa_select plus the number of eligible nodes and blocks whose latent
+    rows were scored (a Python int; synchronises the stream)."""
+    scored = torch.zeros(1, dtype=torch.int64, device=Q.device)
+
+    def fn(h, spp, q, nq, qp, qp0, ii, cc, ms, st):
+        return lib().lsa_select_work(h, spp, q, nq, qp, qp0, ii, cc, ms, _ptr(scored), st)
+
+    idx, cnt = _select(fn, "lsa_select_work", index, sp, Q, q_pos=q_pos, q_pos0=q_pos0, idx=idx, cnt=cnt,
+                       max_sel=max_sel, stream=stream)
+    return idx, cnt, int(scored.item())
 
 
 def lsa_fullscan_select(index, sp, Q, **kw):

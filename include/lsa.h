@@ -190,6 +190,17 @@ int lsa_select_noalloc(const lsa_index* index, const lsa_select_params* params, 
                        int64_t nq, const int64_t* q_pos, int64_t q_pos0,
                        int32_t* idx, int32_t* cnt, int32_t max_sel, void* stream);
 
+/* lsa_select that also adds to *scored (a device uint64 the caller zeroes)
+ * the number of eligible tree nodes and candidate blocks whose latent rows it
+ * scored, summed over all (query, KV head) pairs: the work count behind a
+ * bytes-moved figure (each scored row is r floats).  Same results as
+ * lsa_select; costs one atomic add per warp.  The pages give no counterpart:
+ * it exists for measurement. */
+int lsa_select_work(const lsa_index* index, const lsa_select_params* params, const void* Q,
+                    int64_t nq, const int64_t* q_pos, int64_t q_pos0,
+                    int32_t* idx, int32_t* cnt, int32_t max_sel, unsigned long long* scored,
+                    void* stream);
+
 /* The quadratic baseline indexer: every candidate block is scored, no tree.
  * Same arguments and output format as lsa_select (beam is ignored).
  * [p3 flowchart, red path "Full key scan"] */
@@ -205,7 +216,8 @@ int lsa_fullscan_select(const lsa_index* index, const lsa_select_params* params,
  * O[q,h] = sum_j softmax_j(q_h . k_j / sqrt(d)) v_j over the row of KV head
  * h / (hq/hkv); fp32 accumulation.  A row with cnt = 0 yields O = 0 and
  * lse = -inf.  An index outside [0, ld_tokens) is skipped and latched as
- * LSA_ERR_DEVICE.  [p5 step 3 "the attention kernel is unchanged"; p3
+ * LSA_ERR_DEVICE.  For bf16, Q, K, V and O must be 16-byte aligned (else
+ * LSA_ERR_INVALID_ARG).  [p5 step 3 "the attention kernel is unchanged"; p3
  * flowchart "exact over subset"] */
 int lsa_sparse_attn(const void* Q, const void* K, const void* V, const int32_t* idx,
                     const int32_t* cnt, int64_t batch, int64_t nq, int32_t hq, int32_t hkv,

@@ -227,3 +227,21 @@ def test_banded_argument_errors():
     with pytest.raises(lsa.LsaError):
         lsa.lsa_sparse_attn_banded(inp["Q"], inp["K"], inp["V"], idx, cnt, w.hkv, -1, w.window)
     assert lsa.lsa_check(None) == lsa.LSA_OK
+
+
+def test_attention_rejects_unaligned_bf16_buffers():
+    """bf16 attention moves rows in 16-byte pieces: a buffer that is not
+    16-byte aligned is refused before anything is launched."""
+    w = WORKLOADS["gqa_128k"].scaled(n_tokens=256, level_sizes=(2, 8), needles=0, components=16)
+    inp = make_inputs(w, seed=13, device="cuda")
+    idx = torch.zeros((1, 256, w.hkv, w.max_sel), dtype=torch.int32, device="cuda")
+    cnt = torch.ones((1, 256, w.hkv), dtype=torch.int32, device="cuda")
+    K = inp["K"]
+    flat = torch.empty(K.numel() + 4, dtype=K.dtype, device="cuda")
+    Kmis = flat[4:].view(K.shape)          # 8-byte offset
+    Kmis.copy_(K)
+    with pytest.raises(lsa.LsaError):
+        lsa.lsa_sparse_attn(inp["Q"], Kmis, inp["V"], idx, cnt, w.hkv)
+    with pytest.raises(lsa.LsaError):
+        lsa.lsa_sparse_attn_banded(inp["Q"], Kmis, inp["V"], idx, cnt, w.hkv, w.sink, w.window)
+    assert lsa.lsa_check(None) == lsa.LSA_OK

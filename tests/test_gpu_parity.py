@@ -506,3 +506,35 @@ def test_append_capacity_error_is_latched():
     lsa.lsa_append(ix, K, 64)
     assert lsa.lsa_check(ix) == lsa.LSA_ERR_CAPACITY
     ix.free()
+
+
+def test_select_work_counts_scored_rows():
+    """lsa_select_work returns lsa_select's rows and counts the eligible nodes
+    and blocks it scored.  With a beam wider than every level the tree search
+    scores every eligible node of every level and every candidate block, so
+    the count has a closed form from the index's minpos and the positions."""
+    w = WORKLOADS["gqa_128k"].scaled(n_tokens=4096 + 5, level_sizes=(8, 64), needles=0, components=64)
+    inp = make_inputs(w, seed=12, device="cuda")
+    ix = lsa.lsa_build_index(TU.build_params(w), inp["K"], inp["W"])
+    sp = TU.select_params(w, beam=1024)
+    i1, c1 = lsa.lsa_select(ix, sp, inp["Q"])
+    i2, c2, scored = lsa.lsa_select_work(ix, sp, inp["Q"])
+    assert torch.equal(i1, i2) and torch.equal(c1, c2)
+    pos = np.arange(w.n_tokens, dtype=np.int64)
+    bound = pos - w.window - w.pool + 1
+    want = 0
+    for lvl in range(len(w.level_sizes)):
+        mp = ix.get(lsa.LSA_GET_MINPOS, lvl).cpu().numpy()          # [units][n_l]
+        for u in range(mp.shape[0]):
+            srt = np.sort(mp[u])
+            want += int(np.searchsorted(srt, bound, side="right").sum())
+    b_lo = -(-w.sink // w.pool)
+    b_hi = np.where(bound >= 0, bound // w.pool, -1)
+    nblk = np.maximum(0, np.minimum(b_hi, w.n_tokens // w.pool - 1) - b_lo + 1)
+    want += int(nblk.sum()) * w.hkv
+    assert scored == want
+    # the narrow beam of the workload scores fewer rows
+    _, _, narrow = lsa.lsa_select_work(ix, TU.select_params(w), inp["Q"])
+    assert 0 < narrow <= scored
+    assert lsa.lsa_check(ix) == lsa.LSA_OK
+    ix.free()
