@@ -49,6 +49,10 @@ constexpr int kBandStages = 3;
 constexpr int kGatWarps = LSA_GAT_WARPS;    // queries per CTA (one warp each)
 constexpr int kGatSlice = 16;               // keys per slice
 constexpr int kGatStages = LSA_GAT_STAGES;  // slices in each warp's ring
+#ifndef LSA_GAT_TQ
+#define LSA_GAT_TQ 1
+#endif
+constexpr int kGatTQ = LSA_GAT_TQ;          // slices of token ids read ahead of their copies
 
 struct BandArgs {
     const __nv_bfloat16* Q;
@@ -411,20 +415,33 @@ __global__ __launch_bounds__(kGatWarps * 32) void attn_gather_kernel(const Gathe
             cp_async16(vb + dsto[k], src + vk, nbytes);
         }
     };
-    int tok_next = fetch_tok(0);
+    // token ids of the next TQ slices to load, oldest first (loads issued TQ
+    // slices before the rows they address are copied)
+    int tokq[kGatTQ];
+#pragma unroll
+    for (int j = 0; j < kGatTQ; ++j) tokq[j] = fetch_tok(j);
+    auto pop_tok = [&](int s_next) -> int {
+        const int t0 = tokq[0];
+#pragma unroll
+        for (int j = 0; j + 1 < kGatTQ; ++j) tokq[j] = tokq[j + 1];
+        tokq[kGatTQ - 1] = fetch_tok(s_next);
+        return t0;
+    };
 #pragma unroll
     for (int s = 0; s < kGatStages - 1; ++s) {
-        if (s < nslice) load_slice(s, tok_next);
+        const int tk = pop_tok(s + kGatTQ);
+        if (s < nslice) load_slice(s, tk);
         cp_async_commit();
-        tok_next = fetch_tok(s + 1);
     }
 
     for (int s = 0; s < nslice; ++s) {
         cp_async_wait<kGatStages - 2>();
         __syncwarp();
-        if (s + kGatStages - 1 < nslice) load_slice(s + kGatStages - 1, tok_next);
+        {
+            const int tk = pop_tok(s + kGatStages - 1 + kGatTQ);
+            if (s + kGatStages - 1 < nslice) load_slice(s + kGatStages - 1, tk);
+        }
         cp_async_commit();
-        tok_next = fetch_tok(s + kGatStages);
         const int st = s % kGatStages;
         const uint32_t kb = smem_u32(Ks + st * SLICE_BYTES), vb = smem_u32(Vs + st * SLICE_BYTES);
         // S^T = K_slice Q^T: rows = 16 keys, cols = heads
