@@ -149,17 +149,20 @@ def kernel_source_sha(fname: str) -> str:
 
 
 def recorded_traffic(kernel: str, workload: str, src: str):
-    """DRAM bytes per launch recorded from an ncu capture (profiles/traffic.json),
+    """DRAM bytes per launch recorded from an ncu capture (profiles/traffic.txt),
     or None when absent or when the kernel source changed since."""
-    p = os.path.join(ROOT, "profiles", "traffic.json")
+    p = os.path.join(ROOT, "profiles", "traffic.txt")
     if not os.path.exists(p):
         return None
+    sha = kernel_source_sha(src)
     with open(p) as f:
-        d = json.load(f)
-    e = d.get(kernel, {}).get(workload)
-    if not e or e.get("source_sha") != kernel_source_sha(src):
-        return None
-    return e.get("dram_bytes_per_launch")
+        for line in f:
+            if line.startswith("#") or "|" not in line:
+                continue
+            parts = [x.strip() for x in line.split("|")]
+            if len(parts) >= 5 and parts[0] == kernel and parts[1] == workload and parts[2] == src:
+                return int(parts[4]) if parts[3] == sha else None
+    return None
 
 
 # ------------------------------------------------------------------ our arm
