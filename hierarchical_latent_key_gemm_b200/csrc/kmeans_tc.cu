@@ -222,9 +222,17 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         const float* ccu = cc + (int64_t)u * k;
         for (int t = 0; t < ntile; ++t) {
             const int buf = t & 1;
+            // the tile's centroid norms, one per lane per 32-column chunk, read
+            // before the wait and handed to every lane by shuffles
+            float ccr[kTN / 32];
+#pragma unroll
+            for (int cb = 0; cb < kTN / 32; ++cb) {
+                const int j = t * kTN + cb * 32 + lane;
+                ccr[cb] = j < k ? __ldg(ccu + j) : 0.f;
+            }
             if (!mbar_wait(acc_full + buf, (uint32_t)(t >> 1) & 1u)) { ok = false; latch(err, kErrTimeout); break; }
             asm volatile("tcgen05.fence::after_thread_sync;");
-#pragma unroll 1
+#pragma unroll
             for (int cb = 0; cb < kTN / 32; ++cb) {
                 float v[32];
                 tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + buf * kTN + cb * 32, v);
@@ -232,10 +240,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int j = j0 + i;
-                    if (j < k) {
-                        const float dist = __fmaf_rn(-2.f, v[i], __ldg(ccu + j));
-                        if (dist < best) { best = dist; bestj = j; }
-                    }
+                    const float dist = __fmaf_rn(-2.f, v[i], __shfl_sync(0xffffffffu, ccr[cb], i));
+                    if (j < k && dist < best) { best = dist; bestj = j; }
                 }
             }
             asm volatile("tcgen05.fence::before_thread_sync;");
