@@ -41,7 +41,7 @@ constexpr int kBandTile = 64;       // keys per pipeline stage
 constexpr int kBandStages = 3;
 
 #ifndef LSA_GAT_WARPS
-#define LSA_GAT_WARPS 2
+#define LSA_GAT_WARPS 1
 #endif
 #ifndef LSA_GAT_STAGES
 #define LSA_GAT_STAGES 2

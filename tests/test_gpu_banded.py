@@ -245,3 +245,29 @@ def test_attention_rejects_unaligned_bf16_buffers():
     with pytest.raises(lsa.LsaError):
         lsa.lsa_sparse_attn_banded(inp["Q"], Kmis, inp["V"], idx, cnt, w.hkv, w.sink, w.window)
     assert lsa.lsa_check(None) == lsa.LSA_OK
+
+
+def test_host_prefill_pipeline_matches_device_path():
+    """The overlapped host-to-host layer (K, V, W up; Q up and O down in
+    chunks around select + banded attention on three streams) gives the
+    device path's output: the same selections, attention within 2 bf16 ulps
+    (band tiles start at each chunk's first query)."""
+    from hierarchical_latent_key_gemm_b200.pipeline import HostPrefill
+    w = WORKLOADS["gqa_128k"].scaled(n_tokens=6000 + 7, level_sizes=(8, 64), needles=0, components=256)
+    inp = make_inputs(w, seed=14)
+    hQ, hK, hV, hW = (inp[k].pin_memory() for k in ("Q", "K", "V", "W"))
+    hO = torch.empty(hQ.shape, dtype=hQ.dtype, pin_memory=True)
+    bp, sp = TU.build_params(w), TU.select_params(w)
+    hp = HostPrefill(bp, sp, hQ, hK, hV, hW, hO, w.sink, w.window, chunks=5)
+    for _ in range(2):
+        hp.run().free()
+        torch.cuda.synchronize()
+    d = _dev(inp)
+    ix = lsa.lsa_build_index(bp, d["K"], d["W"])
+    idx, cnt = lsa.lsa_select(ix, sp, d["Q"])
+    O_, _ = lsa.lsa_sparse_attn_banded(d["Q"], d["K"], d["V"], idx, cnt, w.hkv, w.sink, w.window)
+    assert lsa.lsa_check(ix) == lsa.LSA_OK
+    ref = O_.float().cpu()
+    got = hO.float()
+    assert bool(((got - ref).abs() <= ref.abs() * 2.0 ** -6 + 1e-3).all())
+    ix.free()
