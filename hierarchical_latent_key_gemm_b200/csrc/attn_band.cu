@@ -7,10 +7,11 @@
 // so they are read once per tile of consecutive queries instead of once per
 // query:
 //
-//   attn_band_kernel    dense tiles: 128 (query, head) rows per CTA against the
-//                       contiguous key band [0, S) and [i0-W+1, i1], with the
-//                       per-row mask j <= i && (j < S || j >= i-W+1); writes an
-//                       unnormalised partial (acc, running max, sum of weights).
+//   attn_band_tc_kernel (attn_band_tc.cu) dense tcgen05 tiles: 128 (query,
+//                       head) rows per CTA against the contiguous key band
+//                       [0, S) and [i0-W+1, i1], with the per-row mask
+//                       j <= i && (j < S || j >= i-W+1); writes an unnormalised
+//                       partial (acc, running max, sum of weights).
 //   attn_gather_kernel  one warp per (query, KV head): the long-range entries of
 //                       the row list only, starting from the band partial, and
 //                       writes the normalised output.
@@ -35,10 +36,6 @@
 namespace lsa {
 namespace {
 
-constexpr int kBandThreads = 256;   // 8 warps x 16 rows
-constexpr int kBandRows = 128;      // (query, head) rows per CTA
-constexpr int kBandTile = 64;       // keys per pipeline stage
-constexpr int kBandStages = 3;
 
 #ifndef LSA_GAT_WARPS
 #define LSA_GAT_WARPS 1
@@ -49,10 +46,7 @@ constexpr int kBandStages = 3;
 constexpr int kGatWarps = LSA_GAT_WARPS;    // queries per CTA (one warp each)
 constexpr int kGatSlice = 16;               // keys per slice
 constexpr int kGatStages = LSA_GAT_STAGES;  // slices in each warp's ring
-#ifndef LSA_GAT_TQ
-#define LSA_GAT_TQ 1
-#endif
-constexpr int kGatTQ = LSA_GAT_TQ;          // slices of token ids read ahead of their copies
+constexpr int kGatTQ = 1;                   // slices of token ids read ahead of their copies
 
 struct BandArgs {
     const __nv_bfloat16* Q;
@@ -64,222 +58,6 @@ struct BandArgs {
     float* part_o;    // [batch*nq*hq][D] unnormalised sum of p * v
     float2* part_ml;  // [batch*nq*hq] (running max in log2 units, sum of weights)
 };
-
-template <int D, int G>
-__global__ __launch_bounds__(kBandThreads, 1) void attn_band_kernel(const BandArgs a) {
-    constexpr int CH = D / 8;
-    constexpr int QT = kBandRows / G;   // queries per CTA
-    constexpr int QW = 16 / G;          // queries per warp
-    constexpr int TILE_BYTES = kBandTile * D * 2;
-    extern __shared__ __align__(128) unsigned char smem[];
-    unsigned char* Ks = smem;                                  // [stages][64][D]
-    unsigned char* Vs = smem + kBandStages * TILE_BYTES;       // [stages][64][D]
-    unsigned char* Qs = smem + 2 * kBandStages * TILE_BYTES;   // [128][D]
-
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int u = blockIdx.y;
-    const int64_t b = u / a.hkv;
-    const int h = u % a.hkv;
-    const int64_t q0 = (int64_t)blockIdx.x * QT;
-    const int64_t qlast = min(a.nq, q0 + QT) - 1;
-    const int64_t i0 = a.q_pos0 + q0, i1 = a.q_pos0 + qlast;
-    // key segments: sink [0, s_end) and window [w_beg, w_end)
-    const int64_t s_end = min((int64_t)a.sink, i1 + 1);
-    const int64_t w_beg = max((int64_t)a.sink, i0 - a.window + 1);
-    const int64_t w_end = i1 + 1;
-    const int nt_s = (int)((s_end + kBandTile - 1) / kBandTile);
-    const int nt_w = w_end > w_beg ? (int)((w_end - w_beg + kBandTile - 1) / kBandTile) : 0;
-    const int ntile = nt_s + nt_w;
-    auto tile_range = [&](int t, int64_t& jb, int64_t& je) {
-        if (t < nt_s) {
-            jb = (int64_t)t * kBandTile;
-            je = min(jb + kBandTile, s_end);
-        } else {
-            jb = w_beg + (int64_t)(t - nt_s) * kBandTile;
-            je = min(jb + kBandTile, w_end);
-        }
-    };
-
-    // Q rows: row r = (query q0 + r / G, head r % G); rows past nq are zero
-    const uint32_t qsb = smem_u32(Qs);
-    for (int e = tid; e < kBandRows * CH; e += kBandThreads) {
-        const int r = e / CH, c = e % CH;
-        const int64_t q = q0 + r / G;
-        const bool ok = q < a.nq;
-        const __nv_bfloat16* src = a.Q + (((b * a.nq + (ok ? q : 0)) * a.hq + (int64_t)h * G + r % G) * D + c * 8);
-        cp_async16(qsb + swz<D>(r, c), src, ok ? 16 : 0);
-    }
-    cp_async_commit();
-
-    const __nv_bfloat16* kbase = a.K + (b * a.ld_tokens * a.hkv + h) * D;
-    const __nv_bfloat16* vbase = a.V + (b * a.ld_tokens * a.hkv + h) * D;
-    auto load_tile = [&](int t) {
-        int64_t jb, je;
-        tile_range(t, jb, je);
-        const int st = t % kBandStages;
-        const uint32_t kb = smem_u32(Ks + st * TILE_BYTES), vb = smem_u32(Vs + st * TILE_BYTES);
-        for (int e = tid; e < kBandTile * CH; e += kBandThreads) {
-            const int r = e / CH, c = e % CH;
-            const int64_t j = jb + r;
-            const bool ok = j < je;
-            const int64_t off = (ok ? j : 0) * a.hkv * D + c * 8;
-            cp_async16(kb + swz<D>(r, c), kbase + off, ok ? 16 : 0);
-            cp_async16(vb + swz<D>(r, c), vbase + off, ok ? 16 : 0);
-        }
-    };
-#pragma unroll
-    for (int t = 0; t < kBandStages - 1; ++t) {
-        if (t < ntile) load_tile(t);
-        cp_async_commit();
-    }
-    cp_async_wait<kBandStages - 1>();   // the Q group
-    __syncthreads();
-
-    // A-fragment row of this lane in the warp's 16 Q rows (re-read per k step)
-    const int qrow = warp * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
-    // this thread's two rows and their query positions
-    const int r0 = warp * 16 + (lane >> 2), r1 = r0 + 8;
-    const int64_t pa = i0 + r0 / G, pb = i0 + r1 / G;
-    const bool va = q0 + r0 / G <= qlast, vb_ = q0 + r1 / G <= qlast;
-    const int64_t wlo = i0 + warp * QW, whi = min(i0 + warp * QW + QW - 1, i1);
-    const bool warp_live = q0 + warp * QW <= qlast;
-
-    float o[D / 8][4];
-#pragma unroll
-    for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-
-    for (int t = 0; t < ntile; ++t) {
-        cp_async_wait<kBandStages - 2>();
-        __syncthreads();
-        if (t + kBandStages - 1 < ntile) load_tile(t + kBandStages - 1);
-        cp_async_commit();
-        int64_t jb, je;
-        tile_range(t, jb, je);
-        const bool sink_tile = t < nt_s;
-        // does any (row, key) of this warp survive the mask?
-        const bool live = warp_live && jb <= whi && (sink_tile || je - 1 >= wlo - a.window + 1);
-        if (!live) continue;
-        const bool full = je - jb == kBandTile && je - 1 <= wlo && (sink_tile || jb >= whi - a.window + 1) &&
-                          q0 + warp * QW + QW - 1 <= qlast;
-        const int st = t % kBandStages;
-        const uint32_t kb = smem_u32(Ks + st * TILE_BYTES), vb = smem_u32(Vs + st * TILE_BYTES);
-        // S = Q K^T over 64 keys: k steps outermost, so the 8 accumulators
-        // are 8 independent chains
-        float s[8][4];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) s[j][0] = s[j][1] = s[j][2] = s[j][3] = 0.f;
-#pragma unroll
-        for (int kt = 0; kt < D / 16; ++kt) {
-            uint32_t qa[4];
-            ldsm_x4(qsb + swz<D>(qrow, 2 * kt + (lane >> 4)), qa[0], qa[1], qa[2], qa[3]);
-#pragma unroll
-            for (int np = 0; np < 4; ++np) {
-                uint32_t b0, b1, b2, b3;
-                ldsm_x4(kb + swz<D>(np * 16 + (lane & 7) + 8 * (lane >> 4), 2 * kt + ((lane >> 3) & 1)), b0, b1,
-                        b2, b3);
-                mma_bf16(s[2 * np], qa, b0, b1);
-                mma_bf16(s[2 * np + 1], qa, b2, b3);
-            }
-        }
-        // scale and mask: key j = jb + 8 * nt + 2 * (lane & 3) + (e & 1)
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                float x = s[nt][e] * a.scale_log2;
-                if (!full) {
-                    const int64_t j = jb + 8 * nt + 2 * (lane & 3) + (e & 1);
-                    const int64_t i = e < 2 ? pa : pb;
-                    const bool ok = (e < 2 ? va : vb_) && j < je && j <= i && (sink_tile || j >= i - a.window + 1);
-                    x = ok ? x : -INFINITY;
-                }
-                s[nt][e] = x;
-            }
-        }
-        float mx0 = -INFINITY, mx1 = -INFINITY;
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            mx0 = fmaxf(mx0, fmaxf(s[nt][0], s[nt][1]));
-            mx1 = fmaxf(mx1, fmaxf(s[nt][2], s[nt][3]));
-        }
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-        const float al0 = (mn0 == -INFINITY) ? 1.f : exp2f(m0 - mn0);
-        const float al1 = (mn1 == -INFINITY) ? 1.f : exp2f(m1 - mn1);
-        float ls0 = 0.f, ls1 = 0.f;
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt) {
-            s[nt][0] = (mn0 == -INFINITY) ? 0.f : exp2f(s[nt][0] - mn0);
-            s[nt][1] = (mn0 == -INFINITY) ? 0.f : exp2f(s[nt][1] - mn0);
-            s[nt][2] = (mn1 == -INFINITY) ? 0.f : exp2f(s[nt][2] - mn1);
-            s[nt][3] = (mn1 == -INFINITY) ? 0.f : exp2f(s[nt][3] - mn1);
-            ls0 += s[nt][0] + s[nt][1];
-            ls1 += s[nt][2] + s[nt][3];
-        }
-        l0 = l0 * al0 + ls0;
-        l1 = l1 * al1 + ls1;
-        m0 = mn0;
-        m1 = mn1;
-        if (__any_sync(0xffffffffu, al0 != 1.f || al1 != 1.f)) {
-#pragma unroll
-            for (int i = 0; i < D / 8; ++i) {
-                o[i][0] *= al0; o[i][1] *= al0;
-                o[i][2] *= al1; o[i][3] *= al1;
-            }
-        }
-        // O += P V, 16 keys per k step, P = hi + lo
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-            uint32_t ph[4], pl[4];
-            split_pack(s[2 * kk][0], s[2 * kk][1], ph[0], pl[0]);
-            split_pack(s[2 * kk][2], s[2 * kk][3], ph[1], pl[1]);
-            split_pack(s[2 * kk + 1][0], s[2 * kk + 1][1], ph[2], pl[2]);
-            split_pack(s[2 * kk + 1][2], s[2 * kk + 1][3], ph[3], pl[3]);
-            const int vr = kk * 16 + (lane & 7) + 8 * ((lane >> 3) & 1);
-            // per half of the d columns: fragments first, then the hi and the
-            // lo pass (8 MMAs apart on each accumulator)
-#pragma unroll
-            for (int hf = 0; hf < D / 64; ++hf) {
-                uint32_t vf[4][4];
-#pragma unroll
-                for (int j = 0; j < 4; ++j)
-                    ldsm_x4_t(vb + swz<D>(vr, hf * 8 + 2 * j + (lane >> 4)), vf[j][0], vf[j][1], vf[j][2], vf[j][3]);
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    mma_bf16(o[hf * 8 + 2 * j], ph, vf[j][0], vf[j][1]);
-                    mma_bf16(o[hf * 8 + 2 * j + 1], ph, vf[j][2], vf[j][3]);
-                }
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    mma_bf16(o[hf * 8 + 2 * j], pl, vf[j][0], vf[j][1]);
-                    mma_bf16(o[hf * 8 + 2 * j + 1], pl, vf[j][2], vf[j][3]);
-                }
-            }
-        }
-    }
-    cp_async_wait<0>();
-
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
-    const int64_t ga = ((b * a.nq + q0 + r0 / G) * a.hq + (int64_t)h * G + r0 % G);
-    const int64_t gb = ((b * a.nq + q0 + r1 / G) * a.hq + (int64_t)h * G + r1 % G);
-#pragma unroll
-    for (int nt = 0; nt < D / 8; ++nt) {
-        const int c = nt * 8 + 2 * (lane & 3);
-        if (va) *reinterpret_cast<float2*>(a.part_o + ga * D + c) = make_float2(o[nt][0], o[nt][1]);
-        if (vb_) *reinterpret_cast<float2*>(a.part_o + gb * D + c) = make_float2(o[nt][2], o[nt][3]);
-    }
-    if ((lane & 3) == 0) {
-        if (va) a.part_ml[ga] = make_float2(m0, l0);
-        if (vb_) a.part_ml[gb] = make_float2(m1, l1);
-    }
-}
 
 struct GatherArgs {
     const __nv_bfloat16* Q;
@@ -566,33 +344,17 @@ __global__ __launch_bounds__(kGatWarps * 32) void attn_gather_kernel(const Gathe
 
 template <int D, int G>
 int launch_band_g(const BandArgs& ba, const GatherArgs& ga, int64_t batch, cudaStream_t s) {
-    const size_t smem_band = (size_t)2 * kBandStages * kBandTile * D * 2 + (size_t)kBandRows * D * 2;
-    cudaError_t e = cudaFuncSetAttribute(attn_band_kernel<D, G>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem_band);
-    if (e != cudaSuccess) return cuda_status(e);
     constexpr int NT = (G + 7) / 8;
     const size_t smem_gat = (size_t)kGatWarps * 2 * kGatStages * kGatSlice * D * 2 + kGatWarps * kGatStages * 4;
-    e = cudaFuncSetAttribute(attn_gather_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_gat);
+    cudaError_t e = cudaFuncSetAttribute(attn_gather_kernel<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem_gat);
     if (e != cudaSuccess) return cuda_status(e);
-    constexpr int QT = kBandRows / G;
-    const unsigned units = (unsigned)(batch * ba.hkv);
-#ifndef LSA_BAND_MMA_SYNC
-    // tensor-core (tcgen05) band when TMA is usable and every TMA coordinate fits in int32
-    const bool aligned = ((reinterpret_cast<uintptr_t>(ba.Q) | reinterpret_cast<uintptr_t>(ba.K) |
-                           reinterpret_cast<uintptr_t>(ba.V)) & 15u) == 0;
-    if (aligned && batch * ba.nq < INT32_MAX && batch * ba.ld_tokens < INT32_MAX && tma_available()) {
-        const int st = launch_band_tc(ba.Q, ba.K, ba.V, batch, ba.nq, ba.q_pos0, ba.hq, ba.hkv, D, ba.ld_tokens,
-                                      ba.sink, ba.window, ba.part_o, ba.part_ml, ga.err, s);
-        if (st != LSA_OK) return st;
-    } else
-#endif
-    {
-        note_launch();
-        attn_band_kernel<D, G><<<dim3((unsigned)((ba.nq + QT - 1) / QT), units), kBandThreads, smem_band, s>>>(ba);
-    }
+    const int st = launch_band_tc(ba.Q, ba.K, ba.V, batch, ba.nq, ba.q_pos0, ba.hq, ba.hkv, D, ba.ld_tokens, ba.sink,
+                                  ba.window, ba.part_o, ba.part_ml, ga.err, s);
+    if (st != LSA_OK) return st;
     note_launch();
-    attn_gather_kernel<D, NT><<<dim3((unsigned)((ga.nq + kGatWarps - 1) / kGatWarps), units), kGatWarps * 32,
-                                 smem_gat, s>>>(ga);
+    attn_gather_kernel<D, NT><<<dim3((unsigned)((ga.nq + kGatWarps - 1) / kGatWarps), (unsigned)(batch * ba.hkv)),
+                                 kGatWarps * 32, smem_gat, s>>>(ga);
     return cuda_status(cudaGetLastError());
 }
 
@@ -614,6 +376,11 @@ int launch_banded_attn(const void* Q, const void* K, const void* V, const int32_
                        int64_t batch, int64_t nq, int64_t q_pos0, int hq, int hkv, int d, int max_sel,
                        int64_t ld_tokens, int sink, int window, void* O, float* lse, int32_t* err, cudaStream_t s) {
     if (nq <= 0 || batch <= 0) return LSA_OK;
+    // the band runs on TMA + tcgen05 (TMA coordinates are int32); otherwise
+    // the per-row kernels attend every row whole, with the same result
+    if (!tma_available() || batch * nq >= INT32_MAX || batch * ld_tokens >= INT32_MAX)
+        return launch_sparse_attn(Q, K, V, idx, cnt, batch, nq, hq, hkv, d, LSA_BF16, max_sel, ld_tokens, O, lse,
+                                  err, s);
     const int G = hq / hkv;
     const int64_t rows = batch * nq * hq;
     Arena scratch;

@@ -30,9 +30,6 @@ namespace {
 #ifndef LSA_SELECT_UNROLL
 #define LSA_SELECT_UNROLL 1
 #endif
-#ifndef LSA_SELECT_LEAF_SCAN
-#define LSA_SELECT_LEAF_SCAN 1
-#endif
 #ifndef LSA_SELECT_MIN_BLOCKS
 #define LSA_SELECT_MIN_BLOCKS 8
 #endif
@@ -547,7 +544,6 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
             const int cntl = a.leaf_cnt[c];
             const int32_t* bl = a.blk + st;
             int nlo = 0, nle = 0;
-#if LSA_SELECT_LEAF_SCAN
             for (int j0 = 0; j0 < cntl; j0 += 16) {
                 int v[16];
 #pragma unroll
@@ -558,15 +554,6 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
                     nle += v[j] <= b_hi;
                 }
             }
-#else
-            {
-                int hi = cntl;   // first index with bl >= b_lo
-                while (nlo < hi) { const int m = (nlo + hi) >> 1; if (bl[m] < b_lo) nlo = m + 1; else hi = m; }
-                nle = nlo;
-                hi = cntl;       // first index with bl > b_hi
-                while (nle < hi) { const int m = (nle + hi) >> 1; if (bl[m] <= b_hi) nle = m + 1; else hi = m; }
-            }
-#endif
             lo[e] = st + nlo;
             pre[e] = max(0, nle - nlo);
         }
