@@ -47,6 +47,10 @@ constexpr int kGatWarps = LSA_GAT_WARPS;    // queries per CTA (one warp each)
 constexpr int kGatSlice = 16;               // keys per slice
 constexpr int kGatStages = LSA_GAT_STAGES;  // slices in each warp's ring
 constexpr int kGatTQ = 1;                   // slices of token ids read ahead of their copies
+#ifndef LSA_GAT_ORDER_MIN
+#define LSA_GAT_ORDER_MIN 65536
+#endif
+constexpr int64_t kGatOrderMinPairs = LSA_GAT_ORDER_MIN;   // fewer row lists run in row order
 
 struct BandArgs {
     const __nv_bfloat16* Q;
@@ -73,6 +77,8 @@ struct GatherArgs {
     __nv_bfloat16* O;
     float* lse;
     int32_t* err;
+    const int32_t* order;   // optional: pair (row list) processed by warp w of the grid, else w itself
+    int64_t pairs;          // batch * nq * hkv
 };
 
 // NT = n8 tiles of heads (G <= 8 * NT; heads past G are zero and dropped)
@@ -89,11 +95,15 @@ __global__ __launch_bounds__(kGatWarps * 32) void attn_gather_kernel(const Gathe
     // per stage: bit k set when key k of the slice is a real token
     uint32_t* vmask = reinterpret_cast<uint32_t*>(smem + kGatWarps * 2 * kGatStages * SLICE_BYTES) + warp * kGatStages;
     const int G = a.hq / a.hkv;
-    const int u = blockIdx.y;
-    const int64_t b = u / a.hkv;
-    const int h = u % a.hkv;
-    const int64_t qi = (int64_t)blockIdx.x * kGatWarps + warp;
-    if (qi >= a.nq) return;   // warp-uniform; the kernel has no CTA barrier
+    const int64_t wg = (int64_t)blockIdx.x * kGatWarps + warp;
+    if (wg >= a.pairs) return;   // warp-uniform; the kernel has no CTA barrier
+    // row list (b, query, KV head) of this warp: pairs run in the given order
+    // (similar selections next to each other share rows in L2), else in row order
+    const int64_t pr = a.order ? (int64_t)a.order[wg] : wg;
+    const int h = (int)(pr % a.hkv);
+    const int64_t bq = pr / a.hkv;
+    const int64_t qi = bq % a.nq;
+    const int64_t b = bq / a.nq;
     const int64_t i = a.q_pos0 + qi;
     const int64_t row = (b * a.nq + qi) * a.hkv + h;
     int n = a.cnt[row];
@@ -342,6 +352,29 @@ __global__ __launch_bounds__(kGatWarps * 32) void attn_gather_kernel(const Gathe
     for (int e = lane; e < G * D / 8; e += 32) dst[e] = srcv[e];
 }
 
+// Sort key of a row list for the gather order: its first entry after the sink
+// (the smallest long-range token when the row is a selection).  Rows whose
+// long-range sets overlap mostly share that first entry, so sorting by it puts
+// queries that gather the same K/V rows next to each other.
+__global__ void gather_key_kernel(const int32_t* __restrict__ idx, const int32_t* __restrict__ cnt, int64_t nq,
+                                  int hkv, int max_sel, int64_t q_pos0, int sink, int64_t pairs, int64_t ld_tokens,
+                                  uint32_t* __restrict__ keys, int32_t* __restrict__ vals) {
+    const int64_t p = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (p >= pairs) return;
+    const int64_t i = q_pos0 + (p / hkv) % nq;
+    const int n = cnt[p];
+    const int ns = (int)min((int64_t)sink, i + 1);
+    uint32_t key = 0xFFFFFFFFu;
+    if (n > ns && n <= max_sel) {
+        // KV heads apart (their rows are different memory) when (head, token) fits in 32 bits
+        const int64_t t = idx[p * max_sel + ns];
+        const int64_t hk = (int64_t)(p % hkv) * ld_tokens + t;
+        key = (uint32_t)(hkv * ld_tokens < 0xFFFFFFFFll ? hk : t);
+    }
+    keys[p] = key;
+    vals[p] = (int32_t)p;
+}
+
 template <int D, int G>
 int launch_band_g(const BandArgs& ba, const GatherArgs& ga, int64_t batch, cudaStream_t s) {
     constexpr int NT = (G + 7) / 8;
@@ -353,8 +386,7 @@ int launch_band_g(const BandArgs& ba, const GatherArgs& ga, int64_t batch, cudaS
                                   ba.window, ba.part_o, ba.part_ml, ga.err, s);
     if (st != LSA_OK) return st;
     note_launch();
-    attn_gather_kernel<D, NT><<<dim3((unsigned)((ga.nq + kGatWarps - 1) / kGatWarps), (unsigned)(batch * ba.hkv)),
-                                 kGatWarps * 32, smem_gat, s>>>(ga);
+    attn_gather_kernel<D, NT><<<(unsigned)((ga.pairs + kGatWarps - 1) / kGatWarps), kGatWarps * 32, smem_gat, s>>>(ga);
     return cuda_status(cudaGetLastError());
 }
 
@@ -391,9 +423,26 @@ int launch_banded_attn(const void* Q, const void* K, const void* V, const int32_
     if (scratch.status != LSA_OK) return scratch.status;
     BandArgs ba{(const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, nq, q_pos0, ld_tokens,
                 hq, hkv, sink, window, 1.4426950408889634f / sqrtf((float)d), part_o, part_ml};
+    const int64_t pairs = batch * nq * hkv;
     GatherArgs ga{(const __nv_bfloat16*)Q, (const __nv_bfloat16*)K, (const __nv_bfloat16*)V, idx, cnt, nq, q_pos0,
                   ld_tokens, hq, hkv, max_sel, sink, window, ba.scale_log2, part_o, part_ml,
-                  (__nv_bfloat16*)O, lse, err};
+                  (__nv_bfloat16*)O, lse, err, nullptr, pairs};
+    if (pairs >= kGatOrderMinPairs) {
+        // gather order: row lists sorted by their first long-range token
+        uint32_t* k0 = scratch.alloc<uint32_t>(pairs);
+        uint32_t* k1 = scratch.alloc<uint32_t>(pairs);
+        int32_t* v0 = scratch.alloc<int32_t>(pairs);
+        int32_t* v1 = scratch.alloc<int32_t>(pairs);
+        int32_t* rs = scratch.alloc<int32_t>(radix_scratch_elems(pairs));
+        if (scratch.status != LSA_OK) return scratch.status;
+        note_launch();
+        gather_key_kernel<<<(unsigned)((pairs + 255) / 256), 256, 0, s>>>(idx, cnt, nq, hkv, max_sel, q_pos0, sink,
+                                                                         pairs, ld_tokens, k0, v0);
+        uint32_t* ko;
+        int32_t* vo;
+        radix_sort(k0, v0, k1, v1, pairs, 32, rs, s, &ko, &vo);
+        ga.order = vo;
+    }
     int st = LSA_ERR_INVALID_ARG;
     if (d == 128) st = launch_band_d<128>(G, ba, ga, batch, s);
     else if (d == 64) st = launch_band_d<64>(G, ba, ga, batch, s);
