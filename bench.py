@@ -431,20 +431,24 @@ def run_extra(w, inp, bp, sp, dev, select_ms, idx, cnt):
     full_ms_est = full_ms_sample * N / pos.numel()
     tidx = idx[:, pos]
     tcnt = cnt[:, pos]
-    # recall of the tree's long-range picks against the exact full-scan top-K
-    hit = tot = 0
-    for b in range(w.batch):
-        for h in range(w.hkv):
-            for k in range(pos.numel()):
-                f = set(fidx[b, k, h, : fcnt[b, k, h]].tolist())
-                t = set(tidx[b, k, h, : tcnt[b, k, h]].tolist())
-                i = int(pos[k])
-                lo = max(0, i - w.window + 1)
-                base = set(range(min(w.sink, lo))) | set(range(lo, i + 1))
-                f -= base
-                t -= base
-                tot += len(f)
-                hit += len(f & t)
+
+    def recall(sidx, scnt):
+        """share of the exact full-scan long-range picks that a selection also made"""
+        fi, fc, si, sc_ = fidx.cpu(), fcnt.cpu(), sidx.cpu(), scnt.cpu()
+        hit = tot = 0
+        for b in range(w.batch):
+            for h in range(w.hkv):
+                for k in range(pos.numel()):
+                    i = int(pos[k])
+                    lo = max(0, i - w.window + 1)
+                    base = set(range(min(w.sink, lo))) | set(range(lo, i + 1))
+                    f = set(fi[b, k, h, : fc[b, k, h]].tolist()) - base
+                    t = set(si[b, k, h, : sc_[b, k, h]].tolist()) - base
+                    tot += len(f)
+                    hit += len(f & t)
+        return hit / max(1, tot)
+
+    tree_recall = recall(tidx, tcnt)
     needles = inp["needles"]
     nh_tree = nh_full = 0
     for (b, h, p, qp) in needles:
@@ -458,9 +462,40 @@ def run_extra(w, inp, bp, sp, dev, select_ms, idx, cnt):
         for k, (b, h, p, qp) in enumerate(needles):
             nh_full += int((nf[b, k, h, : nfc[b, k, h]] == p).any().item())
     ix.free()
+    # flat-vs-tree study: one level of the same leaf count, same beam, K, S, W
+    flat = None
+    if len(w.level_sizes) > 1:
+        bpf = lsa.make_build_params(w.batch, N, N, w.hkv, w.d, w.r, w.pool,
+                                    lsa.LSA_BF16 if w.dtype == "bf16" else lsa.LSA_F32, (w.level_sizes[-1],),
+                                    w.lloyd_iters, w.grid_log2, w.sink, 0)
+        e0.record()
+        ixf = lsa.lsa_build_index(bpf, K, inp["W"])
+        e1.record()
+        torch.cuda.synchronize()
+        flat_build_ms = e0.elapsed_time(e1)
+        nfq = min(N, 131072)
+        qf = Q[:, N - nfq:].contiguous()
+        lsa.lsa_select(ixf, sp, qf, q_pos0=N - nfq)
+        torch.cuda.synchronize()
+        e0.record()
+        lsa.lsa_select(ixf, sp, qf, q_pos0=N - nfq)
+        e1.record()
+        torch.cuda.synchronize()
+        flat_ms_est = e0.elapsed_time(e1) * N / nfq
+        fsi, fsc = lsa.lsa_select(ixf, sp, qs, q_pos=qpos)
+        nh_flat = 0
+        if needles:
+            ff, ffc = lsa.lsa_select(ixf, sp, nq_, q_pos=nqpos)
+            for k, (b, h, p, qp) in enumerate(needles):
+                nh_flat += int((ff[b, k, h, : ffc[b, k, h]] == p).any().item())
+        flat = {"leaves": w.level_sizes[-1], "build_ms": flat_build_ms,
+                "select_ms_estimate": flat_ms_est, "select_sample_queries": nfq,
+                "recall_vs_fullscan_topk": recall(fsi, fsc),
+                "needle_hit_rate": nh_flat / max(1, len(needles))}
+        ixf.free()
     return {"fullscan_ms_estimate": full_ms_est, "fullscan_sample_queries": int(pos.numel()),
             "tree_select_ms": select_ms, "tree_vs_fullscan_speedup": full_ms_est / select_ms,
-            "tree_recall_vs_fullscan_topk": hit / max(1, tot),
+            "tree_recall_vs_fullscan_topk": tree_recall, "flat_vs_tree": flat,
             "needle_hit_rate_tree": nh_tree / max(1, len(needles)),
             "needle_hit_rate_fullscan": nh_full / max(1, len(needles)), "needles": len(needles),
             "index_device_bytes": int(info.device_bytes),
