@@ -59,6 +59,12 @@ Readings where the pages are silent (each one is also listed in the design doc):
   R12 softmax scale 1/sqrt(d).
   R13 decode: centroids are frozen; a completed block goes to its nearest leaf
       over all leaves.
+  R17 the training-free map [p5 "How does LSA work?", the D-LSA options: "a
+      training-free option that uses a PCA map"]: W = the r leading principal
+      directions of the pooled keys of every (sequence, KV head), i.e. the
+      eigenvectors of their covariance (centred, divided by the count) for the
+      r largest eigenvalues, in descending order; each column's entry of
+      largest magnitude (lowest index among equal magnitudes) is positive.
 
 Parity pins live in tests/test_oracle_pins.py (closed forms, hand-worked
 examples under tests/golden/, invariants, brute force on tiny inputs).  Parity
@@ -88,6 +94,26 @@ def project_pool(K: np.ndarray, W: np.ndarray, pool: int) -> np.ndarray:
     nb = K.shape[0] // pool
     pooled = K[: nb * pool].reshape(nb, pool, K.shape[1]).mean(axis=1)
     return pooled @ W
+
+
+def pca_map(K_units, pool: int, r: int):
+    """Training-free latent map (reading R17).  K_units: sequence of [N, d]
+    key arrays, one per (sequence, KV head); every one is pooled as in
+    ``project_pool`` (the map here is the identity) and all pooled keys are
+    one sample.  Returns (W [d, r], the r largest covariance eigenvalues in
+    descending order)."""
+    X = np.concatenate([project_pool(Ku, np.eye(np.asarray(Ku).shape[1]), pool) for Ku in K_units], axis=0)
+    mu = X.mean(axis=0)
+    Xc = X - mu
+    C = Xc.T @ Xc / X.shape[0]
+    evals, evecs = np.linalg.eigh(C)              # ascending
+    order = np.argsort(-evals, kind="stable")[:r]
+    W = evecs[:, order].copy()
+    for c in range(r):
+        j = int(np.argmax(np.abs(W[:, c])))       # first index of the largest magnitude
+        if W[j, c] < 0:
+            W[:, c] = -W[:, c]
+    return W, evals[order]
 
 
 def query_latent(Qg: np.ndarray, W: np.ndarray) -> np.ndarray:

@@ -343,3 +343,65 @@ def test_integer_workload_stays_exact():
     assert np.all(qb * 4 == np.round(qb * 4))
     s = t.centroids[1] @ qb.T
     assert np.all(s * 64 == np.round(s * 64)) and np.abs(s).max() < 2 ** 20
+
+
+# ---------------------------------------------------------------- PCA map (R17)
+def test_pca_map_axes_closed_form():
+    """Pooled keys +-a_k e_k (k = 0, 1, 2) plus two zero rows: mean 0, covariance
+    diag(2 a_k^2 / n), so the map is the axes in order of a_k and the
+    eigenvalues are those variances."""
+    d, a = 6, [3.0, 1.0, 2.0]
+    rows = [np.zeros(d), np.zeros(d)]
+    for k, ak in enumerate(a):
+        e = np.zeros(d)
+        e[k] = ak
+        rows += [e, -e]
+    K = np.array(rows)
+    n = K.shape[0]
+    W, ev = O.pca_map([K], pool=1, r=3)
+    assert np.allclose(ev, [2 * 9 / n, 2 * 4 / n, 2 * 1 / n])
+    assert np.allclose(W[:, 0], np.eye(d)[0]) and np.allclose(W[:, 1], np.eye(d)[2])
+    assert np.allclose(W[:, 2], np.eye(d)[1])
+
+
+def test_pca_map_pools_before_the_covariance():
+    """Keys alternate +v, -v inside every block of 2: pooling cancels v, so
+    with pool 2 the map ignores v; with pool 1 v is the leading direction."""
+    rng = np.random.default_rng(3)
+    d, n = 5, 400
+    v = np.zeros(d)
+    v[4] = 10.0
+    base = rng.normal(size=(n // 2, d)) * np.array([1.0, 0.5, 0.25, 0.1, 0.0])
+    K = np.repeat(base, 2, axis=0)
+    K[0::2] += v
+    K[1::2] -= v
+    W1, _ = O.pca_map([K], pool=1, r=1)
+    W2, _ = O.pca_map([K], pool=2, r=2)
+    assert abs(W1[4, 0]) > 0.99
+    assert np.all(np.abs(W2[4, :]) < 1e-9)
+
+
+def test_pca_map_invariants_and_sign():
+    rng = np.random.default_rng(4)
+    Ks = [rng.normal(size=(64, 8)) @ rng.normal(size=(8, 8)) for _ in range(3)]
+    W, ev = O.pca_map(Ks, pool=4, r=5)
+    assert np.allclose(W.T @ W, np.eye(5), atol=1e-12)
+    assert np.all(np.diff(ev) <= 0)
+    for c in range(5):
+        j = int(np.argmax(np.abs(W[:, c])))
+        assert W[j, c] > 0
+    # the same sample in another order (units swapped) gives the same map
+    W2, ev2 = O.pca_map(Ks[::-1], pool=4, r=5)
+    assert np.allclose(W, W2) and np.allclose(ev, ev2)
+
+
+def test_pca_map_is_centred():
+    """Adding one large constant vector to every key moves the mean only: the
+    centred covariance, and so the map, do not change (an uncentred second
+    moment would put the constant direction first)."""
+    rng = np.random.default_rng(5)
+    K = rng.normal(size=(256, 6)) * np.array([3.0, 2.0, 1.5, 1.0, 0.5, 0.25])
+    W0, ev0 = O.pca_map([K], pool=1, r=3)
+    shift = np.array([0.0, 0.0, 0.0, 0.0, 0.0, 50.0])
+    W1, ev1 = O.pca_map([K + shift], pool=1, r=3)
+    assert np.allclose(W0, W1, atol=1e-9) and np.allclose(ev0, ev1)
