@@ -493,7 +493,30 @@ def run_extra(w, inp, bp, sp, dev, select_ms, idx, cnt):
                 "recall_vs_fullscan_topk": recall(fsi, fsc),
                 "needle_hit_rate": nh_flat / max(1, len(needles))}
         ixf.free()
+    # training-free PCA map (row f1): its time, and the tree's recall and needle
+    # hits when the map replaces the seeded W (full scan in the same latent space)
+    pca = None
+    if w.d in (64, 128):
+        e0.record()
+        Wp, evp = lsa.lsa_pca_map(K, N, w.pool, w.r)
+        e1.record()
+        torch.cuda.synchronize()
+        pca_ms = e0.elapsed_time(e1)
+        ixp = lsa.lsa_build_index(bp, K, Wp)
+        psi, psc = lsa.lsa_select(ixp, sp, qs, q_pos=qpos)
+        pfi, pfc = lsa.lsa_fullscan_select(ixp, sp, qs, q_pos=qpos)
+        nh_pca = 0
+        if needles:
+            pn, pnc = lsa.lsa_select(ixp, sp, nq_, q_pos=nqpos)
+            for k, (b, h, p, qp) in enumerate(needles):
+                nh_pca += int((pn[b, k, h, : pnc[b, k, h]] == p).any().item())
+        fidx, fcnt = pfi, pfc          # recall() compares against this full scan
+        pca = {"map_ms": pca_ms, "explained_top_r": float(evp.sum().item()),
+               "tree_recall_vs_fullscan_topk": recall(psi, psc),
+               "needle_hit_rate_tree": nh_pca / max(1, len(needles))}
+        ixp.free()
     return {"fullscan_ms_estimate": full_ms_est, "fullscan_sample_queries": int(pos.numel()),
+            "pca_map": pca,
             "tree_select_ms": select_ms, "tree_vs_fullscan_speedup": full_ms_est / select_ms,
             "tree_recall_vs_fullscan_topk": tree_recall, "flat_vs_tree": flat,
             "needle_hit_rate_tree": nh_tree / max(1, len(needles)),

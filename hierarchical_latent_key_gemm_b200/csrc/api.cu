@@ -475,6 +475,17 @@ int lsa_query_latent(const void* Q, const float* W, int64_t batch, int64_t nq, i
     return launch_query_latent(Q, W, batch, nq, hq, hkv, d, r, dtype, qbar, as_stream(stream));
 }
 
+int lsa_pca_map(const void* K, int64_t batch, int64_t n_tokens, int64_t ld_tokens, int32_t hkv, int32_t d,
+                int32_t pool, int32_t dtype, int32_t r, float* W, double* eigvals, void* stream) {
+    if (batch < 1 || n_tokens < 0 || ld_tokens < n_tokens || hkv < 1 || (d != 64 && d != 128) || pool < 1 ||
+        (dtype != LSA_F32 && dtype != LSA_BF16) || r < 1 || r > d || batch * hkv > 65535)
+        return LSA_ERR_INVALID_ARG;
+    if (n_tokens / pool < 1 || batch * hkv * (n_tokens / pool) > ((int64_t)1 << 40)) return LSA_ERR_INVALID_ARG;
+    if (!is_device_ptr(K) || !is_device_ptr(W)) return LSA_ERR_INVALID_ARG;
+    if (eigvals && !is_device_ptr(eigvals)) return LSA_ERR_INVALID_ARG;
+    return launch_pca_map(K, batch, n_tokens, ld_tokens, hkv, d, pool, dtype, r, W, eigvals, as_stream(stream));
+}
+
 int lsa_kmeans(const float* X, int64_t units, int64_t n, int32_t r, int32_t k, int32_t iters, int32_t grid_log2,
                int32_t* labels, float* C, double* objective, void* stream) {
     if (units < 1 || units > 65535 || n < 1 || !valid_r(r) || k < 1 || iters < 1 || grid_log2 < 0 || grid_log2 > 8)

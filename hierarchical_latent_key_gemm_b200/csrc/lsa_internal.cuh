@@ -174,6 +174,9 @@ int launch_sparse_attn(const void* Q, const void* K, const void* V, const int32_
 int launch_banded_attn(const void* Q, const void* K, const void* V, const int32_t* idx, const int32_t* cnt,
                        int64_t batch, int64_t nq, int64_t q_pos0, int hq, int hkv, int d, int max_sel,
                        int64_t ld_tokens, int sink, int window, void* O, float* lse, int32_t* err, cudaStream_t s);
+// training-free latent map (pca.cu)
+int launch_pca_map(const void* K, int64_t batch, int64_t n_tokens, int64_t ld_tokens, int hkv, int d, int pool,
+                   int dtype, int r, float* W, double* evals, cudaStream_t s);
 // tensor-core band of the banded attention (attn_band_tc.cu): partials as the mma.sync band kernel writes them
 int launch_band_tc(const void* Q, const void* K, const void* V, int64_t batch, int64_t nq, int64_t q_pos0, int hq,
                    int hkv, int d, int64_t ld_tokens, int sink, int window, float* part_o, float2* part_ml,

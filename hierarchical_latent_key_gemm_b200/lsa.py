@@ -64,6 +64,7 @@ _SIGS = {
     "lsa_sparse_attn_banded": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _i32, _i32,
                                       _i64, _i32, _i32, _vp, _vp, _vp]),
     "lsa_append": (_i32, [_vp, _vp, _i64, _vp]),
+    "lsa_pca_map": (_i32, [_vp, _i64, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "lsa_project_pool": (_i32, [_vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
     "lsa_query_latent": (_i32, [_vp, _vp, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
     "lsa_kmeans": (_i32, [_vp, _i64, _i64, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp]),
@@ -301,6 +302,19 @@ def lsa_sparse_attn_banded(Q, K, V, idx, cnt, hkv, sink, window, q_pos0=0, O=Non
 
 def lsa_append(index: Index, K: torch.Tensor, n_new: int, stream=None):
     _ok(lib().lsa_append(index.handle, _ptr(K), int(n_new), _stream(stream)), "lsa_append")
+
+
+def lsa_pca_map(K, n_tokens, pool, r, W=None, eigvals=None, stream=None):
+    """Training-free latent map of the pooled keys: returns (W [d, r] float32,
+    eigenvalues [r] float64), both on K's device."""
+    B, ld, hkv, d = K.shape
+    if W is None:
+        W = torch.empty((d, r), dtype=torch.float32, device=K.device)
+    if eigvals is None:
+        eigvals = torch.empty(r, dtype=torch.float64, device=K.device)
+    _ok(lib().lsa_pca_map(_ptr(K), int(B), int(n_tokens), int(ld), int(hkv), int(d), int(pool), dtype_code(K),
+                          int(r), _ptr(W), _ptr(eigvals), _stream(stream)), "lsa_pca_map")
+    return W, eigvals
 
 
 def lsa_project_pool(K, W, n_tokens, pool, Kl=None, stream=None):

@@ -201,6 +201,26 @@ int lsa_select_work(const lsa_index* index, const lsa_select_params* params, con
                     int32_t* idx, int32_t* cnt, int32_t max_sel, unsigned long long* scored,
                     void* stream);
 
+/* Training-free latent map: W = the r leading principal directions of the
+ * pooled keys ([p5] "How does LSA work?", the D-LSA options: a training-free
+ * option that uses a PCA map).  Every (sequence, KV head)'s keys are pooled as
+ * in the build (mean of `pool` consecutive keys, complete blocks only) and all
+ * pooled keys form one sample; their covariance (centred, divided by the
+ * count, accumulated in fp64) is diagonalised on the device (parallel cyclic
+ * Jacobi).
+ *  K: device [batch][ld_tokens][hkv][d] (bf16 or f32), tokens [0, n_tokens).
+ *  W: device float [d][r] out: eigenvectors of the r largest eigenvalues in
+ *     descending order, each signed so that its entry of largest magnitude
+ *     (lowest index among equal magnitudes) is positive; usable directly as
+ *     the W of lsa_build_index / lsa_select.
+ *  eigvals: device double [r] out (the r largest eigenvalues), or NULL.
+ *  d in {64, 128}; 1 <= r <= d; at least one complete block.
+ *  Errors: LSA_ERR_INVALID_ARG before anything is enqueued; LSA_ERR_OOM for
+ *  its stream-ordered scratch (2 d^2 + d doubles). */
+int lsa_pca_map(const void* K, int64_t batch, int64_t n_tokens, int64_t ld_tokens, int32_t hkv,
+                int32_t d, int32_t pool, int32_t dtype, int32_t r, float* W, double* eigvals,
+                void* stream);
+
 /* The quadratic baseline indexer: every candidate block is scored, no tree.
  * Same arguments and output format as lsa_select (beam is ignored).
  * [p3 flowchart, red path "Full key scan"] */
