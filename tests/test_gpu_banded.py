@@ -271,3 +271,41 @@ def test_host_prefill_pipeline_matches_device_path():
     got = hO.float()
     assert bool(((got - ref).abs() <= ref.abs() * 2.0 ** -6 + 1e-3).all())
     ix.free()
+
+
+def test_select_and_banded_attention_capture_in_a_cuda_graph():
+    """Selection runs on the device and every call is stream-ordered (scratch
+    from the stream-ordered pool), so select + banded attention of a prefill
+    can be captured in a CUDA graph; a replay writes the eager outputs bit for
+    bit."""
+    w = WORKLOADS["gqa_128k"].scaled(n_tokens=20000 + 5, level_sizes=(8, 64), needles=0, components=256)
+    inp = make_inputs(w, seed=30, device="cuda")
+    bp, sp = TU.build_params(w), TU.select_params(w)
+    ix = lsa.lsa_build_index(bp, inp["K"], inp["W"])
+    idx = torch.empty((1, w.n_tokens, w.hkv, w.max_sel), dtype=torch.int32, device="cuda")
+    cnt = torch.empty((1, w.n_tokens, w.hkv), dtype=torch.int32, device="cuda")
+    O_ = torch.empty_like(inp["Q"])
+    lse = torch.empty((1, w.n_tokens, w.hq), dtype=torch.float32, device="cuda")
+
+    def run():
+        lsa.lsa_select(ix, sp, inp["Q"], idx=idx, cnt=cnt)
+        lsa.lsa_sparse_attn_banded(inp["Q"], inp["K"], inp["V"], idx, cnt, w.hkv, w.sink, w.window, O=O_, lse=lse)
+
+    run()
+    torch.cuda.synchronize()
+    ref_o, ref_i, ref_c = O_.clone(), idx.clone(), cnt.clone()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        run()
+    O_.zero_()
+    idx.zero_()
+    cnt.zero_()
+    torch.cuda.synchronize()
+    g.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(O_, ref_o) and torch.equal(idx, ref_i) and torch.equal(cnt, ref_c)
+    assert lsa.lsa_check(ix) == lsa.LSA_OK
+    del g
+    ix.free()
