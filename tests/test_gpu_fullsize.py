@@ -47,8 +47,8 @@ def _sample_rows(w, inp, rng, count):
 
 
 def _check_selection_and_attention(w, inp, trees, Kls, sample, seed):
-    """Import the oracle's trees, run select + attention over every query (the
-    bench's grids), compare sampled rows with the oracle."""
+    """Import the oracle's trees, run select + banded attention over every query
+    (the bench's launches), compare sampled rows with the oracle."""
     d = {k: (v.cuda() if torch.is_tensor(v) else v) for k, v in inp.items()}
     leaf, par, cen = TU.trees_to_device(trees, w)
     ix = lsa.lsa_build_index_from_tree(TU.build_params(w), d["K"], d["W"], leaf, par, cen)
@@ -72,7 +72,9 @@ def _check_selection_and_attention(w, inp, trees, Kls, sample, seed):
         ii, cc = TU.rows_to_idx(want, w.max_sel)
         idx[0, torch.as_tensor(rows, device="cuda"), h] = ii
         cnt[0, torch.as_tensor(rows, device="cuda"), h] = cc
-    O_, lse = lsa.lsa_sparse_attn(d["Q"], d["K"], d["V"], idx, cnt, w.hkv)
+    # the bench's attention path: banded (dense sink/window tiles + ordered
+    # long-range gather) over every query
+    O_, lse = lsa.lsa_sparse_attn_banded(d["Q"], d["K"], d["V"], idx, cnt, w.hkv, w.sink, w.window)
     assert lsa.lsa_check(None) == lsa.LSA_OK
     errs = []
     G = w.group
