@@ -1,11 +1,14 @@
-"""A whole prefill layer from host memory, with the copies overlapped.
+"""Orchestration of the library calls on streams and graphs (no arithmetic).
 
-Only binding calls and torch copies on three CUDA streams: K, V and W go up
-first and the index is built while the queries go up chunk by chunk; each
-chunk of consecutive queries is selected and attended (banded attention) as
-soon as its queries have arrived, and its output goes back to the host while
-the next chunk computes.  Every step moves all of Q, K, V and W up and all of
-O down; the overlap only hides the transfers behind the kernels.
+HostPrefill: a whole prefill layer from host memory, with the copies
+overlapped.  Binding calls and torch copies on three CUDA streams: K, V and W
+go up first and the index is built while the queries go up chunk by chunk;
+each chunk of consecutive queries is selected and attended (banded attention)
+as soon as its queries have arrived, and its output goes back to the host
+while the next chunk computes.  Every step moves all of Q, K, V and W up and
+all of O down; the overlap only hides the transfers behind the kernels.
+
+DecodeStep: decode with select + attention replayed from one CUDA graph.
 """
 from __future__ import annotations
 
@@ -16,8 +19,8 @@ from . import lsa
 
 class HostPrefill:
     """Device buffers and streams for repeated host-to-host prefill layers of
-    one shape (batch 1).  `run` enqueues one layer; `end_event` marks its end
-    on the current stream."""
+    one shape (batch 1).  `run` enqueues one layer and makes the current
+    stream wait for it; it returns the layer's index (free it when done)."""
 
     def __init__(self, bp, sp, hQ, hK, hV, hW, hO, sink: int, window: int, chunks: int = 8, device=None):
         if hQ.shape[0] != 1:
@@ -100,3 +103,49 @@ class HostPrefill:
             e.record(s)
             cur.wait_event(e)
         return ix
+
+
+class DecodeStep:
+    """Decode steps with little host work: the append runs as a plain call
+    (whether it launches depends on the token completing a block), and select +
+    attention for the new queries replay one CUDA graph captured at set-up.
+    The graph reads the queries and their positions from fixed device buffers,
+    and the index's device arrays carry every appended block, so one capture
+    serves all later steps (tree selection reads no host-side block count)."""
+
+    def __init__(self, index, sp, K, V, hq: int, max_sel: int, device=None):
+        p = index.params
+        self.dev = device or K.device
+        self.index, self.sp, self.K, self.V = index, sp, K, V
+        self.hkv, self.max_sel = p.hkv, max_sel
+        B, d = p.batch, p.d
+        self.q = torch.zeros((B, 1, hq, d), dtype=K.dtype, device=self.dev)
+        self.pos = torch.full((B, 1), max(0, p.n_tokens - 1), dtype=torch.int64, device=self.dev)
+        self.idx = torch.empty((B, 1, p.hkv, max_sel), dtype=torch.int32, device=self.dev)
+        self.cnt = torch.empty((B, 1, p.hkv), dtype=torch.int32, device=self.dev)
+        self.O = torch.empty((B, 1, hq, d), dtype=K.dtype, device=self.dev)
+        self.lse = torch.empty((B, 1, hq), dtype=torch.float32, device=self.dev)
+        side = torch.cuda.Stream(self.dev)
+        side.wait_stream(torch.cuda.current_stream(self.dev))
+        with torch.cuda.stream(side):
+            self._select_attend()          # eager once: kernel attributes, scratch pool
+        torch.cuda.current_stream(self.dev).wait_stream(side)
+        torch.cuda.synchronize(self.dev)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph, stream=side):
+            self._select_attend()
+
+    def _select_attend(self):
+        lsa.lsa_select(self.index, self.sp, self.q, q_pos=self.pos, idx=self.idx, cnt=self.cnt,
+                       max_sel=self.max_sel)
+        lsa.lsa_sparse_attn(self.q, self.K, self.V, self.idx, self.cnt, self.hkv, O=self.O, lse=self.lse)
+
+    def step(self, q_new, pos: int):
+        """Index the token at `pos` (already written into K), then select and
+        attend for q_new [batch, 1, hq, d] at that position; returns (O, lse)
+        buffers that the next step overwrites."""
+        lsa.lsa_append(self.index, self.K, 1)
+        self.q.copy_(q_new)
+        self.pos.fill_(pos)
+        self.graph.replay()
+        return self.O, self.lse

@@ -309,3 +309,31 @@ def test_select_and_banded_attention_capture_in_a_cuda_graph():
     assert lsa.lsa_check(ix) == lsa.LSA_OK
     del g
     ix.free()
+
+
+def test_decode_graph_steps_match_plain_calls():
+    """Decode with the captured select + attention graph gives, step by step,
+    the rows and outputs of the plain calls (appends cross several blocks)."""
+    from hierarchical_latent_key_gemm_b200.pipeline import DecodeStep
+    w = WORKLOADS["decode_10m_x4"].scaled(n_tokens=8192 + 2, batch=2, level_sizes=(4, 16, 64), needles=0,
+                                          components=256, decode_steps=24)
+    inp = make_inputs(w, seed=31, device="cuda")
+    bp = TU.build_params(w, append_capacity=w.decode_steps)
+    sp = TU.select_params(w)
+    ix_a = lsa.lsa_build_index(bp, inp["K"], inp["W"])
+    ix_b = lsa.lsa_build_index(bp, inp["K"], inp["W"])
+    ds = DecodeStep(ix_b, sp, inp["K"], inp["V"], w.hq, w.max_sel)
+    for s in range(w.decode_steps):
+        t = w.n_tokens + s
+        q = inp["Q"][:, s:s + 1].contiguous()
+        lsa.lsa_append(ix_a, inp["K"], 1)
+        ia, ca = lsa.lsa_select(ix_a, sp, q, q_pos0=t, max_sel=w.max_sel)
+        oa, la = lsa.lsa_sparse_attn(q, inp["K"], inp["V"], ia, ca, w.hkv)
+        ob, lb = ds.step(q, t)
+        torch.cuda.synchronize()
+        assert torch.equal(ia, ds.idx) and torch.equal(ca, ds.cnt), f"step {s}"
+        assert torch.equal(oa, ob) and torch.equal(la, lb), f"step {s}"
+    assert lsa.lsa_check(ix_a) == lsa.LSA_OK and lsa.lsa_check(ix_b) == lsa.LSA_OK
+    del ds
+    ix_a.free()
+    ix_b.free()
