@@ -454,6 +454,26 @@ int lsa_append(lsa_index* index, const void* K, int64_t n_new, void* stream) {
     return LSA_OK;
 }
 
+int lsa_relayout(lsa_index* index, void* stream) {
+    if (!live(index)) return LSA_ERR_INVALID_ARG;
+    Arena scratch;
+    scratch.async = true;
+    scratch.stream = as_stream(stream);
+    int st = relayout_leaves(index, as_stream(stream), scratch);
+    scratch.release();
+    return st != LSA_OK ? st : cuda_status(cudaGetLastError());
+}
+
+int lsa_refresh_centroids(lsa_index* index, void* stream) {
+    if (!live(index)) return LSA_ERR_INVALID_ARG;
+    Arena scratch;
+    scratch.async = true;
+    scratch.stream = as_stream(stream);
+    int st = refresh_centroids(index, as_stream(stream), scratch);
+    scratch.release();
+    return st != LSA_OK ? st : cuda_status(cudaGetLastError());
+}
+
 int lsa_project_pool(const void* K, const float* W, int64_t batch, int64_t n_tokens, int64_t ld_tokens, int32_t hkv,
                      int32_t d, int32_t r, int32_t pool, int32_t dtype, float* Kl, void* stream) {
     if (batch < 1 || n_tokens < 0 || ld_tokens < n_tokens || hkv < 1 || !valid_d(d) || !valid_r(r) || pool < 1 ||

@@ -6,8 +6,9 @@
 // the build (same arithmetic order, so identical bits), placed in its nearest
 // leaf by squared distance over all leaves (frozen centroids, ties to the
 // lower id) at the end of that leaf's ascending member run, and the minpos of
-// the leaf and its ancestors is lowered.  A full leaf latches kErrCapacity
-// and leaves the block unindexed.
+// the leaf and its ancestors is lowered.  A full leaf latches kErrCapacity;
+// the block keeps its leaf label but stays out of the buckets (and out of
+// minpos) until the leaves are laid out again (relayout_leaves).
 //
 // Three launches: latents of the new blocks; the nearest-leaf scan spread over
 // many CTAs (each takes a chunk of leaves, one warp per leaf row, and folds its
@@ -142,8 +143,9 @@ __global__ __launch_bounds__(kAppThreads) void append_insert_kernel(const AppArg
                         }
                     }
                 } else {
+                    // no free slot: the block keeps its label and waits for a relayout
                     latch(a.err, kErrCapacity);
-                    a.leaf_of_block[(int64_t)u * a.nb_cap + b] = -1;
+                    a.leaf_of_block[(int64_t)u * a.nb_cap + b] = leaf;
                 }
             }
             slot_sh = slot;

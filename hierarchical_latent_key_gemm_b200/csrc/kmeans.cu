@@ -376,6 +376,40 @@ int group_by_label(const int32_t* labels, int64_t ldl, int64_t units, int64_t n,
     return cuda_status(cudaGetLastError());
 }
 
+// Decode maintenance (lsa_refresh_centroids): every centroid becomes the
+// mean of its current members, memberships fixed, bottom-up (leaves from the
+// latent keys of their blocks, each upper level from the refreshed level
+// below), by the update of the Lloyd rounds (fp64 sums in ascending member
+// order, empty keeps, grid rounding); then the tree-order copies.
+int refresh_centroids(lsa_index* ix, cudaStream_t s, Arena& A) {
+    const lsa_build_params& p = ix->p;
+    const int levels = p.levels, r = p.r;
+    const int64_t U = ix->units;
+    for (int l = levels - 1; l >= 0; --l) {
+        const int k = p.level_sizes[l];
+        const bool leaf = l == levels - 1;
+        const int64_t n = leaf ? ix->nb : p.level_sizes[l + 1];
+        const float* X = leaf ? ix->Kl : ix->cent[l + 1];
+        const int64_t ldx = leaf ? ix->nb_cap : n;
+        const int32_t* labels = leaf ? ix->leaf_of_block : ix->parent[l + 1];
+        const int64_t nc = U * (int64_t)k;
+        int32_t* perm = A.alloc<int32_t>(U * n);
+        int32_t* off = A.alloc<int32_t>(nc + 1);
+        float* Cn = A.alloc<float>(nc * r);
+        double* cobj = A.alloc<double>(nc);
+        GroupWork gw = alloc_group_work(U, n, k, A);
+        if (A.status != LSA_OK) return A.status;
+        int st = group_by_label(labels, ldx, U, n, k, perm, off, ix->err, s, gw);
+        if (st != LSA_OK) return st;
+        note_launch();
+        update_kernel<<<(unsigned)((nc * 32 + 255) / 256), 256, 0, s>>>(X, ldx, n, r, k, perm, off, ix->cent[l], Cn,
+                                                                       p.grid_log2, cobj, nc, ix->err);
+        cudaMemcpyAsync(ix->cent[l], Cn, nc * r * sizeof(float), cudaMemcpyDeviceToDevice, s);
+    }
+    gather_tree_order(ix, s);
+    return cuda_status(cudaGetLastError());
+}
+
 int run_kmeans(const float* X, int64_t ldx, int64_t units, int64_t n, int r, int k, int iters, int grid_log2,
                KmeansOut out, int64_t ldl, int32_t* err, cudaStream_t s, Arena& A) {
     if (units <= 0 || n <= 0 || k <= 0) return LSA_OK;

@@ -193,4 +193,11 @@ int finish_tree(lsa_index* ix, const int32_t* leaf_perm, const int32_t* leaf_off
                 const int32_t* const* up_perm, const int32_t* const* up_off, cudaStream_t s,
                 Arena& scratch);
 
+// Decode maintenance: lay the leaves out again from the block labels
+// (tree.cu), recompute every centroid from its members (kmeans.cu), and the
+// tree-order copies of centroids and minpos that the selection reads.
+int relayout_leaves(lsa_index* ix, cudaStream_t s, Arena& scratch);
+int refresh_centroids(lsa_index* ix, cudaStream_t s, Arena& scratch);
+void gather_tree_order(lsa_index* ix, cudaStream_t s);
+
 }  // namespace lsa

@@ -64,6 +64,8 @@ _SIGS = {
     "lsa_sparse_attn_banded": (_i32, [_vp, _vp, _vp, _vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _i32, _i32,
                                       _i64, _i32, _i32, _vp, _vp, _vp]),
     "lsa_append": (_i32, [_vp, _vp, _i64, _vp]),
+    "lsa_relayout": (_i32, [_vp, _vp]),
+    "lsa_refresh_centroids": (_i32, [_vp, _vp]),
     "lsa_pca_map": (_i32, [_vp, _i64, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "lsa_project_pool": (_i32, [_vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
     "lsa_query_latent": (_i32, [_vp, _vp, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
@@ -302,6 +304,14 @@ def lsa_sparse_attn_banded(Q, K, V, idx, cnt, hkv, sink, window, q_pos0=0, O=Non
 
 def lsa_append(index: Index, K: torch.Tensor, n_new: int, stream=None):
     _ok(lib().lsa_append(index.handle, _ptr(K), int(n_new), _stream(stream)), "lsa_append")
+
+
+def lsa_relayout(index: Index, stream=None):
+    _ok(lib().lsa_relayout(index.handle, _stream(stream)), "lsa_relayout")
+
+
+def lsa_refresh_centroids(index: Index, stream=None):
+    _ok(lib().lsa_refresh_centroids(index.handle, _stream(stream)), "lsa_refresh_centroids")
 
 
 def lsa_pca_map(K, n_tokens, pool, r, W=None, eigvals=None, stream=None):

@@ -273,10 +273,42 @@ int lsa_sparse_attn_banded(const void* Q, const void* K, const void* V, const in
  * block this completes is pooled, mapped, and placed in its nearest leaf
  * (squared distance over all leaves, frozen centroids, ties to the lower id)
  * after that leaf's older blocks; node eligibility is updated.  A leaf with
- * no free slot latches LSA_ERR_CAPACITY and the block stays unindexed.
+ * no free slot latches LSA_ERR_CAPACITY: the block keeps its leaf label
+ * (LSA_GET_LEAF_OF_BLOCK) but is not selectable until lsa_relayout.
  * [p5 "Prefill, decode and training"; p4 "Prompt processing is not response
  * generation"] */
 int lsa_append(lsa_index* index, const void* K, int64_t n_new, void* stream);
+
+/* Decode maintenance, part 1 (the pages say nothing about keeping the index
+ * up during decode beyond "each new token attends back over the whole
+ * history", p5 "Prefill, decode and training"; this is the plainest
+ * upkeep that leaves the selection rule unchanged).  Lays the leaf buckets of
+ * every unit out again from the current leaf labels: each leaf's blocks in
+ * ascending order, the blocks that lsa_append gave to a full leaf
+ * (LSA_ERR_CAPACITY) included, then fresh free slots for the append capacity
+ * that is left, shared among the leaves in proportion to their sizes as at
+ * the build; minpos of every node is recomputed.  Labels and centroids do not
+ * change, so lsa_select afterwards sees every block exactly where lsa_append
+ * put it.  Clears a latched LSA_ERR_CAPACITY (other latched bits stay).
+ *  - Stream-ordered, no host synchronisation; stream-ordered scratch of about
+ *    5 x 4 B per indexed block.
+ *  - Returns LSA_ERR_CAPACITY, with nothing changed, if the index's slot
+ *    arrays could not hold the layout (cannot happen within the build's
+ *    append_capacity); LSA_ERR_INVALID_ARG for a dead handle. */
+int lsa_relayout(lsa_index* index, void* stream);
+
+/* Decode maintenance, part 2 (a reading like part 1): recompute every
+ * centroid from its current members, memberships fixed, bottom-up: a leaf's
+ * centroid is the mean of the latent keys of its blocks (appended blocks
+ * included, those waiting for lsa_relayout too), an upper node's the mean of
+ * its children's refreshed centroids; the rules of the build's update step
+ * (fp64 sums in ascending member order, an empty node keeps its centroid,
+ * rounding onto the grid when grid_log2 > 0).  Right after a build it changes
+ * nothing.  Later appends use the refreshed leaf centroids.
+ *  - Stream-ordered; scratch as lsa_relayout.  LSA_ERR_INVALID_ARG for a
+ *    dead handle; a broken grid precondition latches LSA_ERR_INEXACT.
+ * [p5 step 1: keys clustered into buckets organised as a hierarchy] */
+int lsa_refresh_centroids(lsa_index* index, void* stream);
 
 /* Stage calls, exposed for checks and for callers that compose the path. */
 

@@ -59,6 +59,16 @@ Readings where the pages are silent (each one is also listed in the design doc):
   R12 softmax scale 1/sqrt(d).
   R13 decode: centroids are frozen; a completed block goes to its nearest leaf
       over all leaves.
+  R18 decode upkeep of the layout: the oracle's leaves are unbounded member
+      lists, so a block always joins its nearest leaf; a device index whose
+      leaf ran out of free slots must, once its leaves are laid out again,
+      hold exactly these lists (nothing in the method changes).
+  R19 centroid refresh during decode (the pages are silent; plainest upkeep
+      consistent with R10): memberships held fixed, every centroid is
+      recomputed bottom-up as the mean of its current members (a leaf from
+      the latent keys of its blocks, appended ones included; an upper node
+      from its children's refreshed centroids), by the rules of
+      ``kmeans_update``.  Right after a build this changes nothing (R10).
   R17 the training-free map [p5 "How does LSA work?", the D-LSA options: "a
       training-free option that uses a PCA map"]: W = the r leading principal
       directions of the pooled keys of every (sequence, KV head), i.e. the
@@ -411,6 +421,21 @@ def nearest_leaf(tree: Tree, x: np.ndarray) -> int:
     """argmin over all leaves of ||x - c||^2 with frozen centroids (R13, R7)."""
     d2 = squared_distances(np.asarray(x, dtype=np.float64)[None, :], tree.centroids[-1])[0]
     return int(np.argmin(d2))
+
+
+def refresh_centroids(tree: Tree, Kl: np.ndarray, grid_log2: int = 0) -> None:
+    """R19: with every membership fixed, each leaf centroid becomes the mean of
+    the latent keys of its blocks (``Kl`` [Nb, r], rows in block order, the
+    appended blocks included), then, level by level upwards, each node's the
+    mean of its children's new centroids; an empty node keeps its centroid and
+    the grid rule of ``kmeans_update`` applies.  Updates ``tree`` in place."""
+    Lv = tree.levels
+    Kl = np.asarray(Kl, dtype=np.float64)
+    if Kl.shape[0] != tree.leaf_of_block.shape[0]:
+        raise ValueError("one latent row per labelled block")
+    tree.centroids[Lv - 1] = kmeans_update(Kl, tree.leaf_of_block, tree.centroids[Lv - 1], grid_log2)
+    for l in range(Lv - 2, -1, -1):
+        tree.centroids[l] = kmeans_update(tree.centroids[l + 1], tree.parent[l + 1], tree.centroids[l], grid_log2)
 
 
 def append_block(tree: Tree, Kl_rows: list, x: np.ndarray) -> int:

@@ -405,3 +405,68 @@ def test_pca_map_is_centred():
     shift = np.array([0.0, 0.0, 0.0, 0.0, 0.0, 50.0])
     W1, ev1 = O.pca_map([K + shift], pool=1, r=3)
     assert np.allclose(W0, W1, atol=1e-9) and np.allclose(ev0, ev1)
+
+
+# ---------------------------------------------------------------- decode upkeep
+def _given_tree(case):
+    """A tree written out by hand (pool 1, sink 0, levels [2, 3])."""
+    t = O.Tree(pool=1, sink=0, level_sizes=[2, 3],
+               centroids=[np.array(case["top_centroids"], dtype=np.float64)[:, None],
+                          np.array(case["leaf_centroids"], dtype=np.float64)[:, None]],
+               parent=[None, np.array([0, 1, 1])],
+               leaf_of_block=np.array(case["leaf_of_block"]), objectives=[[], []])
+    return t.finish()
+
+
+@pytest.mark.parametrize("case", gold("refresh_small.json")["cases"])
+def test_refresh_centroids_worked_examples(case):
+    t = _given_tree(case)
+    rows = [np.array([x]) for x in case["latents"]]
+    for x, want_leaf in zip(case["append"], case["append_leaf"]):
+        assert O.append_block(t, rows, np.array([x])) == want_leaf
+    O.refresh_centroids(t, np.array(rows), case["grid_log2"])
+    np.testing.assert_array_equal(t.centroids[1][:, 0], case["want_leaf_centroids"])
+    np.testing.assert_array_equal(t.centroids[0][:, 0], case["want_top_centroids"])
+
+
+@pytest.mark.parametrize("grid_log2", [0, 4])
+def test_refresh_right_after_a_build_changes_nothing(grid_log2):
+    """R10 makes every built centroid the last update of its level, i.e. the
+    mean of its current members, so a refresh with no append is the identity."""
+    rng = np.random.default_rng(40)
+    X = rng.integers(-4, 5, size=(300, 3)).astype(np.float64) if grid_log2 else rng.standard_normal((300, 3))
+    t = O.build_tree(X, [3, 9, 27], 4, grid_log2, sink=0, pool=1)
+    before = [c.copy() for c in t.centroids]
+    O.refresh_centroids(t, X, grid_log2)
+    for a, b in zip(before, t.centroids):
+        np.testing.assert_array_equal(a, b)
+
+
+def test_refresh_makes_each_centroid_the_mean_of_its_members():
+    """After appends, a refreshed leaf centroid has zero summed offset to its
+    members (the stationarity condition of the squared loss), an upper node's
+    to its children's centroids, and an empty node is unchanged."""
+    rng = np.random.default_rng(41)
+    X = rng.standard_normal((200, 4))
+    t = O.build_tree(X, [2, 6, 40], 3, 0, sink=0, pool=1)
+    rows = [x for x in X]
+    for x in rng.standard_normal((60, 4)) * 2.0:
+        O.append_block(t, rows, x)
+    old = [c.copy() for c in t.centroids]
+    O.refresh_centroids(t, np.array(rows), 0)
+    Kl = np.array(rows)
+    for j in range(t.level_sizes[-1]):
+        mem = np.flatnonzero(t.leaf_of_block == j)
+        if mem.size:
+            assert np.abs((Kl[mem] - t.centroids[-1][j]).sum(axis=0)).max() <= 1e-12 * mem.size
+        else:
+            np.testing.assert_array_equal(t.centroids[-1][j], old[-1][j])
+    for l in range(t.levels - 1):
+        for j in range(t.level_sizes[l]):
+            ch = np.flatnonzero(t.parent[l + 1] == j)
+            if ch.size:
+                assert np.abs((t.centroids[l + 1][ch] - t.centroids[l][j]).sum(axis=0)).max() <= 1e-12 * ch.size
+            else:
+                np.testing.assert_array_equal(t.centroids[l][j], old[l][j])
+    # the appended blocks moved some leaf: the refresh did something
+    assert any(not np.array_equal(a, b) for a, b in zip(old, t.centroids))
