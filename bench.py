@@ -359,6 +359,9 @@ def run_decode(args, w, rank, world, dev):
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / n_timed
     st = lsa.lsa_check(ix)
     info = ix.info()
+    extra = None
+    if not args.no_extra and rank == 0:
+        extra = decode_extra(w, inp, ix, sp, dev)
     ix.free()
     if rank == 0:
         print(json.dumps({
@@ -367,7 +370,55 @@ def run_decode(args, w, rank, world, dev):
             "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic", "config": {"workload": describe(w)}, "build_ms": build_ms,
             "index_device_bytes": int(info.device_bytes), "gpu_launches": lsa.lsa_launch_count() - launches0,
-            "status": lsa.strerror(st), "clocks": clk}), flush=True)
+            "status": lsa.strerror(st), "clocks": clk, "extra": extra}), flush=True)
+
+
+def decode_extra(w, inp, ix, sp, dev):
+    """Not timed in the headline: after the decode steps, every decode query
+    (all steps x sequences, each at its own position; later appends hold only
+    blocks past its causal bound, so its selection is the one it had) is
+    selected at once by the tree and by the full-scan indexer over the whole
+    10M-token context: their times for that batch, the tree's recall of the
+    full scan's long-range picks on a sample, and needle hit rates."""
+    import torch
+    from hierarchical_latent_key_gemm_b200 import lsa
+    N, S = w.n_tokens, w.decode_steps
+    Q = inp["Q"]
+    qpos = (N + torch.arange(S, device=dev, dtype=torch.int64))[None, :].repeat(w.batch, 1).contiguous()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    out = {}
+    for name, fn in (("tree", lsa.lsa_select), ("fullscan", lsa.lsa_fullscan_select)):
+        fn(ix, sp, Q, q_pos=qpos)       # warm-up
+        torch.cuda.synchronize()
+        e0.record()
+        sel = fn(ix, sp, Q, q_pos=qpos)
+        e1.record()
+        torch.cuda.synchronize()
+        out[name] = (e0.elapsed_time(e1), sel)
+    (t_ms, (ti, tc)), (f_ms, (fi, fc)) = out["tree"], out["fullscan"]
+    ti, tc, fi, fc = ti.cpu(), tc.cpu(), fi.cpu(), fc.cpu()
+    hit = tot = 0
+    for b in range(w.batch):
+        for h in range(w.hkv):
+            for s in range(0, S, 8):
+                i = N + s
+                lo = max(0, i - w.window + 1)
+                base = set(range(min(w.sink, lo))) | set(range(lo, i + 1))
+                f = set(fi[b, s, h, : fc[b, s, h]].tolist()) - base
+                t = set(ti[b, s, h, : tc[b, s, h]].tolist()) - base
+                tot += len(f)
+                hit += len(f & t)
+    needles = inp["needles"]
+    nh_t = nh_f = 0
+    for (b, h, p, qp) in needles:
+        s = qp - N
+        nh_t += int(p in set(ti[b, s, h, : tc[b, s, h]].tolist()))
+        nh_f += int(p in set(fi[b, s, h, : fc[b, s, h]].tolist()))
+    return {"queries": w.batch * S, "tree_select_ms": t_ms, "fullscan_select_ms": f_ms,
+            "tree_vs_fullscan_speedup": f_ms / t_ms, "tree_recall_vs_fullscan_topk": hit / max(1, tot),
+            "recall_sample": "every 8th decode step, all sequences",
+            "needle_hit_rate_tree": nh_t / max(1, len(needles)),
+            "needle_hit_rate_fullscan": nh_f / max(1, len(needles)), "needles": len(needles)}
 
 
 def local_rank() -> int:
