@@ -14,11 +14,14 @@
 // One CTA per (query, KV head).  Every tree level is stored in tree order
 // (children of a node are contiguous), so a candidate's minpos, original id
 // and centroid row are independent loads; each sub-warp group of r/16 lanes
-// (16 floats of the row per lane) walks a contiguous run of candidates.  Scores stream through a shared-memory buffer;
-// whenever it holds more than k items a block-wide radix select (on the
-// order-preserving bit pattern of the fp32 score, then on the original id for
-// ties) compacts it to the top k.  The order is total, (score desc, id asc),
-// so the result does not depend on the order in which warps append.
+// (16 floats of the row per lane) walks a contiguous run of candidates.
+// Scores stream through one shared-memory buffer; when it runs low, a
+// block-wide select (on the order-preserving bit pattern of the fp32 score,
+// then on the original id for ties) compacts it in place to the top k.  The
+// order is total, (score desc, id asc), so the result does not depend on the
+// order in which warps append.  One buffer instead of two halves the shared
+// memory of a CTA, which leaves more of each SM's L1 for the centroid rows
+// that every query of a unit reads.
 #include "lsa_internal.cuh"
 
 namespace lsa {
@@ -72,6 +75,8 @@ struct SelShared {
     uint32_t thr;   // no item below this key can be in the current top k (0: none yet)
     uint32_t wmin[32], wmax[32];
     int nres;
+    uint32_t rkey[kResolveCap];   // the items of the threshold bin: key and id
+    int rid[kResolveCap];
 };
 
 // 32 bytes from global memory in one 256-bit read-only load (32-byte aligned).
@@ -158,18 +163,73 @@ __device__ uint32_t block_kth(const float* s, const int* id, int n, int k, int m
     return prefix;
 }
 
-// Keep the top k of the n items in (s, id, ps) by (score desc, id asc), k < n;
-// result in (ds, di, dp)[0..k) in no particular order.  The keys are binned by
-// their offset from the smallest key, shifted so that at most 256 bins are
-// used (monotone in the key); bins above the one that holds the k-th item are
-// taken whole, and that bin's items are ranked exactly by (key, id).  If that
-// bin holds more than kResolveCap items (or all keys are equal), the general
-// radix select below runs instead.
-__device__ void topk_compact_radix(const float* s, const int* id, const int* ps, int n, int k, float* ds, int* di,
-                                   int* dp, SelShared& sh);
+// Keep, in place, the items of (s, id, ps)[0, n) whose (key, id) pass `take`;
+// they end up in [0, sh.count2) in no particular order.  Items move in rounds
+// of kRound per thread: every thread holds its items of a round in registers
+// before any thread writes, and since no more items are kept than were read,
+// a kept item never lands past the round it came from.
+constexpr int kRound = 4;
 
-__device__ void topk_compact(const float* s, const int* id, const int* ps, int n, int k, float* ds, int* di,
-                             int* dp, SelShared& sh) {
+template <typename Take>
+__device__ void filter_in_place(float* s, int* id, int* ps, int n, SelShared& sh, Take&& take) {
+    if (threadIdx.x == 0) sh.count2 = 0;
+    __syncthreads();
+    const int T = blockDim.x;
+    for (int r0 = 0; r0 < n; r0 += kRound * T) {
+        float vs[kRound];
+        int vi[kRound], vp[kRound];
+        bool tk[kRound];
+#pragma unroll
+        for (int j = 0; j < kRound; ++j) {
+            const int i = r0 + j * T + (int)threadIdx.x;
+            tk[j] = false;
+            vs[j] = 0.f;
+            vi[j] = vp[j] = 0;
+            if (i < n) {
+                vs[j] = s[i];
+                vi[j] = id[i];
+                vp[j] = ps[i];
+                tk[j] = take(fkey(vs[j]), vi[j]);
+            }
+        }
+        __syncthreads();   // the whole round is in registers
+#pragma unroll
+        for (int j = 0; j < kRound; ++j) {
+            if (tk[j]) {
+                const int p = atomicAdd(&sh.count2, 1);
+                s[p] = vs[j];
+                id[p] = vi[j];
+                ps[p] = vp[j];
+            }
+        }
+        __syncthreads();
+    }
+}
+
+// General form: exact k-th key by 8-bit radix passes, then ties by id.
+__device__ void topk_compact_radix(float* s, int* id, int* ps, int n, int k, SelShared& sh) {
+    int need, eq;
+    const uint32_t T = block_kth(s, id, n, k, 0, 0u, sh, &need, &eq);
+    const bool split = need < eq;
+    uint32_t T2 = 0;
+    if (split) {
+        int need2, eq2;
+        T2 = block_kth(s, id, n, need, 1, T, sh, &need2, &eq2);
+    }
+    if (threadIdx.x == 0) sh.thr = T;
+    filter_in_place(s, id, ps, n, sh, [&](uint32_t key, int xi) {
+        return key > T || (key == T && (!split || ~(uint32_t)xi >= T2));
+    });
+}
+
+// Keep, in place, the top k of the n items in (s, id, ps) by (score desc, id
+// asc), k < n; the result is (s, id, ps)[0..k) in no particular order.  The
+// keys are binned by their offset from the smallest key, shifted so that at
+// most 256 bins are used (monotone in the key); bins above the one that holds
+// the k-th item are taken whole, and that bin's items are ranked exactly by
+// (key, id).  If that bin holds more than kResolveCap items (or all keys are
+// equal), the general radix select runs instead.
+__device__ void topk_compact(float* s, int* id, int* ps, int n, int k, SelShared& sh) {
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
     uint32_t kmn = 0xffffffffu, kmx = 0u;
     for (int i = tid; i < n; i += blockDim.x) {
@@ -183,7 +243,7 @@ __device__ void topk_compact(const float* s, const int* id, const int* ps, int n
         kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, o));
     }
     if (lane == 0) { sh.wmin[warp] = kmn; sh.wmax[warp] = kmx; }
-    if (tid == 0) { sh.count2 = 0; sh.nres = 0; }
+    if (tid == 0) sh.nres = 0;
     __syncthreads();
     kmn = sh.wmin[0];
     kmx = sh.wmax[0];
@@ -192,7 +252,7 @@ __device__ void topk_compact(const float* s, const int* id, const int* ps, int n
         kmx = max(kmx, sh.wmax[w]);
     }
     if (kmn == kmx) {
-        topk_compact_radix(s, id, ps, n, k, ds, di, dp, sh);
+        topk_compact_radix(s, id, ps, n, k, sh);
         return;
     }
     const int shift = max(0, 24 - __clz(kmx - kmn));   // (kmx - kmn) >> shift <= 255
@@ -226,77 +286,34 @@ __device__ void topk_compact(const float* s, const int* id, const int* ps, int n
     const uint32_t B = (uint32_t)sh.bc[0];
     const int need = sh.bc[1], cntB = sh.bc[2];
     const bool all_b = need == cntB;
-    // bin B's items wait in the free tail [k, k + cntB) of the destination
-    // (the caller's buffers hold at least 2k items): key, id, source index
-    uint32_t* rk = reinterpret_cast<uint32_t*>(ds + k);
-    int* rid = di + k;
-    int* rsrc = dp + k;
     if (!all_b && cntB > min(kResolveCap, k)) {
-        topk_compact_radix(s, id, ps, n, k, ds, di, dp, sh);
+        topk_compact_radix(s, id, ps, n, k, sh);
         return;
     }
-    for (int i = tid; i < n; i += blockDim.x) {
-        const uint32_t key = fkey(s[i]);
-        const uint32_t b = (key - kmn) >> shift;
-        if (b > B || (b == B && all_b)) {
-            const int p = atomicAdd(&sh.count2, 1);
-            ds[p] = s[i];
-            di[p] = id[i];
-            dp[p] = ps[i];
-        } else if (b == B) {
-            const int r = atomicAdd(&sh.nres, 1);
-            rk[r] = key;
-            rid[r] = id[i];
-            rsrc[r] = i;
+    if (!all_b) {
+        // bin B's items, to be ranked among themselves (keys are distinct: ids are)
+        for (int i = tid; i < n; i += blockDim.x) {
+            const uint32_t key = fkey(s[i]);
+            if (((key - kmn) >> shift) == B) {
+                const int r = atomicAdd(&sh.nres, 1);
+                sh.rkey[r] = key;
+                sh.rid[r] = id[i];
+            }
         }
     }
     if (tid == 0) sh.thr = kmn + (B << shift);   // smallest key that falls in bin B
-    __syncthreads();
-    if (!all_b) {
-        // rank of each item of bin B among them (keys are distinct: ids are)
-        for (int r = tid; r < cntB; r += blockDim.x) {
-            const uint32_t xk = rk[r];
-            const int xi = rid[r];
-            int rank = 0;
-            for (int j = 0; j < cntB; ++j) {
-                const uint32_t yk = rk[j];
-                rank += yk > xk || (yk == xk && rid[j] < xi);
-            }
-            if (rank < need) {
-                const int i = rsrc[r];
-                const int p = atomicAdd(&sh.count2, 1);
-                ds[p] = s[i];
-                di[p] = id[i];
-                dp[p] = ps[i];
-            }
+    // (filter_in_place's first barrier publishes the bin-B list and thr)
+    filter_in_place(s, id, ps, n, sh, [&](uint32_t key, int xi) {
+        const uint32_t b = (key - kmn) >> shift;
+        if (b != B) return b > B;
+        if (all_b) return true;
+        int rank = 0;
+        for (int j = 0; j < cntB; ++j) {
+            const uint32_t yk = sh.rkey[j];
+            rank += yk > key || (yk == key && sh.rid[j] < xi);
         }
-        __syncthreads();
-    }
-}
-
-// General form: exact k-th key by 8-bit radix passes, then ties by id.
-__device__ void topk_compact_radix(const float* s, const int* id, const int* ps, int n, int k, float* ds, int* di,
-                                   int* dp, SelShared& sh) {
-    int need, eq;
-    const uint32_t T = block_kth(s, id, n, k, 0, 0u, sh, &need, &eq);
-    const bool split = need < eq;
-    uint32_t T2 = 0;
-    if (split) {
-        int need2, eq2;
-        T2 = block_kth(s, id, n, need, 1, T, sh, &need2, &eq2);
-    }
-    if (threadIdx.x == 0) sh.thr = T;
-    for (int i = threadIdx.x; i < n; i += blockDim.x) {
-        const uint32_t key = fkey(s[i]);
-        const bool take = key > T || (key == T && (!split || ~(uint32_t)id[i] >= T2));
-        if (take) {
-            const int p = atomicAdd(&sh.count2, 1);
-            ds[p] = s[i];
-            di[p] = id[i];
-            dp[p] = ps[i];
-        }
-    }
-    __syncthreads();
+        return rank < need;
+    });
 }
 
 // Exclusive scan of pre[0..n) in place (values are counts), pre[n] = total.
@@ -337,14 +354,11 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
     const SelArgs a) {
     extern __shared__ float4 dyn4[];
     __shared__ SelShared sh;
-    // two buffers of (score, id, position) x cap, selected by `cur`
-    // (pointer arithmetic, not an indexed array, so nothing lives in local memory)
-    float* const buf0 = reinterpret_cast<float*>(dyn4);
-    const int bstride = 3 * a.cap;
-    auto bsb = [&](int c) { return buf0 + c * bstride; };
-    auto bib = [&](int c) { return reinterpret_cast<int*>(buf0 + c * bstride + a.cap); };
-    auto bpb = [&](int c) { return reinterpret_cast<int*>(buf0 + c * bstride + 2 * a.cap); };
-    int* kk = reinterpret_cast<int*>(buf0 + 2 * bstride);   // kept positions [beam]
+    // one buffer of (score, id, position) x cap, compacted in place
+    float* const bs = reinterpret_cast<float*>(dyn4);
+    int* const bi = reinterpret_cast<int*>(bs + a.cap);
+    int* const bp = reinterpret_cast<int*>(bs + 2 * a.cap);
+    int* kk = reinterpret_cast<int*>(bs + 3 * a.cap);   // kept positions [beam]
     int* pre = kk + a.beam;          // [beam + 1]
     int* lo = pre + a.beam + 1;      // [beam]
 
@@ -398,7 +412,6 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
     if (threadIdx.x == 0) { sh.count = 0; sh.nkept = 0; sh.thr = 0u; }
     __syncthreads();
 
-    int cur = 0;
     unsigned nscored = 0;   // eligible candidates this thread's group scored (leader lanes)
     uint32_t lt_mask;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt_mask));
@@ -420,9 +433,6 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
         while (t0 < total) {
             const uint32_t thr = sh.thr;
             const int t1 = min(total, t0 + (a.cap - nbuf));
-            float* bs = bsb(cur);
-            int* bi = bib(cur);
-            int* bp = bpb(cur);
             const int span = (t1 - t0 + NG - 1) / NG;
             const int tb = t0 + gid * span;
             const int te = min(t1, tb + span);
@@ -469,8 +479,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
             const int n = sh.count;
             // compact when done, or when less than a quarter of the buffer is free
             if (n > k && (t0 >= total || a.cap - n < a.cap / 4)) {
-                topk_compact(bs, bi, bp, n, k, bsb(cur ^ 1), bib(cur ^ 1), bpb(cur ^ 1), sh);
-                cur ^= 1;
+                topk_compact(bs, bi, bp, n, k, sh);
                 if (threadIdx.x == 0) sh.count = k;
                 nbuf = k;
             } else {
@@ -514,7 +523,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
                 *el = __ldg(mp + q) <= bound;
             });
             const int n = sh.count;
-            for (int e = threadIdx.x; e < n; e += blockDim.x) kk[e] = bpb(cur)[e];
+            for (int e = threadIdx.x; e < n; e += blockDim.x) kk[e] = bp[e];
             __syncthreads();
             if (threadIdx.x == 0) sh.nkept = n;
             if (l + 1 < a.levels) {
@@ -537,7 +546,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
         // loads of a leaf are in flight together)
         const int nk = sh.nkept;
         const int L = a.n_l[a.levels - 1];
-        const int* kept_id = bib(cur);
+        const int* kept_id = bi;
         for (int e = threadIdx.x; e < nk; e += blockDim.x) {
             const int64_t c = (int64_t)u * L + kept_id[e];
             const int st = a.leaf_start[c];
@@ -584,10 +593,10 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
     const int nsel = sh.count;
 
     // ascending block ids
-    int* arr = bib(cur ^ 1);
+    int* arr = bp;   // the positions are no longer needed
     if (THREADS >= 512) {
         // wide CTAs: rank sort (each id counts the smaller ones), one barrier
-        const int* src = bib(cur);
+        const int* src = bi;
         for (int e = threadIdx.x; e < nsel; e += THREADS) {
             const int x = src[e];
             int rank = 0;
@@ -602,7 +611,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
         // memory
         constexpr int M = 4 * THREADS;
         int v[4];
-        const int* src = bib(cur);
+        const int* src = bi;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
             const int i = 4 * threadIdx.x + k;
@@ -660,7 +669,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
         // bitonic sort, padded to a power of two
         int M = 1;
         while (M < nsel) M <<= 1;
-        for (int e = threadIdx.x; e < M; e += blockDim.x) arr[e] = e < nsel ? bib(cur)[e] : INT32_MAX;
+        for (int e = threadIdx.x; e < M; e += blockDim.x) arr[e] = e < nsel ? bi[e] : INT32_MAX;
         __syncthreads();
         for (int size = 2; size <= M; size <<= 1) {
             for (int stride = size >> 1; stride > 0; stride >>= 1) {
@@ -711,7 +720,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
 
 template <int R, int THREADS>
 int launch_select_t(const SelArgs& a, int64_t nq, int64_t units, bool fullscan, cudaStream_t s) {
-    const size_t smem = (size_t)a.cap * 24 + (size_t)(3 * a.beam + 1) * 4;
+    const size_t smem = (size_t)a.cap * 12 + (size_t)(3 * a.beam + 1) * 4;
     auto kern = fullscan ? select_kernel<R, true, THREADS, false>
                          : (a.work ? select_kernel<R, false, THREADS, true> : select_kernel<R, false, THREADS, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -731,7 +740,7 @@ int launch_select_r(const SelArgs& a, int64_t nq, int64_t units, bool fullscan, 
         // one CTA per SM at most: a buffer that holds a whole level (fewer
         // compaction rounds), within the 227 KB a CTA may use
         SelArgs w = a;
-        while (w.cap < kWideCap && (size_t)(2 * w.cap) * 24 + (size_t)(3 * w.beam + 1) * 4 <= 200 * 1024) w.cap *= 2;
+        while (w.cap < kWideCap && (size_t)(2 * w.cap) * 12 + (size_t)(3 * w.beam + 1) * 4 <= 200 * 1024) w.cap *= 2;
         return launch_select_t<R, kWideThreads>(w, nq, units, fullscan, s);
     }
     return launch_select_t<R, kSelThreads>(a, nq, units, fullscan, s);
