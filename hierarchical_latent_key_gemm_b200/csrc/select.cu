@@ -64,7 +64,13 @@ struct SelArgs {
     unsigned long long* work;   // optional: += eligible nodes and blocks scored
 };
 
-constexpr int kResolveCap = 256;   // most items of the threshold bin ranked pairwise
+constexpr int kResolveCap = 256;
+
+// a candidate group's current owner among the kept nodes: its index, the first
+// candidate past its run, and (its run's first slot - its first candidate)
+struct OwnerState {
+    int o, next, base;
+};   // most items of the threshold bin ranked pairwise
 
 struct SelShared {
     int hist[256];
@@ -365,6 +371,8 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
     constexpr int LPC = R / 16;             // lanes per candidate row (16 floats each)
     constexpr int CPW = 32 / LPC;           // candidates per warp
     constexpr int NG = (THREADS / 32) * CPW;
+    // ids sorted in registers: 512 for the narrow CTAs
+    constexpr int kSortIpt = THREADS >= 512 ? 1 : (512 / THREADS > 4 ? 512 / THREADS : 4);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane / LPC, gl = lane % LPC, gid = warp * CPW + g;
     const unsigned gmask = (LPC == 32) ? 0xffffffffu : (((1u << LPC) - 1u) << (g * LPC));
@@ -436,7 +444,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
             const int span = (t1 - t0 + NG - 1) / NG;
             const int tb = t0 + gid * span;
             const int te = min(t1, tb + span);
-            int state = -1;
+            OwnerState state{-1, 0, 0};
             for (int s0 = 0; s0 < span; s0 += kUnroll) {
                 float y[kUnroll][16];
                 int idv[kUnroll], pv[kUnroll];
@@ -491,12 +499,21 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
 
     // owner of candidate t among the nk kept nodes (ranges pre[o]..pre[o+1]),
     // advanced from the previous candidate's owner
-    auto owner = [&](int t, int nk, int* state) -> int {
-        int o = *state;
-        if (o < 0) o = find_owner(pre, nk, t);
-        while (pre[o + 1] <= t) ++o;
-        *state = o;
-        return o;
+    // slot (or child position) of candidate t: the owner's run starts at
+    // lo[o] for t = pre[o]; the owner, its run's end and base stay in registers
+    auto slot_of = [&](int t, int nk, OwnerState* st) -> int {
+        if (st->o < 0) {
+            const int o = find_owner(pre, nk, t);
+            st->o = o;
+            st->next = pre[o + 1];
+            st->base = lo[o] - pre[o];
+        }
+        while (t >= st->next) {
+            const int o = ++st->o;
+            st->next = pre[o + 1];
+            st->base = lo[o] - pre[o];
+        }
+        return st->base + t;
     };
 
     if (!FULL) {
@@ -509,13 +526,12 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
             const int total = (l == 0) ? nl : pre[nk];
             if (threadIdx.x == 0) sh.count = 0;
             __syncthreads();
-            stream_topk(total, a.beam, [&](int t, int* state, bool* el, int* id, int* p, float* y) {
+            stream_topk(total, a.beam, [&](int t, OwnerState* state, bool* el, int* id, int* p, float* y) {
                 int q;
                 if (l == 0) {
                     q = t;
                 } else {
-                    const int o = owner(t, nk, state);
-                    q = lo[o] + (t - pre[o]);
+                    q = slot_of(t, nk, state);
                 }
                 load_row(cent + (int64_t)q * R, y);
                 *id = __ldg(oid + q);
@@ -569,9 +585,8 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
         scan_pre(pre, nk);
         if (threadIdx.x == 0) sh.count = 0;
         __syncthreads();
-        stream_topk(pre[nk], a.kb, [&](int t, int* state, bool* el, int* id, int* p, float* y) {
-            const int o = owner(t, nk, state);
-            const int64_t slot = lo[o] + (t - pre[o]);
+        stream_topk(pre[nk], a.kb, [&](int t, OwnerState* state, bool* el, int* id, int* p, float* y) {
+            const int64_t slot = slot_of(t, nk, state);
             load_row(a.Klp + slot * R, y);
             *id = __ldg(a.blk + slot);
             *p = 0;
@@ -581,7 +596,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
         const int64_t hi = min(a.nb - 1, b_hi);
         const int total = hi >= b_lo ? (int)(hi - b_lo + 1) : 0;
         const float* kl = a.Kl + (int64_t)u * a.nb_cap * R;
-        stream_topk(total, a.kb, [&](int t, int* state, bool* el, int* id, int* p, float* y) {
+        stream_topk(total, a.kb, [&](int t, OwnerState* state, bool* el, int* id, int* p, float* y) {
             (void)state;
             const int64_t b = b_lo + t;
             load_row(kl + b * R, y);
@@ -604,66 +619,65 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
             arr[rank] = x;
         }
         __syncthreads();
-    } else if (nsel <= 4 * THREADS) {
-        // bitonic sort of 4 * THREADS items (padded with INT32_MAX), 4 per
-        // thread in registers: item i = 4 tid + k; strides 1-2 inside a
-        // thread, 4-64 across lanes by shuffles, 128 and up through shared
-        // memory
-        constexpr int M = 4 * THREADS;
-        int v[4];
+    } else if (nsel <= kSortIpt * THREADS) {
+        // bitonic sort of IPT * THREADS items (padded with INT32_MAX), IPT per
+        // thread in registers: item i = IPT tid + k; strides below IPT inside
+        // a thread, up to 16 IPT across lanes by shuffles, 32 IPT and up
+        // through shared memory
+        constexpr int IPT = kSortIpt;
+        constexpr int M = IPT * THREADS;
+        int v[IPT];
         const int* src = bi;
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-            const int i = 4 * threadIdx.x + k;
+        for (int k = 0; k < IPT; ++k) {
+            const int i = IPT * threadIdx.x + k;
             v[k] = i < nsel ? src[i] : INT32_MAX;
         }
         __syncthreads();   // src and arr may be read and written below
         for (int size = 2; size <= M; size <<= 1) {
             for (int stride = size >> 1; stride > 0; stride >>= 1) {
-                if (stride >= 128) {
+                if (stride >= 32 * IPT) {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) arr[4 * threadIdx.x + k] = v[k];
+                    for (int k = 0; k < IPT; ++k) arr[IPT * threadIdx.x + k] = v[k];
                     __syncthreads();
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const int i = 4 * threadIdx.x + k;
+                    for (int k = 0; k < IPT; ++k) {
+                        const int i = IPT * threadIdx.x + k;
                         const int y = arr[i ^ stride];
                         const bool asc = (i & size) == 0;
                         const bool lower = (i & stride) == 0;
                         v[k] = (lower == asc) ? min(v[k], y) : max(v[k], y);
                     }
                     __syncthreads();
-                } else if (stride >= 4) {
+                } else if (stride >= IPT) {
 #pragma unroll
-                    for (int k = 0; k < 4; ++k) {
-                        const int i = 4 * threadIdx.x + k;
-                        const int y = __shfl_xor_sync(0xffffffffu, v[k], stride >> 2);
+                    for (int k = 0; k < IPT; ++k) {
+                        const int i = IPT * threadIdx.x + k;
+                        const int y = __shfl_xor_sync(0xffffffffu, v[k], stride / IPT);
                         const bool asc = (i & size) == 0;
                         const bool lower = (i & stride) == 0;
                         v[k] = (lower == asc) ? min(v[k], y) : max(v[k], y);
                     }
                 } else {
-                    // pairs (0, s), (1, 1 + s) ... inside the thread; written out
-                    // per stride so every register index is a constant
-                    // (direction of the pair starting at item k: ((4 tid + k) & size) == 0)
-                    auto cx = [&](int k, int& x, int& y) {
-                        const bool asc = ((4 * (int)threadIdx.x + k) & size) == 0;
-                        const int lo = min(x, y), hi = max(x, y);
-                        x = asc ? lo : hi;
-                        y = asc ? hi : lo;
-                    };
-                    if (stride == 2) {
-                        cx(0, v[0], v[2]);
-                        cx(1, v[1], v[3]);
-                    } else {
-                        cx(0, v[0], v[1]);
-                        cx(2, v[2], v[3]);
+                    // pairs (k, k + stride) inside the thread; every stride is
+                    // unrolled so every register index is a constant
+#pragma unroll
+                    for (int st = IPT / 2; st >= 1; st >>= 1) {
+                        if (st != stride) continue;
+#pragma unroll
+                        for (int k = 0; k < IPT; ++k) {
+                            if (k & st) continue;
+                            const bool asc = ((IPT * (int)threadIdx.x + k) & size) == 0;
+                            const int lo = min(v[k], v[k + st]), hi = max(v[k], v[k + st]);
+                            v[k] = asc ? lo : hi;
+                            v[k + st] = asc ? hi : lo;
+                        }
                     }
                 }
             }
         }
 #pragma unroll
-        for (int k = 0; k < 4; ++k) arr[4 * threadIdx.x + k] = v[k];
+        for (int k = 0; k < IPT; ++k) arr[IPT * threadIdx.x + k] = v[k];
         __syncthreads();
     } else {
         // bitonic sort, padded to a power of two
