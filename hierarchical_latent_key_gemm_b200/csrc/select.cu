@@ -64,7 +64,7 @@ struct SelArgs {
     unsigned long long* work;   // optional: += eligible nodes and blocks scored
 };
 
-constexpr int kResolveCap = 256;
+constexpr int kResolveCap = 128;
 
 // a candidate group's current owner among the kept nodes: its index, the first
 // candidate past its run, and (its run's first slot - its first candidate)
@@ -81,8 +81,6 @@ struct SelShared {
     uint32_t thr;   // no item below this key can be in the current top k (0: none yet)
     uint32_t wmin[32], wmax[32];
     int nres;
-    uint32_t rkey[kResolveCap];   // the items of the threshold bin: key and id
-    int rid[kResolveCap];
 };
 
 // 32 bytes from global memory in one 256-bit read-only load (32-byte aligned).
@@ -296,14 +294,17 @@ __device__ void topk_compact(float* s, int* id, int* ps, int n, int k, SelShared
         topk_compact_radix(s, id, ps, n, k, sh);
         return;
     }
+    // bin B's items, to be ranked among themselves (keys are distinct: ids
+    // are), listed in the histogram's storage (all zero again afterwards)
+    uint32_t* const rkey = reinterpret_cast<uint32_t*>(sh.hist);
+    int* const rid = sh.hist + kResolveCap;
     if (!all_b) {
-        // bin B's items, to be ranked among themselves (keys are distinct: ids are)
         for (int i = tid; i < n; i += blockDim.x) {
             const uint32_t key = fkey(s[i]);
             if (((key - kmn) >> shift) == B) {
                 const int r = atomicAdd(&sh.nres, 1);
-                sh.rkey[r] = key;
-                sh.rid[r] = id[i];
+                rkey[r] = key;
+                rid[r] = id[i];
             }
         }
     }
@@ -315,11 +316,16 @@ __device__ void topk_compact(float* s, int* id, int* ps, int n, int k, SelShared
         if (all_b) return true;
         int rank = 0;
         for (int j = 0; j < cntB; ++j) {
-            const uint32_t yk = sh.rkey[j];
-            rank += yk > key || (yk == key && sh.rid[j] < xi);
+            const uint32_t yk = rkey[j];
+            rank += yk > key || (yk == key && rid[j] < xi);
         }
         return rank < need;
     });
+    if (!all_b) {
+        // (filter_in_place ended with a barrier: nobody reads the list any more;
+        // the next user of the histogram is behind further barriers)
+        for (int e = tid; e < 2 * kResolveCap; e += blockDim.x) sh.hist[e] = 0;
+    }
 }
 
 // Exclusive scan of pre[0..n) in place (values are counts), pre[n] = total.
@@ -739,6 +745,15 @@ int launch_select_t(const SelArgs& a, int64_t nq, int64_t units, bool fullscan, 
                          : (a.work ? select_kernel<R, false, THREADS, true> : select_kernel<R, false, THREADS, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_status(e);
+    if (THREADS == kSelThreads) {
+        // ask for no more shared memory than the resident CTAs need (each also
+        // holds 1 KB for the system): the rest of the SM's 256 KB stays L1,
+        // which keeps the upper tree levels that every query scores
+        const int per = (int)(smem + sizeof(SelShared) + 1024);
+        const int pct = (LSA_SELECT_MIN_BLOCKS * per * 100 + 233471) / 233472;
+        cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, pct);
+        cudaGetLastError();
+    }
     dim3 grid((unsigned)nq, (unsigned)units);
     note_launch();
     kern<<<grid, THREADS, smem, s>>>(a);
