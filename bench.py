@@ -428,9 +428,9 @@ def local_rank() -> int:
 def run_e2e(args, w, inp, bp, sp, idx, cnt, O, lse, dev, world):
     """Same metric through the public API with HOST buffers: every step copies
     Q, K, V, W from pinned host memory and reads O back
-    (hierarchical_latent_key_gemm_b200.pipeline.HostPrefill: K, V, W up, index
-    build while Q goes up in 8 chunks, select + banded attention per chunk,
-    each O chunk back while the next computes)."""
+    (hierarchical_latent_key_gemm_b200.pipeline.HostPrefill: K, W up, index
+    build while V and then Q go up (Q in 16 chunks), select + banded attention
+    per chunk, each O chunk back while the next computes)."""
     import torch
     from hierarchical_latent_key_gemm_b200.pipeline import HostPrefill
     hQ = inp["Q"].cpu().pin_memory()
@@ -438,7 +438,7 @@ def run_e2e(args, w, inp, bp, sp, idx, cnt, O, lse, dev, world):
     hV = inp["V"].cpu().pin_memory()
     hW = inp["W"].cpu().pin_memory()
     hO = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
-    hp = HostPrefill(bp, sp, hQ, hK, hV, hW, hO, w.sink, w.window, chunks=8, device=dev)
+    hp = HostPrefill(bp, sp, hQ, hK, hV, hW, hO, w.sink, w.window, chunks=16, device=dev)
 
     n = max(1, min(args.steps, 3))
     hp.run().free()
@@ -453,7 +453,7 @@ def run_e2e(args, w, inp, bp, sp, idx, cnt, O, lse, dev, world):
     ms = max_over_ranks(t0.elapsed_time(t1), world, dev) / n
     return {"value": world * w.n_tokens * w.batch / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
             "h2d_bytes_per_step": hp.h2d_bytes, "d2h_bytes_per_step": hp.d2h_bytes,
-            "pipeline": "3 streams; Q up and O down in 8 chunks overlapped with select + attention"}
+            "pipeline": "3 streams; K, W up, then V during the build; Q up and O down in 16 chunks overlapped with select + attention"}
 
 
 def run_extra(w, inp, bp, sp, dev, select_ms, idx, cnt):

@@ -1,8 +1,8 @@
 """Orchestration of the library calls on streams and graphs (no arithmetic).
 
 HostPrefill: a whole prefill layer from host memory, with the copies
-overlapped.  Binding calls and torch copies on three CUDA streams: K, V and W
-go up first and the index is built while the queries go up chunk by chunk;
+overlapped.  Binding calls and torch copies on three CUDA streams: K and W go
+up first, and the index is built while V and then the queries go up chunk by chunk;
 each chunk of consecutive queries is selected and attended (banded attention)
 as soon as its queries have arrived, and its output goes back to the host
 while the next chunk computes.  Every step moves all of Q, K, V and W up and
@@ -67,20 +67,23 @@ class HostPrefill:
         start.record(cur)
         for s in (self.s_in, self.s_comp, self.s_out):
             s.wait_event(start)
-        ev_kvw = torch.cuda.Event()
+        ev_kw, ev_v = torch.cuda.Event(), torch.cuda.Event()
         q_ev, o_ev = [], []
         with torch.cuda.stream(self.s_in):
+            # K and W first (the build needs them); V goes up during the build
             self.dK.copy_(self.hK, non_blocking=True)
-            self.dV.copy_(self.hV, non_blocking=True)
             self.dW.copy_(self.hW, non_blocking=True)
-            ev_kvw.record(self.s_in)
+            ev_kw.record(self.s_in)
+            self.dV.copy_(self.hV, non_blocking=True)
+            ev_v.record(self.s_in)
             for a, b in zip(self.bounds[:-1], self.bounds[1:]):
                 self.dQ[:, a:b].copy_(self.hQ[:, a:b], non_blocking=True)
                 e = torch.cuda.Event()
                 e.record(self.s_in)
                 q_ev.append(e)
-        self.s_comp.wait_event(ev_kvw)
+        self.s_comp.wait_event(ev_kw)
         ix = lsa.lsa_build_index(self.bp, self.dK, self.dW, stream=self.s_comp)
+        self.s_comp.wait_event(ev_v)
         for c, (a, b) in enumerate(zip(self.bounds[:-1], self.bounds[1:])):
             self.s_comp.wait_event(q_ev[c])
             n = b - a
