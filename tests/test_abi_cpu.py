@@ -35,6 +35,10 @@ def test_status_strings_and_null_handles():
     bogus = C.c_void_p(0x1234)
     L.lsa_free_index(bogus)  # not a live index: ignored, never dereferenced
     assert L.lsa_index_info(bogus, C.byref(info)) == lsa.LSA_ERR_INVALID_ARG
+    # index upkeep refuses handles that are not live indexes before any CUDA call
+    for f in (L.lsa_relayout, L.lsa_refresh_centroids):
+        assert f(None, None) == lsa.LSA_ERR_INVALID_ARG
+        assert f(bogus, None) == lsa.LSA_ERR_INVALID_ARG
 
 
 def test_struct_layout_matches_c_header():
