@@ -11,16 +11,18 @@
 // minpos) until the leaves are laid out again (relayout_leaves).
 //
 // Three launches: latents of the new blocks; the nearest-leaf scan spread over
-// many CTAs (each takes a chunk of leaves, one warp per leaf row, and folds its
-// best (distance, leaf) into one 64-bit key per block with atomicMin, so ties
-// go to the lower leaf); the ordered insertion, one CTA per unit.
+// many CTAs (each takes a chunk of 128 leaves, eight lanes per leaf row, and
+// folds its best (distance, leaf) into one 64-bit key per block with
+// atomicMin, so ties go to the lower leaf); the ordered insertion, one CTA per
+// unit.
 #include "latent_common.cuh"
 
 namespace lsa {
 namespace {
 
 constexpr int kAppThreads = 256;
-constexpr int kLeavesPerCta = 512;
+constexpr int kLeavesPerCta = 128;
+constexpr int kLanesPerLeaf = 8;
 
 struct AppArgs {
     const float* W;
@@ -64,11 +66,17 @@ __global__ __launch_bounds__(kAppThreads) void append_latent_kernel(const T* __r
 }
 
 // Nearest leaf, one chunk of leaves per CTA: blockIdx.x = chunk, blockIdx.y =
-// unit.  One warp per leaf row (lanes split the dims, fixed reduction order).
+// unit.  Groups of kLanesPerLeaf lanes take one leaf row each (a lane sums
+// every kLanesPerLeaf-th dimension, then the group adds by shuffles), so a
+// warp has 32 / kLanesPerLeaf rows in flight; each warp folds its best
+// (distance, leaf) key by shuffles and issues one atomicMin per new block.
 __global__ __launch_bounds__(kAppThreads) void append_nearest_kernel(const AppArgs a) {
     extern __shared__ float xs[];       // [n_new][r] latents of the new blocks
+    constexpr int kGroups = kAppThreads / kLanesPerLeaf;   // leaf rows in flight per CTA
     const int u = blockIdx.y;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int sub = lane % kLanesPerLeaf;
+    const int grp = warp * (32 / kLanesPerLeaf) + lane / kLanesPerLeaf;
     for (int e = threadIdx.x; e < a.n_new * a.r; e += kAppThreads)
         xs[e] = a.Kl[((int64_t)u * a.nb_cap + a.first_block + e / a.r) * a.r + e % a.r];
     __syncthreads();
@@ -79,31 +87,42 @@ __global__ __launch_bounds__(kAppThreads) void append_nearest_kernel(const AppAr
     for (int64_t nb = 0; nb < a.n_new; ++nb) {
         const float* x = xs + nb * a.r;
         unsigned long long best = ~0ull;
-        for (int j = j0 + warp; j < j1; j += kAppThreads / 32) {
-            const float* c = cl + (int64_t)j * a.r;
-            unsigned long long key;
+        // the trip count is the same for every lane (shuffles below); a group
+        // past the chunk's end reads the chunk's first row and drops the result
+        for (int jb = j0; jb < j1; jb += kGroups) {
+            const int j = jb + grp;
+            const bool valid = j < j1;
+            const float* c = cl + (int64_t)(valid ? j : j0) * a.r;
+            unsigned long long key = ~0ull;
             if (a.grid_log2 > 0) {
                 long long s = 0;
-                for (int e = lane; e < a.r; e += 32) {
+                for (int e = sub; e < a.r; e += kLanesPerLeaf) {
                     const long long dd = (long long)(x[e] * scale) - (long long)(c[e] * scale);
                     s += dd * dd;
                 }
 #pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-                if (s >= (1ll << 43)) latch(a.err, kErrInexact);
-                key = ((unsigned long long)s << 20) | (unsigned)j;
+                for (int o = kLanesPerLeaf / 2; o >= 1; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+                if (valid) {
+                    if (s >= (1ll << 43)) latch(a.err, kErrInexact);
+                    key = ((unsigned long long)s << 20) | (unsigned)j;
+                }
             } else {
                 float s = 0.f;
-                for (int e = lane; e < a.r; e += 32) {
+                for (int e = sub; e < a.r; e += kLanesPerLeaf) {
                     const float dd = __fsub_rn(x[e], c[e]);
                     s = __fmaf_rn(dd, dd, s);
                 }
 #pragma unroll
-                for (int o = 16; o >= 1; o >>= 1) s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, o));
+                for (int o = kLanesPerLeaf / 2; o >= 1; o >>= 1) s = __fadd_rn(s, __shfl_xor_sync(0xffffffffu, s, o));
                 // distances are >= 0, so their bit patterns order like the values
-                key = ((unsigned long long)__float_as_uint(s) << 32) | (unsigned)j;
+                if (valid) key = ((unsigned long long)__float_as_uint(s) << 32) | (unsigned)j;
             }
             best = key < best ? key : best;
+        }
+#pragma unroll
+        for (int o = 16; o >= kLanesPerLeaf; o >>= 1) {
+            const unsigned long long other = __shfl_xor_sync(0xffffffffu, best, o);
+            best = other < best ? other : best;
         }
         if (lane == 0 && best != ~0ull) atomicMin(a.best + (int64_t)u * a.n_new + nb, best);
     }
