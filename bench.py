@@ -75,27 +75,34 @@ def barrier(world: int):
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons, sampled every 200 ms."""
+    """nvidia-smi clocks and throttle reasons, sampled every interval_ms (200 ms
+    by default; short timed regions ask for a shorter interval)."""
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
-    def __init__(self, gpu_index: int):
+    def __init__(self, gpu_index: int, interval_ms: int = 200):
         self.gpu = gpu_index
+        self.interval_ms = interval_ms
         self.proc = None
         self.lines = []
         self.thread = None
 
     def start(self):
+        """Start sampling and wait (3 s at most) for the first sample, so that
+        the timed region that follows is covered from its start."""
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+                 "-lms", str(self.interval_ms)], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
         except OSError:
             self.proc = None
             return
         self.thread = threading.Thread(target=self._read, daemon=True)
         self.thread.start()
+        t_end = time.time() + 3.0
+        while not self.lines and time.time() < t_end and self.proc.poll() is None:
+            time.sleep(0.01)
 
     def _read(self):
         for line in self.proc.stdout:
@@ -346,7 +353,7 @@ def run_decode(args, w, rank, world, dev):
     for s in range(warm):
         step(s)
     torch.cuda.synchronize()
-    clocks = ClockSampler(local_rank())
+    clocks = ClockSampler(local_rank(), interval_ms=20)   # the timed region lasts ~20 ms
     clocks.start()
     launches0 = lsa.lsa_launch_count()
     e0.record()
