@@ -125,6 +125,22 @@ def _ptr(t):
     return C.c_void_p(t.data_ptr())
 
 
+def _same_dtype(*ts):
+    """Q, K, V and O share one element type (float32 or bfloat16)."""
+    dt = ts[0].dtype
+    dtype_code(ts[0])
+    for t in ts[1:]:
+        if t is not None and t.dtype != dt:
+            raise ValueError(f"Q, K, V and O must share one dtype, got {dt} and {t.dtype}")
+
+
+def _typed(t, dtype, name):
+    """_ptr after checking the element type the C call expects."""
+    if t is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    return _ptr(t)
+
+
 def dtype_code(t: torch.Tensor) -> int:
     if t.dtype == torch.float32:
         return LSA_F32
@@ -197,9 +213,16 @@ def make_select_params(hq, beam, topk, sink, window) -> SelectParams:
     return s
 
 
+def _check_keys(params: BuildParams, K: torch.Tensor):
+    if dtype_code(K) != params.dtype:
+        raise ValueError(f"K is {K.dtype} but the build parameters say dtype {params.dtype}")
+
+
 def lsa_build_index(params: BuildParams, K: torch.Tensor, W: torch.Tensor, stream=None) -> Index:
     h = C.c_void_p()
-    _ok(lib().lsa_build_index(C.byref(params), _ptr(K), _ptr(W), _stream(stream), C.byref(h)), "lsa_build_index")
+    _check_keys(params, K)
+    _ok(lib().lsa_build_index(C.byref(params), _ptr(K), _typed(W, torch.float32, "W"), _stream(stream), C.byref(h)),
+        "lsa_build_index")
     return Index(h, params)
 
 
@@ -208,8 +231,13 @@ def lsa_build_index_from_tree(params: BuildParams, K, W, leaf_of_block, parents,
     L = params.levels
     par = (C.c_void_p * L)(*([None] + [C.c_void_p(parents[l].data_ptr()) for l in range(1, L)]))
     cen = (C.c_void_p * L)(*[C.c_void_p(centroids[l].data_ptr()) for l in range(L)])
-    for t in list(parents[1:]) + list(centroids) + [leaf_of_block]:
-        _ptr(t)
+    _check_keys(params, K)
+    for t in parents[1:]:
+        _typed(t, torch.int32, "parents")
+    for t in centroids:
+        _typed(t, torch.float32, "centroids")
+    _typed(leaf_of_block, torch.int32, "leaf_of_block")
+    _typed(W, torch.float32, "W")
     h = C.c_void_p()
     _ok(lib().lsa_build_index_from_tree(C.byref(params), _ptr(K), _ptr(W), _ptr(leaf_of_block), par, cen,
                                         _stream(stream), C.byref(h)), "lsa_build_index_from_tree")
@@ -226,8 +254,10 @@ def _select(fn, name, index, sp, Q, q_pos=None, q_pos0=0, idx=None, cnt=None, ma
         idx = torch.empty((B, nq, p.hkv, max_sel), dtype=torch.int32, device=Q.device)
     if cnt is None:
         cnt = torch.empty((B, nq, p.hkv), dtype=torch.int32, device=Q.device)
-    st = fn(index.handle, C.byref(sp), _ptr(Q), int(nq), _ptr(q_pos), int(q_pos0), _ptr(idx), _ptr(cnt),
-            int(max_sel), _stream(stream))
+    if dtype_code(Q) != p.dtype:
+        raise ValueError(f"Q is {Q.dtype} but the index was built for dtype {p.dtype}")
+    st = fn(index.handle, C.byref(sp), _ptr(Q), int(nq), _typed(q_pos, torch.int64, "q_pos"), int(q_pos0),
+            _typed(idx, torch.int32, "idx"), _typed(cnt, torch.int32, "cnt"), int(max_sel), _stream(stream))
     _ok(st, name)
     return idx, cnt
 
@@ -248,8 +278,9 @@ def lsa_select_noalloc(index, sp, Q, idx, cnt, q_pos=None, q_pos0=0, stream=None
     if need > LSA_SELECT_NOALLOC_MAX_FLOATS:
         raise ValueError(f"lsa_select_noalloc: {need} latent-query floats exceed the fixed buffer of "
                          f"{LSA_SELECT_NOALLOC_MAX_FLOATS}; select in smaller query chunks")
-    st = lib().lsa_select_noalloc(index.handle, C.byref(sp), _ptr(Q), int(Q.shape[1]), _ptr(q_pos), int(q_pos0),
-                                  _ptr(idx), _ptr(cnt), int(idx.shape[-1]), _stream(stream))
+    st = lib().lsa_select_noalloc(index.handle, C.byref(sp), _ptr(Q), int(Q.shape[1]),
+                                  _typed(q_pos, torch.int64, "q_pos"), int(q_pos0), _typed(idx, torch.int32, "idx"),
+                                  _typed(cnt, torch.int32, "cnt"), int(idx.shape[-1]), _stream(stream))
     _ok(st, "lsa_select_noalloc")
     return idx, cnt
 
@@ -279,9 +310,11 @@ def lsa_sparse_attn(Q, K, V, idx, cnt, hkv, O=None, lse=None, want_lse=True, str
         O = torch.empty_like(Q)
     if lse is None and want_lse:
         lse = torch.empty((B, nq, hq), dtype=torch.float32, device=Q.device)
-    st = lib().lsa_sparse_attn(_ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(cnt), int(B), int(nq), int(hq), int(hkv),
-                               int(d), dtype_code(Q), int(max_sel), int(ld_tokens), _ptr(O), _ptr(lse),
-                               _stream(stream))
+    _same_dtype(Q, K, V, O)
+    st = lib().lsa_sparse_attn(_ptr(Q), _ptr(K), _ptr(V), _typed(idx, torch.int32, "idx"),
+                               _typed(cnt, torch.int32, "cnt"), int(B), int(nq), int(hq), int(hkv),
+                               int(d), dtype_code(Q), int(max_sel), int(ld_tokens), _ptr(O),
+                               _typed(lse, torch.float32, "lse"), _stream(stream))
     _ok(st, "lsa_sparse_attn")
     return O, lse
 
@@ -295,9 +328,12 @@ def lsa_sparse_attn_banded(Q, K, V, idx, cnt, hkv, sink, window, q_pos0=0, O=Non
         O = torch.empty_like(Q)
     if lse is None and want_lse:
         lse = torch.empty((B, nq, hq), dtype=torch.float32, device=Q.device)
-    st = lib().lsa_sparse_attn_banded(_ptr(Q), _ptr(K), _ptr(V), _ptr(idx), _ptr(cnt), int(B), int(nq), int(q_pos0),
+    _same_dtype(Q, K, V, O)
+    st = lib().lsa_sparse_attn_banded(_ptr(Q), _ptr(K), _ptr(V), _typed(idx, torch.int32, "idx"),
+                                      _typed(cnt, torch.int32, "cnt"), int(B), int(nq), int(q_pos0),
                                       int(hq), int(hkv), int(d), dtype_code(Q), int(max_sel), int(ld_tokens),
-                                      int(sink), int(window), _ptr(O), _ptr(lse), _stream(stream))
+                                      int(sink), int(window), _ptr(O), _typed(lse, torch.float32, "lse"),
+                                      _stream(stream))
     _ok(st, "lsa_sparse_attn_banded")
     return O, lse
 

@@ -70,3 +70,21 @@ def test_binding_rejects_host_tensors():
     import torch
     with pytest.raises(ValueError):
         lsa._ptr(torch.zeros(4))
+
+
+def test_binding_checks_element_types_before_the_call():
+    """The binding refuses tensors of the wrong element type (the C ABI takes
+    untyped pointers) before anything reaches the library."""
+    import torch
+    with pytest.raises(ValueError, match="idx must be torch.int32"):
+        lsa._typed(torch.zeros(4, dtype=torch.int64), torch.int32, "idx")
+    assert lsa._typed(None, torch.int32, "idx") is None
+    q = torch.zeros(1, 2, 4, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="share one dtype"):
+        lsa._same_dtype(q, q.float(), q, None)
+    with pytest.raises(ValueError, match="unsupported dtype"):
+        lsa._same_dtype(q.half(), q.half(), q.half(), None)
+    lsa._same_dtype(q, q, q, None)
+    bp = lsa.make_build_params(1, 8, 8, 1, 64, 16, 1, lsa.LSA_BF16, (2, 4), 1, 0, 0, 0)
+    with pytest.raises(ValueError, match="build parameters"):
+        lsa.lsa_build_index(bp, torch.zeros(1, 8, 1, 64, dtype=torch.float32), torch.zeros(64, 16))
