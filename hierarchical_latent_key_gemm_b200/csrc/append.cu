@@ -1,6 +1,8 @@
-// Decode append ("each new token attends back over the whole history", LSA
-// explainer, "Prefill, decode and training"; decode is the response phase of
-// "Prompt processing is not response generation").
+// Decode append.  In decode every generated token's query looks at the whole
+// history, so the index must keep up with the tokens that decode adds (LSA
+// explainer, section "Prefill, decode and training"; the decode phase is the
+// subject of the 72.4x report's section "Prompt processing is not response
+// generation").
 //
 // Every block that the new tokens complete is pooled and mapped exactly as in
 // the build (same arithmetic order, so identical bits), placed in its nearest

@@ -1,7 +1,7 @@
-// Exact softmax attention over the selected tokens ("the attention kernel is
-// unchanged. LSA only decides which keys it reads", LSA explainer, "How does
-// LSA work?" step 3; "Sparse attention, exact over subset", tree-search wiki
-// note, flowchart).
+// Exact softmax attention over the selected tokens.  LSA changes only which
+// keys attention reads; the attention itself is ordinary exact softmax over
+// that subset (LSA explainer, "How does LSA work?" step 3; tree-search wiki
+// note, flowchart, the sparse-attention node).
 //
 // One CTA per (query, KV head): the G query heads of the group share the
 // selected row list, so every gathered K/V row is read once for all G heads.

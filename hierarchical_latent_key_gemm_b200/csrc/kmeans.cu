@@ -1,6 +1,6 @@
-// Lloyd k-means for the bucket hierarchy ("first groups keys into clusters",
-// 10M-token attention post; "clustered into buckets ... organized as a
-// hierarchy", LSA explainer, "How does LSA work?" step 1).
+// Lloyd k-means for the bucket hierarchy: the keys are grouped into clusters
+// before any query is scored (10M-token attention post), and the buckets form
+// a hierarchy (LSA explainer, "How does LSA work?" step 1).
 //
 // Rules: centroid j starts at point floor(j*n/k); assign = argmin squared
 // distance with ties to the lower centroid id; update = mean of the members,

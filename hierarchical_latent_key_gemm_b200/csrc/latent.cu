@@ -1,8 +1,8 @@
 // Latent keys and latent queries.
 //
 // Keys: Kl[b] = W^T * mean(K[bP .. bP+P-1]) for every complete block of P
-// keys ("Keys are pooled and clustered into buckets in a learned latent
-// space", LSA explainer, section "How does LSA work?", step 1).
+// keys: blocks of keys are averaged, then clustered in a learned low-rank
+// space (LSA explainer, section "How does LSA work?", step 1).
 // Queries: qbar = mean over a KV head's query heads of W^T q (the group shares
 // one selection).
 //

@@ -1,6 +1,6 @@
 // Training-free latent map: W = the r leading principal directions of the
-// pooled keys (LSA explainer, "How does LSA work?": among the D-LSA options,
-// "a training-free option that uses a PCA map").
+// pooled keys (LSA explainer, "How does LSA work?": one of the D-LSA options
+// needs no training and takes its map from a PCA).
 //
 // Pooled keys of every (sequence, KV head) form one sample; their covariance
 // (centred, divided by the count) is accumulated in fp64 and diagonalised by a

@@ -1,14 +1,14 @@
 // Key selection: tree search and the full-scan baseline.
 //
-// Tree search ("a query scores cluster centroids and descends into the best
-// few buckets", tree-search wiki note, TL;DR; "scores the clusters, and then
-// scores the keys within the selected clusters", 10M-token attention post;
-// LSA explainer, "How does LSA work?" steps 2-3): per (query, KV head), level
+// Tree search (tree-search wiki note, TL;DR: the query compares itself with
+// the cluster centroids and goes down into a few of the best buckets;
+// 10M-token attention post: clusters are scored first, then the keys inside
+// the chosen ones; LSA explainer, "How does LSA work?" steps 2-3): per (query, KV head), level
 // by level, score the eligible nodes (all top nodes, then the children of the
 // kept ones) and keep the best `beam`; score the candidate blocks inside the
 // kept leaves and keep the best ceil(K/P); emit sink + blocks + window.
 //
-// Full scan (the "old indexer" of the wiki note's flowchart): the same top-K
+// Full scan (the previous indexer, the wiki note's flowchart, red path): the same top-K
 // over every candidate block, no tree.
 //
 // One CTA per (query, KV head).  Every tree level is stored in tree order
@@ -749,10 +749,12 @@ int launch_select_t(const SelArgs& a, int64_t nq, int64_t units, bool fullscan, 
         // ask for no more shared memory than the resident CTAs need (each also
         // holds 1 KB for the system): the rest of the SM's 256 KB stays L1,
         // which keeps the upper tree levels that every query scores
+        // (a hint: the percentage is clamped to 100, and a refusal leaves the
+        // driver's own choice, which is correct, only slower)
         const int per = (int)(smem + sizeof(SelShared) + 1024);
-        const int pct = (LSA_SELECT_MIN_BLOCKS * per * 100 + 233471) / 233472;
-        cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, pct);
-        cudaGetLastError();
+        const int pct = min(100, (LSA_SELECT_MIN_BLOCKS * per * 100 + 233471) / 233472);
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, pct);
+        if (e != cudaSuccess) return cuda_status(e);
     }
     dim3 grid((unsigned)nq, (unsigned)units);
     note_launch();

@@ -44,14 +44,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         "l"(reinterpret_cast<uint64_t>(map)), "r"(su32(bar)), "r"(x), "r"(y)
         : "memory");
 }
-__device__ __forceinline__ void tma_gather4(void* dst, const CUtensorMap* map, uint64_t* bar, int x, int y0, int y1,
-                                            int y2, int y3) {
-    asm volatile(
-        "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes [%0], [%1, {%3, "
-        "%4, %5, %6, %7}], [%2];" ::"r"(su32(dst)),
-        "l"(reinterpret_cast<uint64_t>(map)), "r"(su32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
-        : "memory");
-}
 
 // Host: the driver's tensor-map encoder (through the runtime's entry-point
 // query, so the library does not link libcuda), and a 2D map with 128-byte

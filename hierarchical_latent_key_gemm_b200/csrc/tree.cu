@@ -1,7 +1,7 @@
 // Bucket layout of a built tree.
 //
-// Leaves store their blocks contiguously ("descends into the best few
-// buckets", tree-search wiki note, TL;DR): slots [leaf_start, leaf_start +
+// Leaves store their blocks contiguously (a query reads whole buckets once
+// it has descended into them, tree-search wiki note, TL;DR): slots [leaf_start, leaf_start +
 // leaf_cnt) hold the member blocks in ascending block order, followed by
 // free slots that decode appends fill.  The latent keys are copied into the
 // same order (Klp), so scoring a bucket reads one contiguous run.  Child

@@ -244,18 +244,40 @@ def lsa_build_index_from_tree(params: BuildParams, K, W, leaf_of_block, parents,
     return Index(h, params)
 
 
+def _shape(t, want, name):
+    if t is not None and tuple(t.shape) != tuple(int(x) for x in want):
+        raise ValueError(f"{name} must have shape {tuple(int(x) for x in want)}, got {tuple(t.shape)}")
+
+
+def _check_select_args(p, sp, Q, q_pos, idx, cnt, max_sel):
+    """The C ABI takes untyped pointers and cannot see sizes: every buffer's
+    element type and shape is checked here, before anything is enqueued, so a
+    wrong tensor is an error and never an out-of-bounds device access."""
+    if Q.dim() != 4:
+        raise ValueError(f"Q must be [batch, nq, hq, d], got shape {tuple(Q.shape)}")
+    if dtype_code(Q) != p.dtype:
+        raise ValueError(f"Q is {Q.dtype} but the index was built for dtype {p.dtype}")
+    nq = Q.shape[1]
+    _shape(Q, (p.batch, nq, sp.hq, p.d), "Q")
+    _shape(q_pos, (p.batch, nq), "q_pos")
+    _shape(idx, (p.batch, nq, p.hkv, max_sel), "idx")
+    _shape(cnt, (p.batch, nq, p.hkv), "cnt")
+    for t, dt, nm in ((q_pos, torch.int64, "q_pos"), (idx, torch.int32, "idx"), (cnt, torch.int32, "cnt")):
+        if t is not None and t.dtype != dt:
+            raise ValueError(f"{nm} must be {dt}, got {t.dtype}")
+
+
 def _select(fn, name, index, sp, Q, q_pos=None, q_pos0=0, idx=None, cnt=None, max_sel=None, stream=None):
     p = index.params
     B, nq = Q.shape[0], Q.shape[1]
     kb = -(-sp.topk // p.pool)
     if max_sel is None:
-        max_sel = kb * p.pool + p.sink + sp.window
+        max_sel = idx.shape[-1] if idx is not None else kb * p.pool + p.sink + sp.window
+    _check_select_args(p, sp, Q, q_pos, idx, cnt, max_sel)
     if idx is None:
         idx = torch.empty((B, nq, p.hkv, max_sel), dtype=torch.int32, device=Q.device)
     if cnt is None:
         cnt = torch.empty((B, nq, p.hkv), dtype=torch.int32, device=Q.device)
-    if dtype_code(Q) != p.dtype:
-        raise ValueError(f"Q is {Q.dtype} but the index was built for dtype {p.dtype}")
     st = fn(index.handle, C.byref(sp), _ptr(Q), int(nq), _typed(q_pos, torch.int64, "q_pos"), int(q_pos0),
             _typed(idx, torch.int32, "idx"), _typed(cnt, torch.int32, "cnt"), int(max_sel), _stream(stream))
     _ok(st, name)
@@ -274,7 +296,8 @@ def lsa_select_noalloc(index, sp, Q, idx, cnt, q_pos=None, q_pos0=0, stream=None
     queries use the library's fixed 4 MiB device buffer (see include/lsa.h).
     batch * nq * hkv * r must not exceed LSA_SELECT_NOALLOC_MAX_FLOATS."""
     p = index.params
-    need = Q.shape[0] * Q.shape[1] * p.hkv * p.r
+    _check_select_args(p, sp, Q, q_pos, idx, cnt, idx.shape[-1])
+    need = p.batch * Q.shape[1] * p.hkv * p.r
     if need > LSA_SELECT_NOALLOC_MAX_FLOATS:
         raise ValueError(f"lsa_select_noalloc: {need} latent-query floats exceed the fixed buffer of "
                          f"{LSA_SELECT_NOALLOC_MAX_FLOATS}; select in smaller query chunks")
@@ -302,7 +325,27 @@ def lsa_fullscan_select(index, sp, Q, **kw):
     return _select(lib().lsa_fullscan_select, "lsa_fullscan_select", index, sp, Q, **kw)
 
 
+def _check_attn_args(Q, K, V, idx, cnt, hkv, O, lse):
+    """Shapes and element types of an attention call (see _check_select_args)."""
+    if Q.dim() != 4 or K.dim() != 4:
+        raise ValueError("Q must be [batch, nq, hq, d] and K, V [batch, ld_tokens, hkv, d]")
+    B, nq, hq, d = Q.shape
+    _shape(K, (B, K.shape[1], hkv, d), "K")
+    _shape(V, tuple(K.shape), "V")
+    if idx.dim() != 4:
+        raise ValueError(f"idx must be [batch, nq, hkv, max_sel], got shape {tuple(idx.shape)}")
+    _shape(idx, (B, nq, hkv, idx.shape[-1]), "idx")
+    _shape(cnt, (B, nq, hkv), "cnt")
+    _shape(O, tuple(Q.shape), "O")
+    _shape(lse, (B, nq, hq), "lse")
+    _same_dtype(Q, K, V, O)
+    for t, dt, nm in ((idx, torch.int32, "idx"), (cnt, torch.int32, "cnt"), (lse, torch.float32, "lse")):
+        if t is not None and t.dtype != dt:
+            raise ValueError(f"{nm} must be {dt}, got {t.dtype}")
+
+
 def lsa_sparse_attn(Q, K, V, idx, cnt, hkv, O=None, lse=None, want_lse=True, stream=None):
+    _check_attn_args(Q, K, V, idx, cnt, hkv, O, lse)
     B, nq, hq, d = Q.shape
     ld_tokens = K.shape[1]
     max_sel = idx.shape[-1]
@@ -310,7 +353,6 @@ def lsa_sparse_attn(Q, K, V, idx, cnt, hkv, O=None, lse=None, want_lse=True, str
         O = torch.empty_like(Q)
     if lse is None and want_lse:
         lse = torch.empty((B, nq, hq), dtype=torch.float32, device=Q.device)
-    _same_dtype(Q, K, V, O)
     st = lib().lsa_sparse_attn(_ptr(Q), _ptr(K), _ptr(V), _typed(idx, torch.int32, "idx"),
                                _typed(cnt, torch.int32, "cnt"), int(B), int(nq), int(hq), int(hkv),
                                int(d), dtype_code(Q), int(max_sel), int(ld_tokens), _ptr(O),
@@ -321,6 +363,7 @@ def lsa_sparse_attn(Q, K, V, idx, cnt, hkv, O=None, lse=None, want_lse=True, str
 
 def lsa_sparse_attn_banded(Q, K, V, idx, cnt, hkv, sink, window, q_pos0=0, O=None, lse=None, want_lse=True,
                            stream=None):
+    _check_attn_args(Q, K, V, idx, cnt, hkv, O, lse)
     B, nq, hq, d = Q.shape
     ld_tokens = K.shape[1]
     max_sel = idx.shape[-1]
@@ -328,7 +371,6 @@ def lsa_sparse_attn_banded(Q, K, V, idx, cnt, hkv, sink, window, q_pos0=0, O=Non
         O = torch.empty_like(Q)
     if lse is None and want_lse:
         lse = torch.empty((B, nq, hq), dtype=torch.float32, device=Q.device)
-    _same_dtype(Q, K, V, O)
     st = lib().lsa_sparse_attn_banded(_ptr(Q), _ptr(K), _ptr(V), _typed(idx, torch.int32, "idx"),
                                       _typed(cnt, torch.int32, "cnt"), int(B), int(nq), int(q_pos0),
                                       int(hq), int(hkv), int(d), dtype_code(Q), int(max_sel), int(ld_tokens),

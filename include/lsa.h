@@ -125,7 +125,7 @@ typedef enum {
  * block; Lloyd k-means of the latent keys into level_sizes[levels-1] leaves
  * (centroid j starts at point floor(j*n/k); ties to the lower id; an empty
  * cluster keeps its centroid); then k-means of each level's centroids into
- * the level above.  [p1 "first groups keys into clusters"; p5 step 1; p2]
+ * the level above.  [p1: keys are clustered before any query is scored; p5 step 1; p2]
  * On success *out receives a new index owned by the caller (lsa_free_index).
  * On failure *out is set to NULL and no device memory is left allocated.
  * The build is enqueued on `stream`; lsa_check() reports device-side errors. */
@@ -223,7 +223,7 @@ int lsa_pca_map(const void* K, int64_t batch, int64_t n_tokens, int64_t ld_token
 
 /* The quadratic baseline indexer: every candidate block is scored, no tree.
  * Same arguments and output format as lsa_select (beam is ignored).
- * [p3 flowchart, red path "Full key scan"] */
+ * [p3 flowchart, red path: the full key scan] */
 int lsa_fullscan_select(const lsa_index* index, const lsa_select_params* params, const void* Q,
                         int64_t nq, const int64_t* q_pos, int64_t q_pos0,
                         int32_t* idx, int32_t* cnt, int32_t max_sel, void* stream);
@@ -237,8 +237,8 @@ int lsa_fullscan_select(const lsa_index* index, const lsa_select_params* params,
  * h / (hq/hkv); fp32 accumulation.  A row with cnt = 0 yields O = 0 and
  * lse = -inf.  An index outside [0, ld_tokens) is skipped and latched as
  * LSA_ERR_DEVICE.  For bf16, Q, K, V and O must be 16-byte aligned (else
- * LSA_ERR_INVALID_ARG).  [p5 step 3 "the attention kernel is unchanged"; p3
- * flowchart "exact over subset"] */
+ * LSA_ERR_INVALID_ARG).  [p5 step 3: LSA leaves the attention itself as it
+ * was; p3 flowchart: exact attention over the subset] */
 int lsa_sparse_attn(const void* Q, const void* K, const void* V, const int32_t* idx,
                     const int32_t* cnt, int64_t batch, int64_t nq, int32_t hq, int32_t hkv,
                     int32_t d, int32_t dtype, int32_t max_sel, int64_t ld_tokens,

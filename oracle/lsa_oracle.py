@@ -33,11 +33,11 @@ space, organised as a hierarchy [p5 step 1; p2; p4]; a query scores the bucket
 centroids, descends into the best few buckets and scores the keys inside them
 [p1; p3 TL;DR; p5 step 2]; the query then attends exactly to the selected
 long-range keys plus the attention sink and a local window, with an unchanged
-attention kernel [p5 step 3; p3 flowchart "exact over subset"].  The old
+attention kernel [p5 step 3; p3 flowchart, the sparse-attention node].  The old
 indexer scores every key [p3 flowchart, red path].  Decode attends each new
 token over the whole history [p5 "Prefill, decode and training"].
 
-Readings where the pages are silent (each one is also listed in the design doc):
+Readings where the pages are silent:
   R1  one latent map W (d x r) serves keys and queries.
   R2  scores are unscaled inner products in latent space; k-means uses squared
       Euclidean distance.
@@ -135,8 +135,8 @@ def query_latent(Qg: np.ndarray, W: np.ndarray) -> np.ndarray:
 
 
 # ---------------------------------------------------------------------------
-# Lloyd k-means  [p1: "first groups keys into clusters"; p5 step 1: "clustered
-# into buckets"]
+# Lloyd k-means  [p1: keys are grouped into clusters first; p5 step 1: the
+# clusters are the buckets]
 # ---------------------------------------------------------------------------
 def squared_distances(X: np.ndarray, C: np.ndarray) -> np.ndarray:
     """||x - c||^2 for every (point, centroid) pair, [n, k].  Uses the exact
@@ -229,9 +229,8 @@ def kmeans(X: np.ndarray, k: int, iters: int, grid_log2: int = 0) -> KMeansResul
 
 
 # ---------------------------------------------------------------------------
-# The bucket hierarchy  [p2: "hierarchical tree variant"; p3 TL;DR: "clusters
-# keys hierarchically"; p4: "a hierarchy of clusters"; p5 step 1: "organized as
-# a hierarchy"]
+# The bucket hierarchy  [p2: the tree form of the index; p3 TL;DR: keys are
+# clustered level by level; p4 and p5 step 1: the clusters form a hierarchy]
 # ---------------------------------------------------------------------------
 @dataclass
 class Tree:
@@ -312,10 +311,10 @@ def build_tree(Kl: np.ndarray, level_sizes, iters: int, grid_log2: int,
 
 
 # ---------------------------------------------------------------------------
-# Selection  [p3 TL;DR: "a query scores cluster centroids and descends into the
-# best few buckets"; p1: "scores the clusters, and then scores the keys within
-# the selected clusters"; p5 step 3: "selected long-range keys plus the
-# attention sink and a local window"]
+# Selection  [p3 TL;DR: the query scores centroids and goes down into a few of
+# the best buckets; p1: clusters are scored first, then the keys inside the
+# chosen ones; p5 step 3: the chosen far-away keys join the attention sink and
+# a local window]
 # ---------------------------------------------------------------------------
 def top_by_score(ids: np.ndarray, scores: np.ndarray, k: int) -> np.ndarray:
     """The k ids with the highest scores; equal scores go to the lower id (R7)."""
@@ -394,8 +393,8 @@ def selection_tokens(blocks: np.ndarray, i: int, sink: int, window: int, pool: i
 
 
 # ---------------------------------------------------------------------------
-# Exact attention over the selected set  [p5 step 3: "the attention kernel is
-# unchanged"; p3 flowchart: "Sparse attention, exact over subset"]
+# Exact attention over the selected set  [p5 step 3: LSA leaves the attention
+# itself as it was; p3 flowchart: exact attention over the subset]
 # ---------------------------------------------------------------------------
 def sparse_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, sel: np.ndarray):
     """softmax(q . k_j / sqrt(d)) weighted sum of v_j over j in ``sel``.

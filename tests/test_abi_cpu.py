@@ -88,3 +88,66 @@ def test_binding_checks_element_types_before_the_call():
     bp = lsa.make_build_params(1, 8, 8, 1, 64, 16, 1, lsa.LSA_BF16, (2, 4), 1, 0, 0, 0)
     with pytest.raises(ValueError, match="build parameters"):
         lsa.lsa_build_index(bp, torch.zeros(1, 8, 1, 64, dtype=torch.float32), torch.zeros(64, 16))
+
+
+def test_binding_checks_shapes_before_the_call():
+    """The C ABI cannot see buffer sizes, so the binding checks every shape
+    against the index and the call's parameters before the library is called:
+    a mismatched tensor raises instead of reaching a kernel as an
+    out-of-bounds read or write.  (Host tensors: each case must fail on its
+    shape, before the device-pointer check.)"""
+    import torch
+    bp = lsa.make_build_params(1, 64, 64, 2, 64, 16, 1, lsa.LSA_BF16, (2, 4), 1, 0, 0, 0)
+    ix = lsa.Index(C.c_void_p(None), bp)
+    sp = lsa.make_select_params(4, 2, 8, 0, 4)
+    bf = torch.bfloat16
+    Q = torch.zeros(1, 8, 4, 64, dtype=bf)
+    ms = 8 + 0 + 4
+    idx = torch.zeros(1, 8, 2, ms, dtype=torch.int32)
+    cnt = torch.zeros(1, 8, 2, dtype=torch.int32)
+    cases = [
+        (dict(Q=torch.zeros(1, 8, 3, 64, dtype=bf)), "Q must have shape"),
+        (dict(Q=torch.zeros(2, 8, 4, 64, dtype=bf)), "Q must have shape"),
+        (dict(Q=torch.zeros(1, 8, 4, 128, dtype=bf)), "Q must have shape"),
+        (dict(Q=Q.float()), "built for dtype"),
+        (dict(idx=torch.zeros(1, 7, 2, ms, dtype=torch.int32)), "idx must have shape"),
+        (dict(idx=torch.zeros(1, 8, 1, ms, dtype=torch.int32)), "idx must have shape"),
+        (dict(cnt=torch.zeros(1, 8, 1, dtype=torch.int32)), "cnt must have shape"),
+        (dict(cnt=torch.zeros(1, 8, 2, dtype=torch.int64)), "cnt must be"),
+        (dict(q_pos=torch.zeros(1, 9, dtype=torch.int64)), "q_pos must have shape"),
+        (dict(q_pos=torch.zeros(1, 8, dtype=torch.int32)), "q_pos must be"),
+    ]
+    for over, msg in cases:
+        a = dict(Q=Q, idx=idx, cnt=cnt, q_pos=None)
+        a.update(over)
+        with pytest.raises(ValueError, match=msg):
+            lsa.lsa_select(ix, sp, a["Q"], idx=a["idx"], cnt=a["cnt"], q_pos=a["q_pos"])
+        with pytest.raises(ValueError, match=msg):
+            lsa.lsa_select_noalloc(ix, sp, a["Q"], a["idx"], a["cnt"], q_pos=a["q_pos"])
+    # well-formed host tensors get past the shape checks and stop at the
+    # device-pointer check
+    with pytest.raises(ValueError, match="CUDA device"):
+        lsa.lsa_select(ix, sp, Q, idx=idx, cnt=cnt)
+    # attention
+    K = torch.zeros(1, 64, 2, 64, dtype=bf)
+    O = torch.zeros_like(Q)
+    lse = torch.zeros(1, 8, 4)
+    att = [
+        (dict(K=torch.zeros(1, 64, 1, 64, dtype=bf)), "K must have shape"),
+        (dict(V=torch.zeros(1, 63, 2, 64, dtype=bf)), "V must have shape"),
+        (dict(idx=torch.zeros(1, 8, 1, ms, dtype=torch.int32)), "idx must have shape"),
+        (dict(cnt=torch.zeros(1, 7, 2, dtype=torch.int32)), "cnt must have shape"),
+        (dict(O=torch.zeros(1, 8, 4, 32, dtype=bf)), "O must have shape"),
+        (dict(lse=torch.zeros(1, 8, 2)), "lse must have shape"),
+        (dict(lse=torch.zeros(1, 8, 4, dtype=torch.float64)), "lse must be"),
+        (dict(V=K.float()), "share one dtype"),
+    ]
+    for over, msg in att:
+        a = dict(Q=Q, K=K, V=K, idx=idx, cnt=cnt, O=O, lse=lse)
+        a.update(over)
+        for fn in (lambda a: lsa.lsa_sparse_attn(a["Q"], a["K"], a["V"], a["idx"], a["cnt"], 2, O=a["O"],
+                                                 lse=a["lse"]),
+                   lambda a: lsa.lsa_sparse_attn_banded(a["Q"], a["K"], a["V"], a["idx"], a["cnt"], 2, 0, 4,
+                                                        O=a["O"], lse=a["lse"])):
+            with pytest.raises(ValueError, match=msg):
+                fn(a)

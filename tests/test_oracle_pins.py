@@ -159,6 +159,45 @@ def test_tree_partition_and_minpos_brute_force():
             np.testing.assert_allclose(t.centroids[1][j], Kl[mem].mean(axis=0), atol=1e-12)
 
 
+def _minpos_list(v):
+    return np.array([math.inf if x == "inf" else float(x) for x in v])
+
+
+@pytest.mark.parametrize("case", gold("tree_small.json")["builds"])
+def test_build_tree_upper_levels_worked_examples(case):
+    """Hand-worked two-level builds: the leaf clustering, then the clustering
+    of the leaf centroids (unweighted, stride init over the leaf ids), the
+    parents, the centroids and objectives of both levels, and minpos."""
+    X = np.array(case["latents"], dtype=np.float64)[:, None]
+    t = O.build_tree(X, case["level_sizes"], case["iters"], 0, case["sink"], case["pool"])
+    np.testing.assert_array_equal(t.leaf_of_block, case["leaf_of_block"])
+    np.testing.assert_array_equal(t.centroids[1][:, 0], case["leaf_centroids"])
+    np.testing.assert_array_equal(t.objectives[1], case["leaf_objectives"])
+    np.testing.assert_array_equal(t.parent[1], case["parent_of_leaf"])
+    np.testing.assert_array_equal(t.centroids[0][:, 0], case["top_centroids"])
+    np.testing.assert_array_equal(t.objectives[0], case["top_objectives"])
+    np.testing.assert_array_equal(t.minpos[1], _minpos_list(case["minpos_leaf"]))
+    np.testing.assert_array_equal(t.minpos[0], _minpos_list(case["minpos_top"]))
+
+
+@pytest.mark.parametrize("case", gold("tree_small.json")["minpos_trees"])
+def test_minpos_worked_examples(case):
+    """minpos on given trees: blocks before the sink and empty leaves count as
+    +inf, and each upper node takes the minimum over its children."""
+    L = len(case["level_sizes"])
+    parent = [None] * L
+    parent[L - 1] = np.array(case["parent_of_leaf"])
+    if L == 3:
+        parent[1] = np.array(case["parent_of_mid"])
+    cents = [np.zeros((n, 1)) for n in case["level_sizes"]]
+    t = O.Tree(case["pool"], case["sink"], case["level_sizes"], cents, parent, np.array(case["leaf_of_block"]),
+               [[]] * L).finish()
+    np.testing.assert_array_equal(t.minpos[L - 1], _minpos_list(case["minpos_leaf"]))
+    np.testing.assert_array_equal(t.minpos[0], _minpos_list(case["minpos_top"]))
+    if L == 3:
+        np.testing.assert_array_equal(t.minpos[1], _minpos_list(case["minpos_mid"]))
+
+
 def _tree_from_gold(g):
     tr = g["tree"]
     return O.Tree(tr["pool"], tr["sink"], tr["level_sizes"],

@@ -38,6 +38,25 @@ def test_select_noalloc_matches_select_on_two_calls():
         assert lsa.lsa_check(ix) == lsa.LSA_OK
         assert torch.equal(cnt, ref_cnt)
         assert torch.equal(idx, ref_idx)
+    # it allocates nothing: with the library's next device allocation set to
+    # fail, lsa_select_noalloc still succeeds with the same rows, while
+    # lsa_select (which takes its scratch from the pool) reports the failure
+    Qc = Q[:, 1000:1000 + nq].contiguous()
+    ref_idx, ref_cnt = lsa.lsa_select(ix, sp, Qc, q_pos0=1000)
+    idx = torch.full_like(ref_idx, -7)
+    cnt = torch.full_like(ref_cnt, -7)
+    lsa.lsa_debug_fail_alloc_after(1)
+    try:
+        st = L.lsa_select_noalloc(ix.handle, C.byref(sp), C.c_void_p(Qc.data_ptr()), nq, None, 1000,
+                                  C.c_void_p(idx.data_ptr()), C.c_void_p(cnt.data_ptr()), idx.shape[-1], stream)
+        assert st == lsa.LSA_OK, lsa.strerror(st)
+        st = L.lsa_select(ix.handle, C.byref(sp), C.c_void_p(Qc.data_ptr()), nq, None, 1000,
+                          C.c_void_p(idx.data_ptr()), C.c_void_p(cnt.data_ptr()), idx.shape[-1], stream)
+        assert st == lsa.LSA_ERR_OOM
+    finally:
+        lsa.lsa_debug_fail_alloc_after(0)
+    assert lsa.lsa_check(ix) == lsa.LSA_OK
+    assert torch.equal(cnt, ref_cnt) and torch.equal(idx, ref_idx)
     # a request beyond the fixed buffer is refused before anything runs
     big = Q[:, :9000].contiguous()  # 9000 x 2 x 64 = 1,152,000 floats
     bidx = torch.empty((1, 9000, w.hkv, w.max_sel), dtype=torch.int32, device="cuda")
