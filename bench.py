@@ -30,6 +30,11 @@ sys.path.insert(0, ROOT)
 
 METRIC = "LSA prefill tokens/s per layer (index+select+attn) at 1M ctx; % of roofline"
 UNIT = "tokens/s"
+# The CPU oracle's bounded sample, the same for the bench's cpu_baseline and
+# for every step of the reference arm: one Lloyd round timed on every 8th
+# block, select + attention on 128 sampled queries.
+CPU_SAMPLE_QUERIES = 128
+CPU_LLOYD_STRIDE = 8
 
 
 def parse_args():
@@ -43,7 +48,7 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
-    ap.add_argument("--cpu-sample-queries", type=int, default=256)
+    ap.add_argument("--cpu-sample-queries", type=int, default=CPU_SAMPLE_QUERIES)
     ap.add_argument("--query-range", default=None,
                     help="START:COUNT - profiling case: full index, select+attention on that query range only")
     return ap.parse_args()
@@ -145,8 +150,9 @@ def measured_peaks() -> dict:
     if os.path.exists(p):
         with open(p) as f:
             d = json.load(f)
-        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"], "source": "measured"}
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
 def kernel_source_sha(fname: str) -> str:
@@ -170,6 +176,15 @@ def recorded_traffic(kernel: str, workload: str, src: str):
             if len(parts) >= 5 and parts[0] == kernel and parts[1] == workload and parts[2] == src:
                 return int(parts[4]) if parts[3] == sha else None
     return None
+
+
+def run_config(w, world: int, seed: int) -> dict:
+    """The workload description both arms print (the reference arm runs the
+    same workload on the host cores of rank 0)."""
+    from hierarchical_latent_key_gemm_b200.workloads import describe
+    return {"workload": describe(w), "global_batch": w.batch * world, "seq_len": w.n_tokens,
+            "parallelism": f"dp{world} (one independent layer instance per GPU)",
+            "l2": "inputs larger than L2 (Q 4 GiB, K and V 0.5 GiB each); no flush needed", "seed": seed}
 
 
 # ------------------------------------------------------------------ our arm
@@ -254,37 +269,27 @@ def run_ours(args):
     attn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
 
     peaks = measured_peaks()
-    stages = {"build_ms": build_ms, "select_ms": select_ms, "attn_ms": attn_ms}
     # Work counts for the rooflines, taken outside the timed region on the
-    # same inputs: the rows select scored, and the selection sizes.
+    # same inputs: the tree nodes and candidate blocks select scored, and the
+    # selection sizes.
     ix = lsa.lsa_build_index(bp, K, W)
-    _, _, scored = lsa.lsa_select_work(ix, sp, Q, idx=idx, cnt=cnt, max_sel=max_sel, q_pos0=q0)
+    _, _, nodes, blocks = lsa.lsa_select_work(ix, sp, Q, idx=idx, cnt=cnt, max_sel=max_sel, q_pos0=q0)
     ix.free()
     torch.cuda.synchronize()
     sel_tokens = int(cnt.sum(dtype=torch.int64).item())
-    # dominant kernel: select_kernel (the select stage = query-latent kernel + select kernel).
-    # Algorithmic bytes = latent rows scored (r fp32 each) + the selection written (4 B per
-    # token) + the queries read once for the latent queries.
-    sel_bytes = scored * w.r * 4 + sel_tokens * 4 + Q.numel() * Q.element_size()
-    achieved = sel_bytes / (select_ms / 1e3) / 1e9
-    roofline = {"bound": "hbm", "kernel": "select_kernel<64, tree>", "achieved": achieved,
-                "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": achieved / peaks["hbm_gbs"],
+    stages = stage_rooflines(w, inp, bp, dev, peaks, build_ms, select_ms, attn_ms, nodes, blocks, sel_tokens,
+                             q0, nq)
+    sel = stages["select"]
+    roofline = {"bound": "hbm", "kernel": "select_kernel<64, tree> (select stage: query latents + select)",
+                "achieved": sel["achieved_GBps"], "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": sel["frac"],
                 "traffic": recorded_traffic("select_kernel<64, tree>", w.name, "select.cu"),
-                "algorithmic_bytes_per_launch": sel_bytes, "rows_scored_per_launch": scored,
-                "peak_source": peaks["source"],
-                "note": ("achieved = (eligible latent rows scored x r x 4 B + selected tokens x 4 B + Q bytes) "
-                         "/ mean select-stage time; the latents (64 MiB per KV head) stay L2-resident, so "
-                         "DRAM traffic (traffic) is far below the algorithmic bytes")}
-    # the attention kernels, for context: gathered K/V bytes and tensor FLOPs
-    attn_bytes = sel_tokens * w.d * 2 * 2
-    attn_flops = sel_tokens * w.d * 4 * w.group
-    stages["attn_gathered_GBps"] = attn_bytes / (attn_ms / 1e3) / 1e9
-    stages["attn_TFLOPs"] = attn_flops / (attn_ms / 1e3) / 1e12
+                "algorithmic_bytes_per_launch": sel["algorithmic_bytes"], "peak_source": peaks["source"],
+                "note": sel["formula"]}
 
     if args.query_range:
         # profiling case: report the stages only
         print(json.dumps({"profile_case": args.query_range, "stages": stages, "gpu_launches_per_step":
-                          launches / args.steps, "select_GBps": achieved}), flush=True)
+                          launches / args.steps}), flush=True)
         return
     e2e = None
     if not args.no_e2e:
@@ -298,17 +303,22 @@ def run_ours(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_oracle_estimate(w, inp, args.cpu_sample_queries)
 
+    # the other workloads, one after another on the same GPU (the prefill
+    # buffers freed first): per-layer and per-step figures
+    others = None
+    if not args.no_extra and rank == 0:
+        del idx, cnt, O, lse, inp, Q, K, V
+        torch.cuda.empty_cache()
+        others = run_other_workloads(dev, peaks)
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": describe(w), "global_batch": w.batch * world, "seq_len": N,
-                       "parallelism": f"dp{world} (one independent layer instance per GPU)",
-                       "l2": "inputs larger than L2 (Q 4 GiB, K and V 0.5 GiB each); no flush needed",
-                       "seed": args.seed},
+            "config": run_config(w, world, args.seed),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": launches,
-            "clocks": clk, "stages": stages, "extra": extra,
+            "clocks": clk, "stages": stages, "extra": extra, "workloads": others,
         }
         print(json.dumps(line), flush=True)
     if world > 1:
@@ -317,13 +327,26 @@ def run_ours(args):
 
 
 def run_decode(args, w, rank, world, dev):
+    """Decode workload as the bench line (see decode_measure)."""
+    from hierarchical_latent_key_gemm_b200.workloads import describe
+    r = decode_measure(w, dev, args.seed + 1000 * rank, args.warmup, world, not args.no_extra and rank == 0)
+    if rank == 0:
+        print(json.dumps({
+            "metric": "LSA decode ms per step (append + select + attention, all sequences) at 10M context",
+            "value": r["ms_per_step"], "unit": "ms/step", "n_gpus": world, "steps": r["steps"],
+            "warmup": r["warmup"], "higher_is_better": False, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic", "config": {"workload": describe(w)}, "build_ms": r["build_ms"],
+            "index_device_bytes": r["index_device_bytes"], "gpu_launches": r["gpu_launches"],
+            "status": r["status"], "clocks": r["clocks"], "extra": r["extra"]}), flush=True)
+
+
+def decode_measure(w, dev, seed, warmup, world=1, extra=True):
     """Decode workload: build the index over every sequence's context (timed
     once), then time decode steps: append the new token's key, select for the
     new query, attend; one step covers all sequences of the batch."""
     import torch
     from hierarchical_latent_key_gemm_b200 import lsa
-    from hierarchical_latent_key_gemm_b200.workloads import describe, make_inputs
-    seed = args.seed + 1000 * rank
+    from hierarchical_latent_key_gemm_b200.workloads import make_inputs
     inp = make_inputs(w, seed=seed, device=dev)
     K, V, Q, W = inp["K"], inp["V"], inp["Q"], inp["W"]
     N = w.n_tokens
@@ -349,7 +372,7 @@ def run_decode(args, w, rank, world, dev):
         lsa.lsa_select(ix, sp, qs[s], q_pos0=N + s, idx=idx, cnt=cnt, max_sel=w.max_sel)
         lsa.lsa_sparse_attn(qs[s], K, V, idx, cnt, w.hkv, O=O, lse=lse)
 
-    warm = min(args.warmup, w.decode_steps // 4)
+    warm = min(warmup, w.decode_steps // 4)
     for s in range(warm):
         step(s)
     torch.cuda.synchronize()
@@ -364,20 +387,16 @@ def run_decode(args, w, rank, world, dev):
     clk = clocks.stop()
     n_timed = w.decode_steps - warm
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / n_timed
+    launches = lsa.lsa_launch_count() - launches0
     st = lsa.lsa_check(ix)
     info = ix.info()
-    extra = None
-    if not args.no_extra and rank == 0:
-        extra = decode_extra(w, inp, ix, sp, dev)
+    ext = decode_extra(w, inp, ix, sp, dev) if extra else None
     ix.free()
-    if rank == 0:
-        print(json.dumps({
-            "metric": "LSA decode ms per step (append + select + attention, all sequences) at 10M context",
-            "value": ms, "unit": "ms/step", "n_gpus": world, "steps": n_timed, "warmup": warm,
-            "higher_is_better": False, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": {"workload": describe(w)}, "build_ms": build_ms,
-            "index_device_bytes": int(info.device_bytes), "gpu_launches": lsa.lsa_launch_count() - launches0,
-            "status": lsa.strerror(st), "clocks": clk, "extra": extra}), flush=True)
+    del inp, idx, cnt, O, lse, qs
+    torch.cuda.empty_cache()
+    return {"ms_per_step": ms, "steps": n_timed, "warmup": warm, "build_ms": build_ms,
+            "index_device_bytes": int(info.device_bytes), "gpu_launches": launches, "status": lsa.strerror(st),
+            "clocks": clk, "extra": ext}
 
 
 def decode_extra(w, inp, ix, sp, dev):
@@ -583,6 +602,229 @@ def run_extra(w, inp, bp, sp, dev, select_ms, idx, cnt):
             "select_queries_per_s": N * w.batch * w.hkv / (select_ms / 1e3)}
 
 
+# ------------------------------------------------------------------ stages
+def time_ms(fn, reps: int = 3) -> float:
+    """Median device time of fn() in ms (CUDA events on the current stream,
+    one untimed call first)."""
+    import torch
+    fn()
+    torch.cuda.synchronize()
+    out = []
+    for _ in range(reps):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        fn()
+        e1.record()
+        torch.cuda.synchronize()
+        out.append(e0.elapsed_time(e1))
+    return statistics.median(out)
+
+
+def stage_rooflines(w, inp, bp, dev, peaks, build_ms, select_ms, attn_ms, nodes, blocks, sel_tokens, q0, nq):
+    """Every stage against its roofline, on the survey's algorithmic work:
+      a1 project + pool   HBM: K read (2 B per element) + latent keys written (r x 4 B per block)
+      a5 query latent     HBM: Q read + latent queries written (r x 4 B per (query, KV head))
+      a2 leaf k-means     tensor (bf16 dense peak): 2 x blocks x leaves x r flops per round
+      select (a5-a8)      HBM: a5 + tree nodes scored x r x 2 B (a6) + candidate blocks scored
+                          x r x 2 B (a7) + selected tokens x 4 B (a8)
+      attention (a9)      tensor: |Sel| x d x 4 x G flops; also gathered K/V rows |Sel| x d x 2 x 2 B
+    a1, a5 and a2 are timed alone here (their kernels, outside the step); select
+    and attention are the step's own stage times."""
+    import torch
+    from hierarchical_latent_key_gemm_b200 import lsa
+    K, Q, W = inp["K"], inp["Q"], inp["W"]
+    if q0 or nq != Q.shape[1]:
+        Q = Q[:, q0:q0 + nq].contiguous()
+    N, P, r, d, G = w.n_tokens, w.pool, w.r, w.d, w.group
+    units = w.batch * w.hkv
+    nb = N // P
+    L = w.level_sizes[-1]
+    hbm, tf, tfs = peaks["hbm_gbs"], peaks["bf16_tflops"], peaks["bf16_tflops_sustained"]
+    es = 2 if w.dtype == "bf16" else 4
+    Kl = torch.empty((units, nb, r), dtype=torch.float32, device=dev)
+    t_a1 = time_ms(lambda: lsa.lsa_project_pool(K, W, N, P, Kl=Kl))
+    a1 = w.batch * N * w.hkv * d * es + units * nb * r * 4
+    qbar = torch.empty((w.batch, nq, w.hkv, r), dtype=torch.float32, device=dev)
+    t_a5 = time_ms(lambda: lsa.lsa_query_latent(Q, W, w.hkv, qbar=qbar))
+    a5 = Q.numel() * es + qbar.numel() * 4
+    t_a2 = time_ms(lambda: lsa.lsa_kmeans(Kl, L, w.lloyd_iters), reps=2)
+    a2 = 2 * nb * L * r * w.lloyd_iters * units
+    del Kl, qbar
+    torch.cuda.empty_cache()
+    a6, a7, a8 = nodes * r * 2, blocks * r * 2, sel_tokens * 4
+    sel_bytes = a5 + a6 + a7 + a8
+    sel_gbs = sel_bytes / (select_ms / 1e3) / 1e9
+    attn_flops = sel_tokens * d * 4 * G
+    attn_bytes = sel_tokens * d * 2 * 2
+    attn_tf = attn_flops / (attn_ms / 1e3) / 1e12
+    return {
+        "build": {"ms": build_ms, "note": "a1 + a2 + upper levels + bucket layout, in the step"},
+        "a1_project_pool": {"ms": t_a1, "bytes": a1, "achieved_GBps": a1 / (t_a1 / 1e3) / 1e9, "peak_GBps": hbm,
+                            "frac": a1 / (t_a1 / 1e3) / 1e9 / hbm, "bound": "hbm"},
+        "a5_query_latent": {"ms": t_a5, "bytes": a5, "achieved_GBps": a5 / (t_a5 / 1e3) / 1e9, "peak_GBps": hbm,
+                            "frac": a5 / (t_a5 / 1e3) / 1e9 / hbm, "bound": "hbm"},
+        "a2_leaf_kmeans": {"ms": t_a2, "flops": a2, "rounds": w.lloyd_iters,
+                           "achieved_TFLOPs": a2 / (t_a2 / 1e3) / 1e12, "peak_TFLOPs": tf,
+                           "frac": a2 / (t_a2 / 1e3) / 1e12 / tf, "bound": "tensor",
+                           "note": "whole leaf k-means (assign on tensor cores + update + grouping) against the "
+                                   "assign's dense flops; bf16 burst peak"},
+        "select": {"ms": select_ms, "queries_per_s": nq * w.batch * w.hkv / (select_ms / 1e3),
+                   "tree_nodes_scored": nodes, "candidate_blocks_scored": blocks, "selected_tokens": sel_tokens,
+                   "bytes": {"a5_query_latent": a5, "a6_nodes": a6, "a7_blocks": a7, "a8_selection": a8},
+                   "algorithmic_bytes": sel_bytes, "achieved_GBps": sel_gbs, "peak_GBps": hbm,
+                   "frac": sel_gbs / hbm, "bound": "hbm",
+                   "formula": ("(Q bytes + latent queries r x 4 B + tree nodes scored x r x 2 B + candidate "
+                               "blocks scored x r x 2 B + selected tokens x 4 B) / select-stage time; the "
+                               "latents stay L2-resident, so DRAM carries far fewer bytes (traffic)")},
+        "attention": {"ms": attn_ms, "tokens_per_s": nq * w.batch / (attn_ms / 1e3), "selected_rows": sel_tokens,
+                      "flops": attn_flops, "achieved_TFLOPs": attn_tf, "peak_TFLOPs": tfs,
+                      "frac": attn_tf / tfs, "bound": "tensor",
+                      "gathered_bytes": attn_bytes, "gathered_GBps": attn_bytes / (attn_ms / 1e3) / 1e9,
+                      "gathered_frac_of_hbm": attn_bytes / (attn_ms / 1e3) / 1e9 / hbm,
+                      "note": ("flops = |Sel| x d x 4 x G (QK and PV); bf16 sustained peak (timed inside the "
+                               "step); gathered bytes = |Sel| x d x 2 B x 2 (K and V rows), mostly served by L2 "
+                               "because neighbouring queries share rows, so they can exceed the HBM rate")},
+    }
+
+
+def _sampled_positions(w, count: int):
+    import torch
+    pos = torch.linspace(0, w.n_tokens - 1, count).round().to(torch.int64)
+    return torch.unique(pos)
+
+
+def _long_range(row, i, w):
+    lo = max(0, i - w.window + 1)
+    base = set(range(min(w.sink, lo))) | set(range(lo, i + 1))
+    return set(row) - base
+
+
+def recall_of(w, pos, fidx, fcnt, sidx, scnt) -> float:
+    """Share of the exact full-scan long-range picks that a selection also made
+    (rows at positions pos, every sequence and KV head)."""
+    fi, fc, si, sc = fidx.cpu(), fcnt.cpu(), sidx.cpu(), scnt.cpu()
+    hit = tot = 0
+    for b in range(w.batch):
+        for h in range(w.hkv):
+            for k in range(pos.numel()):
+                i = int(pos[k])
+                f = _long_range(fi[b, k, h, : fc[b, k, h]].tolist(), i, w)
+                t = _long_range(si[b, k, h, : sc[b, k, h]].tolist(), i, w)
+                tot += len(f)
+                hit += len(f & t)
+    return hit / max(1, tot)
+
+
+def recall_study(w, inp, dev, pool=None, sample: int = 2048) -> dict:
+    """Tree selection against the exact full-scan top-K on the same data (one
+    build, sampled queries, every KV head), and the planted needles' hit
+    rates; `pool` overrides the workload's block size (same K, Q, W)."""
+    import torch
+    from hierarchical_latent_key_gemm_b200 import lsa
+    P = pool or w.pool
+    dt = lsa.LSA_BF16 if w.dtype == "bf16" else lsa.LSA_F32
+    bp = lsa.make_build_params(w.batch, w.n_tokens, w.n_tokens, w.hkv, w.d, w.r, P, dt, w.level_sizes,
+                               w.lloyd_iters, w.grid_log2, w.sink, 0)
+    sp = lsa.make_select_params(w.hq, w.beam, w.topk, w.sink, w.window)
+    ix = lsa.lsa_build_index(bp, inp["K"], inp["W"])
+    pos = _sampled_positions(w, sample).to(dev)
+    qs = inp["Q"][:, pos].contiguous()
+    qpos = pos[None, :].repeat(w.batch, 1).contiguous()
+    ti, tc = lsa.lsa_select(ix, sp, qs, q_pos=qpos)
+    fi, fc = lsa.lsa_fullscan_select(ix, sp, qs, q_pos=qpos)
+    rec = recall_of(w, pos.cpu(), fi, fc, ti, tc)
+    needles = inp["needles"]
+    nh_t = nh_f = 0
+    if needles:
+        npos = torch.tensor([qp for (_, _, _, qp) in needles], device=dev)
+        nq_ = inp["Q"][:, npos].contiguous()
+        nqpos = npos[None, :].repeat(w.batch, 1).contiguous()
+        a, ac = lsa.lsa_select(ix, sp, nq_, q_pos=nqpos)
+        f, fcn = lsa.lsa_fullscan_select(ix, sp, nq_, q_pos=nqpos)
+        for k, (b, h, p, qp) in enumerate(needles):
+            nh_t += int((a[b, k, h, : ac[b, k, h]] == p).any().item())
+            nh_f += int((f[b, k, h, : fcn[b, k, h]] == p).any().item())
+    ix.free()
+    return {"pool": P, "sample_queries": int(pos.numel()), "tree_recall_vs_fullscan_topk": rec,
+            "needle_hit_rate_tree": nh_t / max(1, len(needles)),
+            "needle_hit_rate_fullscan": nh_f / max(1, len(needles)), "needles": len(needles)}
+
+
+def layer_measure(w, dev, steps: int = 3, warmup: int = 2, seed: int = 0, inp=None) -> dict:
+    """One prefill layer of workload w (build + select for every query +
+    banded attention), stage times by CUDA events, mean over `steps`."""
+    import torch
+    from hierarchical_latent_key_gemm_b200 import lsa
+    from hierarchical_latent_key_gemm_b200.workloads import describe, make_inputs
+    if inp is None:
+        inp = make_inputs(w, seed=seed, device=dev)
+    Q, K, V, W = inp["Q"], inp["K"], inp["V"], inp["W"]
+    N = w.n_tokens
+    dt = lsa.LSA_BF16 if w.dtype == "bf16" else lsa.LSA_F32
+    bp = lsa.make_build_params(w.batch, N, N, w.hkv, w.d, w.r, w.pool, dt, w.level_sizes, w.lloyd_iters,
+                               w.grid_log2, w.sink, 0)
+    sp = lsa.make_select_params(w.hq, w.beam, w.topk, w.sink, w.window)
+    idx = torch.empty((w.batch, N, w.hkv, w.max_sel), dtype=torch.int32, device=dev)
+    cnt = torch.empty((w.batch, N, w.hkv), dtype=torch.int32, device=dev)
+    O = torch.empty_like(Q)
+    lse = torch.empty((w.batch, N, w.hq), dtype=torch.float32, device=dev)
+
+    def step(ev=None):
+        if ev:
+            ev[0].record()
+        ix = lsa.lsa_build_index(bp, K, W)
+        if ev:
+            ev[1].record()
+        lsa.lsa_select(ix, sp, Q, idx=idx, cnt=cnt, max_sel=w.max_sel)
+        if ev:
+            ev[2].record()
+        lsa.lsa_sparse_attn_banded(Q, K, V, idx, cnt, w.hkv, w.sink, w.window, O=O, lse=lse)
+        if ev:
+            ev[3].record()
+        return ix
+
+    for _ in range(warmup):
+        step().free()
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+    for k in range(steps):
+        step(evs[k]).free()
+    torch.cuda.synchronize()
+    st = lsa.lsa_check(None)
+    b_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    s_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    a_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    layer = statistics.mean(e[0].elapsed_time(e[3]) for e in evs)
+    del idx, cnt, O, lse
+    return {"workload": describe(w), "layer_ms": layer, "tokens_per_s": N * w.batch / (layer / 1e3),
+            "build_ms": b_ms, "select_ms": s_ms, "select_queries_per_s": N * w.batch * w.hkv / (s_ms / 1e3),
+            "attn_ms": a_ms, "attn_tokens_per_s": N * w.batch / (a_ms / 1e3), "steps": steps, "warmup": warmup,
+            "status": lsa.strerror(st)}
+
+
+def run_other_workloads(dev, peaks) -> dict:
+    """The other four workloads, measured after the headline one on the same
+    GPU: per-layer prefill figures (and, for gqa_128k, the tree's recall and
+    needle hits with the configured pooling and without pooling), and the
+    decode step at 10M tokens x 4 sequences."""
+    import torch
+    from hierarchical_latent_key_gemm_b200.workloads import WORKLOADS, make_inputs
+    out = {}
+    for name in ("flat_4k_f32", "int_exact_16k", "gqa_128k"):
+        w = WORKLOADS[name]
+        inp = make_inputs(w, seed=0, device=dev)
+        out[name] = layer_measure(w, dev, inp=inp)
+        if name == "gqa_128k":
+            out[name]["recall"] = [recall_study(w, inp, dev), recall_study(w, inp, dev, pool=1)]
+        del inp
+        torch.cuda.empty_cache()
+    w = WORKLOADS["decode_10m_x4"]
+    r = decode_measure(w, dev, 0, 3, 1, True)
+    r.pop("clocks", None)
+    out[w.name] = r
+    return out
+
+
 # ------------------------------------------------------------------ CPU oracle
 def cpu_cores() -> int:
     try:
@@ -595,7 +837,7 @@ def cpu_cores() -> int:
     return os.cpu_count() or 1
 
 
-def cpu_oracle_estimate(w, inp, sample_queries: int, lloyd_stride: int = 2) -> dict:
+def cpu_oracle_estimate(w, inp, sample_queries: int, lloyd_stride: int = CPU_LLOYD_STRIDE) -> dict:
     """Time the oracle, as it stands, on a bounded sample of the workload and
     scale to one whole layer: latents of every block; one Lloyd round of one
     KV head over every lloyd_stride-th block against all leaf centroids
@@ -681,7 +923,7 @@ def run_reference(args):
     vals = []
     cpu = None
     for k in range(args.warmup + args.steps):
-        r = cpu_oracle_estimate(w, inp, max(8, args.cpu_sample_queries // 4), lloyd_stride=32)
+        r = cpu_oracle_estimate(w, inp, args.cpu_sample_queries)
         if k >= args.warmup:
             vals.append(r["value"])
             cpu = r
@@ -689,8 +931,7 @@ def run_reference(args):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * w.n_tokens / value, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
-            "config": {"workload": describe(w), "global_batch": w.batch, "seq_len": w.n_tokens,
-                       "parallelism": "host cores of rank 0"},
+            "config": run_config(w, world, args.seed),
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu["cores"], "kind": "oracle",
                              "sample": cpu["sample"]},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}

@@ -398,6 +398,85 @@ int lsa_fullscan_select(const lsa_index* index, const lsa_select_params* params,
     return do_select(index, params, Q, nq, q_pos, q_pos0, idx, cnt, max_sel, stream, true);
 }
 
+int lsa_select_blocks(const lsa_index* index, const lsa_select_params* params, const void* Q, int64_t nq,
+                      const int64_t* q_pos, int64_t q_pos0, int64_t token_offset, float* scores, int32_t* blocks,
+                      int32_t* count, int32_t kb_cap, void* stream) {
+    if (!live(index) || !params) return LSA_ERR_INVALID_ARG;
+    const lsa_build_params& p = index->p;
+    const lsa_select_params& sp = *params;
+    if (sp.hq < p.hkv || sp.hq % p.hkv || sp.beam < 1 || sp.beam > 1024 || sp.topk < 0 || sp.window < 1 ||
+        sp.sink != p.sink)
+        return LSA_ERR_INVALID_ARG;
+    const int64_t kb = (sp.topk + p.pool - 1) / p.pool;
+    if (kb > 4096 || kb_cap < kb || kb_cap < 1) return LSA_ERR_INVALID_ARG;
+    if (token_offset < 0 || token_offset % p.pool || token_offset / p.pool + index->nb_cap > INT32_MAX)
+        return LSA_ERR_INVALID_ARG;
+    if (nq < 0 || nq > INT32_MAX) return LSA_ERR_INVALID_ARG;
+    if (!q_pos && (q_pos0 < 0 || q_pos0 + nq > INT32_MAX)) return LSA_ERR_INVALID_ARG;
+    if (nq == 0) return LSA_OK;
+    if (!is_device_ptr(Q) || !is_device_ptr(scores) || !is_device_ptr(blocks) || !is_device_ptr(count))
+        return LSA_ERR_INVALID_ARG;
+    if (q_pos && !is_device_ptr(q_pos)) return LSA_ERR_INVALID_ARG;
+    cudaStream_t s = as_stream(stream);
+    keep_pool_memory();
+    Arena scratch;
+    scratch.async = true;
+    scratch.stream = s;
+    float* qbar = scratch.alloc<float>(p.batch * nq * p.hkv * p.r);
+    if (scratch.status != LSA_OK) return scratch.status;
+    ScoredOut so{token_offset, (int32_t)(token_offset / p.pool), kb_cap, scores, blocks, count};
+    int st = launch_query_latent(Q, index->W, p.batch, nq, sp.hq, p.hkv, p.d, p.r, p.dtype, qbar, s);
+    if (st == LSA_OK)
+        st = launch_select(index, params, qbar, nq, q_pos, q_pos0, nullptr, nullptr, 0, false, s, nullptr, &so);
+    scratch.release();
+    return st;
+}
+
+int lsa_merge_selection(int32_t parts, const float* scores, const int32_t* blocks, const int32_t* count,
+                        int32_t kb_cap, int64_t batch, int64_t nq, int32_t hkv, const int64_t* q_pos, int64_t q_pos0,
+                        int32_t pool, int32_t topk, int32_t sink, int32_t window, int32_t* idx, int32_t* cnt,
+                        int32_t max_sel, void* stream) {
+    if (parts < 1 || parts > 64 || kb_cap < 1 || (int64_t)parts * kb_cap > 16384) return LSA_ERR_INVALID_ARG;
+    if (batch < 1 || nq < 0 || hkv < 1 || pool < 1 || pool > 16 || topk < 0 || sink < 0 || window < 1)
+        return LSA_ERR_INVALID_ARG;
+    const int64_t kb = ((int64_t)topk + pool - 1) / pool;
+    if (kb > (int64_t)parts * kb_cap || (int64_t)max_sel < kb * pool + sink + window) return LSA_ERR_INVALID_ARG;
+    if (batch * nq * hkv > INT32_MAX) return LSA_ERR_INVALID_ARG;
+    if (!q_pos && (q_pos0 < 0 || q_pos0 + nq > INT32_MAX)) return LSA_ERR_INVALID_ARG;
+    if (nq == 0) return LSA_OK;
+    if (!is_device_ptr(scores) || !is_device_ptr(blocks) || !is_device_ptr(count) || !is_device_ptr(idx) ||
+        !is_device_ptr(cnt))
+        return LSA_ERR_INVALID_ARG;
+    if (q_pos && !is_device_ptr(q_pos)) return LSA_ERR_INVALID_ARG;
+    return launch_merge_selection(parts, scores, blocks, count, kb_cap, batch, nq, hkv, q_pos, q_pos0, pool, (int)kb,
+                                  sink, window, idx, cnt, max_sel, as_stream(stream));
+}
+
+int lsa_localize_rows(const int32_t* idx, const int32_t* cnt, int64_t rows, int32_t max_sel, int64_t lo, int64_t hi,
+                      int32_t* idx_out, int32_t* cnt_out, void* stream) {
+    if (rows < 0 || max_sel < 1 || lo < 0 || hi < lo || rows > ((int64_t)1 << 36)) return LSA_ERR_INVALID_ARG;
+    if (rows == 0) return LSA_OK;
+    if (!is_device_ptr(idx) || !is_device_ptr(cnt) || !is_device_ptr(idx_out) || !is_device_ptr(cnt_out))
+        return LSA_ERR_INVALID_ARG;
+    // idx_out is idx, or does not overlap it
+    const int64_t bytes = rows * max_sel * (int64_t)sizeof(int32_t);
+    const char* a = reinterpret_cast<const char*>(idx);
+    const char* b = reinterpret_cast<const char*>(idx_out);
+    if (a != b && a < b + bytes && b < a + bytes) return LSA_ERR_INVALID_ARG;
+    return launch_localize_rows(idx, cnt, rows, max_sel, lo, hi, idx_out, cnt_out, as_stream(stream));
+}
+
+int lsa_merge_attn(int32_t parts, const void* O_parts, const float* lse_parts, int64_t rows, int32_t hq, int32_t d,
+                   int32_t dtype, void* O, float* lse, void* stream) {
+    if (parts < 1 || rows < 0 || hq < 1 || d < 1 || d > 1024 || (dtype != LSA_F32 && dtype != LSA_BF16))
+        return LSA_ERR_INVALID_ARG;
+    if (rows * hq > ((int64_t)1 << 36)) return LSA_ERR_INVALID_ARG;
+    if (rows == 0) return LSA_OK;
+    if (!is_device_ptr(O_parts) || !is_device_ptr(lse_parts) || !is_device_ptr(O)) return LSA_ERR_INVALID_ARG;
+    if (lse && !is_device_ptr(lse)) return LSA_ERR_INVALID_ARG;
+    return launch_merge_attn(parts, O_parts, lse_parts, rows, hq, d, dtype, O, lse, as_stream(stream));
+}
+
 int lsa_sparse_attn(const void* Q, const void* K, const void* V, const int32_t* idx, const int32_t* cnt,
                     int64_t batch, int64_t nq, int32_t hq, int32_t hkv, int32_t d, int32_t dtype, int32_t max_sel,
                     int64_t ld_tokens, void* O, float* lse, void* stream) {
@@ -507,18 +586,24 @@ int lsa_pca_map(const void* K, int64_t batch, int64_t n_tokens, int64_t ld_token
 }
 
 int lsa_kmeans(const float* X, int64_t units, int64_t n, int32_t r, int32_t k, int32_t iters, int32_t grid_log2,
-               int32_t* labels, float* C, double* objective, void* stream) {
+               int32_t* labels, float* C, const float* C_init, double* objective, void* stream) {
     if (units < 1 || units > 65535 || n < 1 || !valid_r(r) || k < 1 || iters < 1 || grid_log2 < 0 || grid_log2 > 8)
         return LSA_ERR_INVALID_ARG;
     if (units * n > INT32_MAX / 2 || units * (int64_t)k > INT32_MAX / 4) return LSA_ERR_INVALID_ARG;
     if (!is_device_ptr(X) || !is_device_ptr(labels) || !is_device_ptr(C)) return LSA_ERR_INVALID_ARG;
     if (objective && !is_device_ptr(objective)) return LSA_ERR_INVALID_ARG;
+    if (C_init) {
+        const int64_t bytes = units * (int64_t)k * r * (int64_t)sizeof(float);
+        const char* a = reinterpret_cast<const char*>(C_init);
+        const char* b = reinterpret_cast<const char*>(C);
+        if (!is_device_ptr(C_init) || (a < b + bytes && b < a + bytes)) return LSA_ERR_INVALID_ARG;
+    }
     cudaStream_t s = as_stream(stream);
     Arena scratch;
     scratch.async = true;
     scratch.stream = s;
     KmeansOut ko{labels, C, nullptr, nullptr, objective};
-    int st = run_kmeans(X, n, units, n, r, k, iters, grid_log2, ko, n, global_err_word(), s, scratch);
+    int st = run_kmeans(X, n, units, n, r, k, iters, grid_log2, ko, n, global_err_word(), s, scratch, C_init);
     scratch.release();
     return st;
 }

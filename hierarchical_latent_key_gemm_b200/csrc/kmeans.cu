@@ -411,7 +411,7 @@ int refresh_centroids(lsa_index* ix, cudaStream_t s, Arena& A) {
 }
 
 int run_kmeans(const float* X, int64_t ldx, int64_t units, int64_t n, int r, int k, int iters, int grid_log2,
-               KmeansOut out, int64_t ldl, int32_t* err, cudaStream_t s, Arena& A) {
+               KmeansOut out, int64_t ldl, int32_t* err, cudaStream_t s, Arena& A, const float* C_init) {
     if (units <= 0 || n <= 0 || k <= 0) return LSA_OK;
     if (r != 16 && r != 32 && r != 64 && r != 128) return LSA_ERR_INVALID_ARG;
     const int64_t nc = units * (int64_t)k;
@@ -429,12 +429,17 @@ int run_kmeans(const float* X, int64_t ldx, int64_t units, int64_t n, int r, int
     GroupWork gw = alloc_group_work(units, n, k, A);
     if (A.status != LSA_OK) return A.status;
     const int64_t tot = nc * r;
-    note_launch();
-    init_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, s>>>(X, ldx, units, n, k, r, out.C);
+    if (C_init) {
+        const cudaError_t e = cudaMemcpyAsync(out.C, C_init, tot * sizeof(float), cudaMemcpyDeviceToDevice, s);
+        if (e != cudaSuccess) return cuda_status(e);
+    } else {
+        note_launch();
+        init_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, s>>>(X, ldx, units, n, k, r, out.C);
+    }
     if (simt) launch_transpose(X, units, n, ldx, r, XT, ldxt, s);
     void* tcw = nullptr;
     if (tc) {
-        const int st = assign_tc_prepare_points(X, ldx, units, n, r, k, A, s, &tcw);
+        const int st = assign_tc_prepare_points(X, ldx, units, n, r, k, out.C, A, s, &tcw);
         if (st != LSA_OK) return st;
     }
     float* cur = out.C;

@@ -2,22 +2,27 @@
 //
 // distance(x, c_j) = ||c_j||^2 - 2 x.c_j (||x||^2 is common to a row); the
 // x.c products of a 128-point tile against 256-centroid tiles are one dense
-// GEMM per tile.  Operands are fp32; each is split into two tf32 parts
-// (x = xb + xs, c = cb + cs) and the GEMM runs over K = 3r with
-// A = [xb | xb | xs], B = [cb | cs | cb], so the accumulator holds
-// xb.cb + xb.cs + xs.cb: the dropped xs.cs term and the tf32 roundings leave an
-// error near 2^-21 of |x||c|, i.e. fp32-like assignments.
+// GEMM per tile.  Operands are fp32; each is scaled by one power of two
+// (exact; chosen from the largest magnitude so that every value fits fp16)
+// and split into two fp16 parts (x = xh + xl, c = ch + cl), and the GEMM runs
+// over K = 3r with A = [xh | xh | xl], B = [ch | cl | ch] (zero-padded to a
+// multiple of 64), so the accumulator holds xh.ch + xh.cl + xl.ch: fp16 keeps
+// 11 significant bits like tf32, so the dropped xl.cl term and the roundings
+// leave an error near 2^-21 of |x||c| (fp32-like assignments), at the f16 MMA
+// rate, twice the tf32 one.
 //
 // One CTA per 128 points, persistent over all centroid tiles of its unit:
-//   warp 0    TMA producer: the point tile once (6 K-chunks resident), then
+//   warp 0    TMA producer: the point tile once (all K-chunks resident), then
 //             centroid K-chunks through a 3-stage ring (128B swizzle)
-//   warp 1    TMEM owner and MMA issuer (one thread): tcgen05.mma kind::tf32,
-//             M=128, N=256, K=8 per instruction, into one of two TMEM
-//             accumulators (2 x 256 columns)
+//   warp 1    TMEM owner and MMA issuer (one thread): tcgen05.mma kind::f16
+//             (fp16 A and B), M=128, N=256, K=16 per instruction, into one of
+//             two TMEM accumulators (2 x 256 columns)
 //   warps 2-5 epilogue: tcgen05.ld of the accumulator rows, running
 //             (distance, id) minimum per point, ties to the lower id
 // Every mbarrier wait is bounded; a timeout latches kErrTimeout and the CTA
 // winds down (TMEM is always released).
+#include <cuda_fp16.h>
+
 #include <mutex>
 #include <new>
 
@@ -28,7 +33,7 @@ namespace {
 
 constexpr int kTM = 128;          // points per CTA (UMMA M)
 constexpr int kTN = 256;          // centroids per tile (UMMA N)
-constexpr int kKC = 32;           // tf32 per K-chunk: one 128-byte swizzle row
+constexpr int kKC = 64;           // fp16 per K-chunk: one 128-byte swizzle row
 constexpr int kStagesB = 3;
 constexpr int kThreadsTC = 192;
 // K-major operand, 128-byte swizzle: 8-row x 128-byte atoms, 1024 bytes apart.
@@ -42,17 +47,21 @@ __device__ __forceinline__ uint64_t umma_desc(const void* p) {
     d |= (uint64_t)2 << 61;                // 128-byte swizzle
     return d;
 }
-// kind::tf32, fp32 accumulate, K-major A and B, M = 128, N = 256.
-constexpr uint32_t kIdesc = (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(kTN >> 3) << 17) |
+// kind::f16 with fp16 A and B (format 0), fp32 accumulate, K-major A and B,
+// M = 128, N = 256.
+constexpr uint32_t kIdesc = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(kTN >> 3) << 17) |
                             ((uint32_t)(kTM >> 4) << 24);
 
-__device__ __forceinline__ void umma_tf32(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accumulate) {
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accumulate) {
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(tmem_d),
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(tmem_d),
         "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate), "r"(0u));
 }
+
+// K extent of the split operands: 3r rounded up to whole 64-element chunks.
+__host__ __device__ constexpr int split_k(int r) { return (3 * r + kKC - 1) / kKC * kKC; }
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(bar))
                  : "memory");
@@ -72,52 +81,79 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
     for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
-__device__ __forceinline__ float to_tf32(float x) {
-    uint32_t r;
-    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
-    return __uint_as_float(r);
+// Largest |value| of the points and the starting centroids, as float bits
+// (non-negative floats order like their bit patterns).
+__global__ void absmax_kernel(const float* __restrict__ X, int64_t ldx, int64_t n, int r, int64_t units,
+                              const float* __restrict__ C, int64_t nc, uint32_t* __restrict__ out) {
+    uint32_t m = 0;
+    const int64_t tot = units * n * r;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < tot + nc;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        float v;
+        if (e < tot) {
+            const int64_t c = e % r, row = e / r;
+            v = X[((row / n) * ldx + row % n) * r + c];
+        } else {
+            v = C[e - tot];
+        }
+        m = max(m, __float_as_uint(fabsf(v)));
+    }
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) m = max(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if ((threadIdx.x & 31) == 0) atomicMax(out, m);
 }
 
-// Xs[u*n_pad + p] = [tf32(x) | tf32(x) | tf32(x - tf32(x))], zero rows past n.
+// The power of two 2^-e that brings the largest magnitude into [2^13, 2^14)
+// (|scaled value| < 2^14 fits fp16 with room for sums of parts).
+__device__ __forceinline__ int scale_exp(const uint32_t* absmax) {
+    const float m = __uint_as_float(*absmax);
+    if (!(m > 0.f) || isinf(m)) return 0;
+    // (clamped so that 2^(2e+1), the epilogue's factor, stays a normal float)
+    return max(-60, min(60, ilogbf(m) - 13));
+}
+
+// Xs[u*n_pad + p] = [xh | xh | xl | 0], x scaled by 2^-e, zero rows past n.
 __global__ void split_points_kernel(const float* __restrict__ X, int64_t ldx, int64_t n, int64_t n_pad, int r,
-                                    int64_t units, float* __restrict__ Xs) {
+                                    int64_t units, const uint32_t* __restrict__ absmax, __half* __restrict__ Xs) {
+    const int kp = split_k(r);
     const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (e >= units * n_pad * r) return;
-    const int c = (int)(e % r);
-    const int64_t row = e / r;
+    if (e >= units * n_pad * kp) return;
+    const int c = (int)(e % kp);
+    const int64_t row = e / kp;
     const int64_t u = row / n_pad, p = row % n_pad;
+    const int sc = -scale_exp(absmax);
+    const int src = c < r ? c : (c < 2 * r ? c - r : (c < 3 * r ? c - 2 * r : -1));
     float x = 0.f;
-    if (p < n) x = X[(u * ldx + p) * r + c];
-    const float xb = to_tf32(x);
-    float* o = Xs + row * 3 * r;
-    o[c] = xb;
-    o[r + c] = xb;
-    o[2 * r + c] = to_tf32(x - xb);
+    if (p < n && src >= 0) x = ldexpf(X[(u * ldx + p) * r + src], sc);
+    const __half xh = __float2half_rn(x);
+    const __half xl = __float2half_rn(x - __half2float(xh));
+    Xs[row * kp + c] = (c < 2 * r) ? xh : (c < 3 * r ? xl : __float2half_rn(0.f));
 }
 
-// Cs[u*k_pad + j] = [tf32(c) | tf32(c - tf32(c)) | tf32(c)], zero rows past k.
+// Cs[u*k_pad + j] = [ch | cl | ch | 0], c scaled by 2^-e, zero rows past k.
 __global__ void split_centroids_kernel(const float* __restrict__ C, int k, int k_pad, int r, int64_t units,
-                                       float* __restrict__ Cs) {
+                                       const uint32_t* __restrict__ absmax, __half* __restrict__ Cs) {
+    const int kp = split_k(r);
     const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (e >= units * k_pad * r) return;
-    const int c = (int)(e % r);
-    const int64_t row = e / r;
+    if (e >= units * k_pad * kp) return;
+    const int c = (int)(e % kp);
+    const int64_t row = e / kp;
     const int64_t u = row / k_pad, j = row % k_pad;
+    const int sc = -scale_exp(absmax);
+    const int src = c < r ? c : (c < 2 * r ? c - r : (c < 3 * r ? c - 2 * r : -1));
     float x = 0.f;
-    if (j < k) x = C[(u * k + j) * r + c];
-    const float xb = to_tf32(x);
-    float* o = Cs + row * 3 * r;
-    o[c] = xb;
-    o[r + c] = to_tf32(x - xb);
-    o[2 * r + c] = xb;
+    if (j < k && src >= 0) x = ldexpf(C[(u * k + j) * r + src], sc);
+    const __half xh = __float2half_rn(x);
+    const __half xl = __float2half_rn(x - __half2float(xh));
+    Cs[row * kp + c] = (c < 3 * r && c >= r && c < 2 * r) ? xl : (c < 3 * r ? xh : __float2half_rn(0.f));
 }
 
 template <int R>
 __global__ void __launch_bounds__(kThreadsTC, 1)
     assign_tc_kernel(const __grid_constant__ CUtensorMap map_x, const __grid_constant__ CUtensorMap map_c,
                      int64_t n, int64_t n_pad, int k, int k_pad, const float* __restrict__ cc,
-                     int32_t* __restrict__ labels, int64_t ldl, int32_t* err) {
-    constexpr int KS = 3 * R / kKC;                  // K-chunks
+                     const uint32_t* __restrict__ absmax, int32_t* __restrict__ labels, int64_t ldl, int32_t* err) {
+    constexpr int KS = split_k(R) / kKC;             // K-chunks
     constexpr int A_CHUNK = kTM * 128;               // bytes per A chunk
     constexpr int B_CHUNK = kTN * 128;               // bytes per B stage
     extern __shared__ unsigned char smem_raw[];
@@ -200,10 +236,10 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
                     if (!mbar_wait(b_full + s, (uint32_t)(it / kStagesB) & 1u)) { ok = false; break; }
                     asm volatile("tcgen05.fence::after_thread_sync;");
 #pragma unroll
-                    for (int kk = 0; kk < kKC / 8; ++kk) {
+                    for (int kk = 0; kk < kKC / 16; ++kk) {
                         const uint64_t da = umma_desc(As + c * A_CHUNK + kk * 32);
                         const uint64_t db = umma_desc(Bs + s * B_CHUNK + kk * 32);
-                        umma_tf32(d, da, db, (c | kk) ? 1u : 0u);
+                        umma_f16(d, da, db, (c | kk) ? 1u : 0u);
                     }
                     umma_commit(b_empty + s);
                 }
@@ -220,6 +256,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         float best = INFINITY;
         int bestj = 0;
         const float* ccu = cc + (int64_t)u * k;
+        // x.c = 2^(2e) (scaled x).(scaled c): -2 x.c is one exact power-of-two multiple
+        const float m2 = -ldexpf(2.f, 2 * scale_exp(absmax));
         for (int t = 0; t < ntile; ++t) {
             const int buf = t & 1;
             // the tile's centroid norms, one per lane per 32-column chunk, read
@@ -240,7 +278,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     const int j = j0 + i;
-                    const float dist = __fmaf_rn(-2.f, v[i], __shfl_sync(0xffffffffu, ccr[cb], i));
+                    const float dist = __fmaf_rn(m2, v[i], __shfl_sync(0xffffffffu, ccr[cb], i));
                     if (j < k && dist < best) { best = dist; bestj = j; }
                 }
             }
@@ -257,7 +295,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 
 template <int R>
 size_t tc_smem_bytes() {
-    return (size_t)(3 * R / kKC) * kTM * 128 + (size_t)kStagesB * kTN * 128 + 256 + 1024;
+    return (size_t)(split_k(R) / kKC) * kTM * 128 + (size_t)kStagesB * kTN * 128 + 256 + 1024;
 }
 
 }  // namespace
@@ -267,24 +305,34 @@ bool assign_tc_supported(int r, int grid_log2) { return (r == 32 || r == 64) && 
 // Scratch for the tensor-core assign of (units, n, k, r): split points and
 // split centroids.
 struct AssignTcWork {
-    float* Xs = nullptr;
-    float* Cs = nullptr;
+    __half* Xs = nullptr;
+    __half* Cs = nullptr;
+    uint32_t* absmax = nullptr;
     int64_t n_pad = 0;
     int k_pad = 0;
 };
 
-int assign_tc_prepare_points(const float* X, int64_t ldx, int64_t units, int64_t n, int r, int k, Arena& A,
-                             cudaStream_t s, void** work_out) {
+int assign_tc_prepare_points(const float* X, int64_t ldx, int64_t units, int64_t n, int r, int k, const float* C0,
+                             Arena& A, cudaStream_t s, void** work_out) {
     AssignTcWork* w = new (std::nothrow) AssignTcWork();
     if (!w) return LSA_ERR_OOM;
     w->n_pad = (n + kTM - 1) / kTM * kTM;
     w->k_pad = (k + kTN - 1) / kTN * kTN;
-    w->Xs = A.alloc<float>(units * w->n_pad * 3 * r);
-    w->Cs = A.alloc<float>(units * (int64_t)w->k_pad * 3 * r);
+    const int kp = split_k(r);
+    w->Xs = A.alloc<__half>(units * w->n_pad * kp);
+    w->Cs = A.alloc<__half>(units * (int64_t)w->k_pad * kp);
+    w->absmax = A.alloc<uint32_t>(1);
     if (A.status != LSA_OK) { delete w; return A.status; }
-    const int64_t tot = units * w->n_pad * r;
+    // one scale for the run: the points, and the centroids it starts from
+    // (later centroids are means of points, never larger)
+    cudaError_t e = cudaMemsetAsync(w->absmax, 0, sizeof(uint32_t), s);
+    if (e != cudaSuccess) { delete w; return cuda_status(e); }
     note_launch();
-    split_points_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, s>>>(X, ldx, n, w->n_pad, r, units, w->Xs);
+    absmax_kernel<<<592, 256, 0, s>>>(X, ldx, n, r, units, C0, units * (int64_t)k * r, w->absmax);
+    const int64_t tot = units * w->n_pad * kp;
+    note_launch();
+    split_points_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, s>>>(X, ldx, n, w->n_pad, r, units, w->absmax,
+                                                                      w->Xs);
     *work_out = w;
     return cuda_status(cudaGetLastError());
 }
@@ -294,14 +342,14 @@ void assign_tc_release(void* work) { delete static_cast<AssignTcWork*>(work); }
 int assign_tc_run(void* work, const float* C, const float* cc, int64_t units, int64_t n, int r, int k,
                   int32_t* labels, int64_t ldl, int32_t* err, cudaStream_t s) {
     AssignTcWork* w = static_cast<AssignTcWork*>(work);
-    const int64_t tot = units * (int64_t)w->k_pad * r;
+    const int kp = split_k(r);
+    const int64_t tot = units * (int64_t)w->k_pad * kp;
     note_launch();
-    split_centroids_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, s>>>(C, k, w->k_pad, r, units, w->Cs);
+    split_centroids_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, s>>>(C, k, w->k_pad, r, units, w->absmax,
+                                                                         w->Cs);
     CUtensorMap mx, mc;
-    if (!make_tensor_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->Xs, units * w->n_pad, 3 * r, 3 * r * 4, kKC,
-                            kTM) ||
-        !make_tensor_map_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, w->Cs, units * w->k_pad, 3 * r, 3 * r * 4, kKC,
-                            kTN))
+    if (!make_tensor_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, w->Xs, units * w->n_pad, kp, kp * 2, kKC, kTM) ||
+        !make_tensor_map_2d(&mc, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, w->Cs, units * w->k_pad, kp, kp * 2, kKC, kTN))
         return LSA_ERR_CUDA;
     dim3 grid((unsigned)(w->n_pad / kTM), (unsigned)units);
     cudaError_t e;
@@ -310,13 +358,15 @@ int assign_tc_run(void* work, const float* C, const float* cc, int64_t units, in
         e = cudaFuncSetAttribute(assign_tc_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return cuda_status(e);
         note_launch();
-        assign_tc_kernel<64><<<grid, kThreadsTC, smem, s>>>(mx, mc, n, w->n_pad, k, w->k_pad, cc, labels, ldl, err);
+        assign_tc_kernel<64><<<grid, kThreadsTC, smem, s>>>(mx, mc, n, w->n_pad, k, w->k_pad, cc, w->absmax, labels,
+                                                             ldl, err);
     } else {
         const size_t smem = tc_smem_bytes<32>();
         e = cudaFuncSetAttribute(assign_tc_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return cuda_status(e);
         note_launch();
-        assign_tc_kernel<32><<<grid, kThreadsTC, smem, s>>>(mx, mc, n, w->n_pad, k, w->k_pad, cc, labels, ldl, err);
+        assign_tc_kernel<32><<<grid, kThreadsTC, smem, s>>>(mx, mc, n, w->n_pad, k, w->k_pad, cc, w->absmax, labels,
+                                                             ldl, err);
     }
     return cuda_status(cudaGetLastError());
 }

@@ -132,7 +132,8 @@ struct KmeansOut {
 // X: [units][ldx][r] (rows 0..n-1 of each unit are the points); labels are
 // written at out.labels[u*ldl + i].
 int run_kmeans(const float* X, int64_t ldx, int64_t units, int64_t n, int r, int k, int iters,
-               int grid_log2, KmeansOut out, int64_t ldl, int32_t* err, cudaStream_t s, Arena& scratch);
+               int grid_log2, KmeansOut out, int64_t ldl, int32_t* err, cudaStream_t s, Arena& scratch,
+               const float* C_init = nullptr);
 
 // Stable grouping of points by label (see run_kmeans); workspace sized for
 // (units, n, k) by alloc_group_work.
@@ -148,8 +149,8 @@ int group_by_label(const int32_t* labels, int64_t ldl, int64_t units, int64_t n,
 // Tensor-core assign (kmeans_tc.cu): prepare the split points once per run,
 // then one call per Lloyd round.
 bool assign_tc_supported(int r, int grid_log2);
-int assign_tc_prepare_points(const float* X, int64_t ldx, int64_t units, int64_t n, int r, int k, Arena& A,
-                             cudaStream_t s, void** work_out);
+int assign_tc_prepare_points(const float* X, int64_t ldx, int64_t units, int64_t n, int r, int k, const float* C0,
+                             Arena& A, cudaStream_t s, void** work_out);
 int assign_tc_run(void* work, const float* C, const float* cc, int64_t units, int64_t n, int r, int k,
                   int32_t* labels, int64_t ldl, int32_t* err, cudaStream_t s);
 void assign_tc_release(void* work);
@@ -162,9 +163,32 @@ int launch_query_latent(const void* Q, const float* W, int64_t batch, int64_t nq
                         int d, int r, int dtype, float* qbar, cudaStream_t s);
 
 // ---------------------------------------------------------------- select
+// Scored-blocks output of the tree search (context-parallel shards): per
+// (query, KV head) row the kept blocks (index block id + blk_shift) and their
+// scores in [row][kb_cap], any order, -1 / -inf after *n; query positions are
+// index positions + pos_shift.
+struct ScoredOut {
+    int64_t pos_shift;
+    int32_t blk_shift;
+    int kb_cap;
+    float* score;
+    int32_t* block;
+    int32_t* n;
+};
 int launch_select(const lsa_index* ix, const lsa_select_params* sp, const float* qbar, int64_t nq,
                   const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt, int max_sel,
-                  bool fullscan, cudaStream_t s, unsigned long long* work = nullptr);
+                  bool fullscan, cudaStream_t s, unsigned long long* work = nullptr,
+                  const ScoredOut* scored = nullptr);
+// Merge of per-shard scored blocks into selection rows (select.cu).
+int launch_merge_selection(int parts, const float* score, const int32_t* block, const int32_t* count, int kb_cap,
+                           int64_t batch, int64_t nq, int hkv, const int64_t* q_pos, int64_t q_pos0, int pool,
+                           int kb, int sink, int window, int32_t* idx, int32_t* cnt, int max_sel, cudaStream_t s);
+// Rows of a selection inside [lo, hi), shifted by -lo (cp.cu); LSE merge of
+// attention parts (cp.cu).
+int launch_localize_rows(const int32_t* idx, const int32_t* cnt, int64_t rows, int max_sel, int64_t lo, int64_t hi,
+                         int32_t* idx_out, int32_t* cnt_out, cudaStream_t s);
+int launch_merge_attn(int parts, const void* O_parts, const float* lse_parts, int64_t rows, int hq, int d, int dtype,
+                      void* O, float* lse, cudaStream_t s);
 
 // ---------------------------------------------------------------- attention
 int launch_sparse_attn(const void* Q, const void* K, const void* V, const int32_t* idx,

@@ -22,7 +22,7 @@
 // order in which warps append.  One buffer instead of two halves the shared
 // memory of a CTA, which leaves more of each SM's L1 for the centroid rows
 // that every query of a unit reads.
-#include "lsa_internal.cuh"
+#include "select_common.cuh"
 
 namespace lsa {
 namespace {
@@ -61,298 +61,15 @@ struct SelArgs {
     int32_t* cnt;
     int max_sel;
     int cap;
-    unsigned long long* work;   // optional: += eligible nodes and blocks scored
+    unsigned long long* work;   // optional: [0] += eligible nodes scored, [1] += candidate blocks scored
+    // scored-blocks output (SCORED): the kept blocks and their scores, [row][kb_cap]
+    int64_t pos_shift;          // query positions are given in the caller's numbering; index position = pos - shift
+    int32_t blk_shift;          // block id written = index block id + blk_shift
+    int kb_cap;
+    float* out_score;
+    int32_t* out_block;
+    int32_t* out_n;
 };
-
-constexpr int kResolveCap = 128;
-
-// a candidate group's current owner among the kept nodes: its index, the first
-// candidate past its run, and (its run's first slot - its first candidate)
-struct OwnerState {
-    int o, next, base;
-};   // most items of the threshold bin ranked pairwise
-
-struct SelShared {
-    int hist[256];
-    int bc[4];
-    int count;
-    int count2;
-    int nkept;
-    uint32_t thr;   // no item below this key can be in the current top k (0: none yet)
-    uint32_t wmin[32], wmax[32];
-    int nres;
-};
-
-// 32 bytes from global memory in one 256-bit read-only load (32-byte aligned).
-__device__ __forceinline__ void ldg256(const float* p, float* v) {
-    asm volatile("ld.global.nc.v8.f32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
-                 : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
-                 : "l"(p));
-}
-
-// Order-preserving map of a float onto uint32 (-0 and +0 map together).
-__device__ __forceinline__ uint32_t fkey(float f) {
-    const uint32_t u = __float_as_uint(__fadd_rn(f, 0.0f));
-    return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-
-__device__ __forceinline__ int warp_incl_scan(int v) {
-    const int lane = threadIdx.x & 31;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const int t = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += t;
-    }
-    return v;
-}
-
-// k-th largest key among n items (1 <= k <= n).  mode 0: key = fkey(score);
-// mode 1: key = ~id, restricted to items with fkey(score) == tkey.
-// Precondition: sh.hist is all zero; it is left all zero.  Two barriers per
-// 8-bit pass.  Returns the key; *need = how many items equal to it belong to
-// the top k, *eq = how many items equal it.  Also clears sh.count2.
-__device__ uint32_t block_kth(const float* s, const int* id, int n, int k, int mode, uint32_t tkey,
-                              SelShared& sh, int* need, int* eq) {
-    uint32_t prefix = 0, pmask = 0;
-    int kk = k, eqc = 0;
-#pragma unroll 1
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        for (int i = threadIdx.x; i < n; i += blockDim.x) {
-            uint32_t key;
-            bool act;
-            if (mode == 0) {
-                key = fkey(s[i]);
-                act = true;
-            } else {
-                act = fkey(s[i]) == tkey;
-                key = ~(uint32_t)id[i];
-            }
-            if (act && (key & pmask) == prefix) atomicAdd(&sh.hist[(key >> shift) & 255u], 1);
-        }
-        __syncthreads();
-        if (threadIdx.x < 32) {
-            const int lane = threadIdx.x;
-            int c[8], sum = 0;
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                c[t] = sh.hist[255 - lane * 8 - t];
-                sh.hist[255 - lane * 8 - t] = 0;
-                sum += c[t];
-            }
-            const int incl = warp_incl_scan(sum);
-            const int excl = incl - sum;
-            if (excl < kk && kk <= incl) {
-                int run = excl;
-#pragma unroll
-                for (int t = 0; t < 8; ++t) {
-                    if (run + c[t] >= kk) {
-                        sh.bc[0] = 255 - lane * 8 - t;
-                        sh.bc[1] = kk - run;
-                        sh.bc[2] = c[t];
-                        break;
-                    }
-                    run += c[t];
-                }
-            }
-            if (lane == 0 && shift == 0) sh.count2 = 0;
-        }
-        __syncthreads();
-        prefix |= (uint32_t)sh.bc[0] << shift;
-        pmask |= 255u << shift;
-        kk = sh.bc[1];
-        eqc = sh.bc[2];
-    }
-    *need = kk;
-    *eq = eqc;
-    return prefix;
-}
-
-// Keep, in place, the items of (s, id, ps)[0, n) whose (key, id) pass `take`;
-// they end up in [0, sh.count2) in no particular order.  Items move in rounds
-// of kRound per thread: every thread holds its items of a round in registers
-// before any thread writes, and since no more items are kept than were read,
-// a kept item never lands past the round it came from.
-constexpr int kRound = 4;
-
-template <typename Take>
-__device__ void filter_in_place(float* s, int* id, int* ps, int n, SelShared& sh, Take&& take) {
-    if (threadIdx.x == 0) sh.count2 = 0;
-    __syncthreads();
-    const int T = blockDim.x;
-    for (int r0 = 0; r0 < n; r0 += kRound * T) {
-        float vs[kRound];
-        int vi[kRound], vp[kRound];
-        bool tk[kRound];
-#pragma unroll
-        for (int j = 0; j < kRound; ++j) {
-            const int i = r0 + j * T + (int)threadIdx.x;
-            tk[j] = false;
-            vs[j] = 0.f;
-            vi[j] = vp[j] = 0;
-            if (i < n) {
-                vs[j] = s[i];
-                vi[j] = id[i];
-                vp[j] = ps[i];
-                tk[j] = take(fkey(vs[j]), vi[j]);
-            }
-        }
-        __syncthreads();   // the whole round is in registers
-#pragma unroll
-        for (int j = 0; j < kRound; ++j) {
-            if (tk[j]) {
-                const int p = atomicAdd(&sh.count2, 1);
-                s[p] = vs[j];
-                id[p] = vi[j];
-                ps[p] = vp[j];
-            }
-        }
-        __syncthreads();
-    }
-}
-
-// General form: exact k-th key by 8-bit radix passes, then ties by id.
-__device__ void topk_compact_radix(float* s, int* id, int* ps, int n, int k, SelShared& sh) {
-    int need, eq;
-    const uint32_t T = block_kth(s, id, n, k, 0, 0u, sh, &need, &eq);
-    const bool split = need < eq;
-    uint32_t T2 = 0;
-    if (split) {
-        int need2, eq2;
-        T2 = block_kth(s, id, n, need, 1, T, sh, &need2, &eq2);
-    }
-    if (threadIdx.x == 0) sh.thr = T;
-    filter_in_place(s, id, ps, n, sh, [&](uint32_t key, int xi) {
-        return key > T || (key == T && (!split || ~(uint32_t)xi >= T2));
-    });
-}
-
-// Keep, in place, the top k of the n items in (s, id, ps) by (score desc, id
-// asc), k < n; the result is (s, id, ps)[0..k) in no particular order.  The
-// keys are binned by their offset from the smallest key, shifted so that at
-// most 256 bins are used (monotone in the key); bins above the one that holds
-// the k-th item are taken whole, and that bin's items are ranked exactly by
-// (key, id).  If that bin holds more than kResolveCap items (or all keys are
-// equal), the general radix select runs instead.
-__device__ void topk_compact(float* s, int* id, int* ps, int n, int k, SelShared& sh) {
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5, nw = blockDim.x >> 5;
-    uint32_t kmn = 0xffffffffu, kmx = 0u;
-    for (int i = tid; i < n; i += blockDim.x) {
-        const uint32_t key = fkey(s[i]);
-        kmn = min(kmn, key);
-        kmx = max(kmx, key);
-    }
-#pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) {
-        kmn = min(kmn, __shfl_xor_sync(0xffffffffu, kmn, o));
-        kmx = max(kmx, __shfl_xor_sync(0xffffffffu, kmx, o));
-    }
-    if (lane == 0) { sh.wmin[warp] = kmn; sh.wmax[warp] = kmx; }
-    if (tid == 0) sh.nres = 0;
-    __syncthreads();
-    kmn = sh.wmin[0];
-    kmx = sh.wmax[0];
-    for (int w = 1; w < nw; ++w) {
-        kmn = min(kmn, sh.wmin[w]);
-        kmx = max(kmx, sh.wmax[w]);
-    }
-    if (kmn == kmx) {
-        topk_compact_radix(s, id, ps, n, k, sh);
-        return;
-    }
-    const int shift = max(0, 24 - __clz(kmx - kmn));   // (kmx - kmn) >> shift <= 255
-    for (int i = tid; i < n; i += blockDim.x) atomicAdd(&sh.hist[(fkey(s[i]) - kmn) >> shift], 1);
-    __syncthreads();
-    if (warp == 0) {
-        int c[8], sum = 0;
-#pragma unroll
-        for (int t = 0; t < 8; ++t) {
-            c[t] = sh.hist[255 - lane * 8 - t];
-            sh.hist[255 - lane * 8 - t] = 0;
-            sum += c[t];
-        }
-        const int incl = warp_incl_scan(sum);
-        const int excl = incl - sum;
-        if (excl < k && k <= incl) {
-            int run = excl;
-#pragma unroll
-            for (int t = 0; t < 8; ++t) {
-                if (run + c[t] >= k) {
-                    sh.bc[0] = 255 - lane * 8 - t;   // bin B of the k-th item
-                    sh.bc[1] = k - run;              // items of B in the top k
-                    sh.bc[2] = c[t];                 // items in B
-                    break;
-                }
-                run += c[t];
-            }
-        }
-    }
-    __syncthreads();
-    const uint32_t B = (uint32_t)sh.bc[0];
-    const int need = sh.bc[1], cntB = sh.bc[2];
-    const bool all_b = need == cntB;
-    if (!all_b && cntB > min(kResolveCap, k)) {
-        topk_compact_radix(s, id, ps, n, k, sh);
-        return;
-    }
-    // bin B's items, to be ranked among themselves (keys are distinct: ids
-    // are), listed in the histogram's storage (all zero again afterwards)
-    uint32_t* const rkey = reinterpret_cast<uint32_t*>(sh.hist);
-    int* const rid = sh.hist + kResolveCap;
-    if (!all_b) {
-        for (int i = tid; i < n; i += blockDim.x) {
-            const uint32_t key = fkey(s[i]);
-            if (((key - kmn) >> shift) == B) {
-                const int r = atomicAdd(&sh.nres, 1);
-                rkey[r] = key;
-                rid[r] = id[i];
-            }
-        }
-    }
-    if (tid == 0) sh.thr = kmn + (B << shift);   // smallest key that falls in bin B
-    // (filter_in_place's first barrier publishes the bin-B list and thr)
-    filter_in_place(s, id, ps, n, sh, [&](uint32_t key, int xi) {
-        const uint32_t b = (key - kmn) >> shift;
-        if (b != B) return b > B;
-        if (all_b) return true;
-        int rank = 0;
-        for (int j = 0; j < cntB; ++j) {
-            const uint32_t yk = rkey[j];
-            rank += yk > key || (yk == key && rid[j] < xi);
-        }
-        return rank < need;
-    });
-    if (!all_b) {
-        // (filter_in_place ended with a barrier: nobody reads the list any more;
-        // the next user of the histogram is behind further barriers)
-        for (int e = tid; e < 2 * kResolveCap; e += blockDim.x) sh.hist[e] = 0;
-    }
-}
-
-// Exclusive scan of pre[0..n) in place (values are counts), pre[n] = total.
-__device__ void scan_pre(int* pre, int n) {
-    __syncthreads();
-    if (threadIdx.x < 32) {
-        const int lane = threadIdx.x;
-        int carry = 0;
-        for (int base = 0; base < n; base += 32) {
-            const int v = (base + lane < n) ? pre[base + lane] : 0;
-            const int incl = warp_incl_scan(v);
-            if (base + lane < n) pre[base + lane] = carry + incl - v;
-            carry += __shfl_sync(0xffffffffu, incl, 31);
-        }
-        if (lane == 0) pre[n] = carry;
-    }
-    __syncthreads();
-}
-
-__device__ __forceinline__ int find_owner(const int* pre, int nk, int t) {
-    int lo = 0, hi = nk;  // pre[lo] <= t < pre[hi]
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (pre[mid] <= t) lo = mid; else hi = mid;
-    }
-    return lo;
-}
 
 // THREADS = kSelThreads for large grids; small grids (decode: a few queries)
 // give each (query, KV head) kWideThreads so the few CTAs use more of the SM.
@@ -361,7 +78,7 @@ constexpr int kWideCap = 8192;
 
 // COUNT: also add the number of eligible rows scored to *a.work (a separate
 // instantiation, so the counting costs the timed path nothing)
-template <int R, bool FULL, int THREADS, bool COUNT>
+template <int R, bool FULL, int THREADS, bool COUNT, bool SCORED = false>
 __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BLOCKS : 1) void select_kernel(
     const SelArgs a) {
     extern __shared__ float4 dyn4[];
@@ -377,8 +94,6 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
     constexpr int LPC = R / 16;             // lanes per candidate row (16 floats each)
     constexpr int CPW = 32 / LPC;           // candidates per warp
     constexpr int NG = (THREADS / 32) * CPW;
-    // ids sorted in registers: 512 for the narrow CTAs
-    constexpr int kSortIpt = THREADS >= 512 ? 1 : (512 / THREADS > 4 ? 512 / THREADS : 4);
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane / LPC, gl = lane % LPC, gid = warp * CPW + g;
     const unsigned gmask = (LPC == 32) ? 0xffffffffu : (((1u << LPC) - 1u) << (g * LPC));
@@ -388,7 +103,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
     const int64_t bseq = u / a.hkv;
     const int h = u % a.hkv;
     const int64_t row = (bseq * a.nq + qi) * a.hkv + h;
-    const int64_t pos = a.q_pos ? a.q_pos[bseq * a.nq + qi] : a.q_pos0 + qi;
+    const int64_t pos = (a.q_pos ? a.q_pos[bseq * a.nq + qi] : a.q_pos0 + qi) - a.pos_shift;
     const int64_t bound = pos - a.window - a.pool + 1;
     const int64_t b_lo = (a.sink + a.pool - 1) / a.pool;
     const int64_t b_hi = bound >= 0 ? bound / a.pool : -1;
@@ -426,7 +141,10 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
     if (threadIdx.x == 0) { sh.count = 0; sh.nkept = 0; sh.thr = 0u; }
     __syncthreads();
 
-    unsigned nscored = 0;   // eligible candidates this thread's group scored (leader lanes)
+    // eligible candidates this thread's group scored (leader lanes): tree nodes
+    // while phase is 0, candidate blocks once it is 1
+    unsigned nsc_node = 0, nsc_blk = 0;
+    int phase = FULL ? 1 : 0;
     uint32_t lt_mask;
     asm("mov.u32 %0, %%lanemask_lt;" : "=r"(lt_mask));
     // Push candidates t in [0, total) through the buffer, keeping the top k.
@@ -468,7 +186,10 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
                 for (int v = 0; v < kUnroll; ++v) {
                     if (ok[v]) {
                         sc[v] = dot(y[v]);
-                        if (COUNT) nscored += (gl == 0);
+                        if (COUNT) {
+                            if (phase) nsc_blk += (gl == 0);
+                            else nsc_node += (gl == 0);
+                        }
                         ok[v] = fkey(sc[v]) >= thr;
                     }
                     bal[v] = __ballot_sync(0xffffffffu, ok[v] && gl == 0);
@@ -591,6 +312,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
         scan_pre(pre, nk);
         if (threadIdx.x == 0) sh.count = 0;
         __syncthreads();
+        phase = 1;
         stream_topk(pre[nk], a.kb, [&](int t, OwnerState* state, bool* el, int* id, int* p, float* y) {
             const int64_t slot = slot_of(t, nk, state);
             load_row(a.Klp + slot * R, y);
@@ -612,129 +334,30 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
         });
     }
     const int nsel = sh.count;
-
-    // ascending block ids
-    int* arr = bp;   // the positions are no longer needed
-    if (THREADS >= 512) {
-        // wide CTAs: rank sort (each id counts the smaller ones), one barrier
-        const int* src = bi;
-        for (int e = threadIdx.x; e < nsel; e += THREADS) {
-            const int x = src[e];
-            int rank = 0;
-            for (int j = 0; j < nsel; ++j) rank += src[j] < x;
-            arr[rank] = x;
+    if (SCORED) {
+        // the chosen blocks with their scores, block ids shifted to the caller's numbering
+        float* os = a.out_score + row * a.kb_cap;
+        int32_t* ob = a.out_block + row * a.kb_cap;
+        for (int e = threadIdx.x; e < a.kb_cap; e += blockDim.x) {
+            os[e] = e < nsel ? bs[e] : -INFINITY;
+            ob[e] = e < nsel ? bi[e] + a.blk_shift : -1;
         }
-        __syncthreads();
-    } else if (nsel <= kSortIpt * THREADS) {
-        // bitonic sort of IPT * THREADS items (padded with INT32_MAX), IPT per
-        // thread in registers: item i = IPT tid + k; strides below IPT inside
-        // a thread, up to 16 IPT across lanes by shuffles, 32 IPT and up
-        // through shared memory
-        constexpr int IPT = kSortIpt;
-        constexpr int M = IPT * THREADS;
-        int v[IPT];
-        const int* src = bi;
-#pragma unroll
-        for (int k = 0; k < IPT; ++k) {
-            const int i = IPT * threadIdx.x + k;
-            v[k] = i < nsel ? src[i] : INT32_MAX;
-        }
-        __syncthreads();   // src and arr may be read and written below
-        for (int size = 2; size <= M; size <<= 1) {
-            for (int stride = size >> 1; stride > 0; stride >>= 1) {
-                if (stride >= 32 * IPT) {
-#pragma unroll
-                    for (int k = 0; k < IPT; ++k) arr[IPT * threadIdx.x + k] = v[k];
-                    __syncthreads();
-#pragma unroll
-                    for (int k = 0; k < IPT; ++k) {
-                        const int i = IPT * threadIdx.x + k;
-                        const int y = arr[i ^ stride];
-                        const bool asc = (i & size) == 0;
-                        const bool lower = (i & stride) == 0;
-                        v[k] = (lower == asc) ? min(v[k], y) : max(v[k], y);
-                    }
-                    __syncthreads();
-                } else if (stride >= IPT) {
-#pragma unroll
-                    for (int k = 0; k < IPT; ++k) {
-                        const int i = IPT * threadIdx.x + k;
-                        const int y = __shfl_xor_sync(0xffffffffu, v[k], stride / IPT);
-                        const bool asc = (i & size) == 0;
-                        const bool lower = (i & stride) == 0;
-                        v[k] = (lower == asc) ? min(v[k], y) : max(v[k], y);
-                    }
-                } else {
-                    // pairs (k, k + stride) inside the thread; every stride is
-                    // unrolled so every register index is a constant
-#pragma unroll
-                    for (int st = IPT / 2; st >= 1; st >>= 1) {
-                        if (st != stride) continue;
-#pragma unroll
-                        for (int k = 0; k < IPT; ++k) {
-                            if (k & st) continue;
-                            const bool asc = ((IPT * (int)threadIdx.x + k) & size) == 0;
-                            const int lo = min(v[k], v[k + st]), hi = max(v[k], v[k + st]);
-                            v[k] = asc ? lo : hi;
-                            v[k + st] = asc ? hi : lo;
-                        }
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int k = 0; k < IPT; ++k) arr[IPT * threadIdx.x + k] = v[k];
-        __syncthreads();
-    } else {
-        // bitonic sort, padded to a power of two
-        int M = 1;
-        while (M < nsel) M <<= 1;
-        for (int e = threadIdx.x; e < M; e += blockDim.x) arr[e] = e < nsel ? bi[e] : INT32_MAX;
-        __syncthreads();
-        for (int size = 2; size <= M; size <<= 1) {
-            for (int stride = size >> 1; stride > 0; stride >>= 1) {
-                for (int t = threadIdx.x; t < (M >> 1); t += blockDim.x) {
-                    const int i = 2 * stride * (t / stride) + (t % stride);
-                    const int j = i + stride;
-                    const bool asc = (i & size) == 0;
-                    const int x = arr[i], y = arr[j];
-                    if ((x > y) == asc) { arr[i] = y; arr[j] = x; }
-                }
-                __syncthreads();
-            }
-        }
+        if (threadIdx.x == 0) a.out_n[row] = nsel;
+        return;
     }
-
-    // row = sink [0, ns) | blocks (P tokens each, ascending) | window [lo_w, pos] | -1 padding;
-    // positions fit in int32 (checked by the caller), so no 64-bit division here
-    const int lo_w = (int)max((int64_t)0, pos - a.window + 1);
-    const int ns = min(a.sink, lo_w);
-    const int nblk_tok = nsel * a.pool;
-    const int total = ns + nblk_tok + ((int)pos - lo_w + 1);
-    int32_t* out = a.idx + row * a.max_sel;
-    // (consecutive threads write consecutive entries: the row is written coalesced)
-    const unsigned P = (unsigned)a.pool;
-    for (int e = threadIdx.x; e < a.max_sel; e += blockDim.x) {
-        int v;
-        if (e < ns) {
-            v = e;
-        } else if (e < ns + nblk_tok) {
-            const unsigned t = (unsigned)(e - ns);
-            const unsigned j = t / P;
-            v = arr[j] * a.pool + (int)(t - j * P);
-        } else if (e < total) {
-            v = lo_w + (e - ns - nblk_tok);
-        } else {
-            v = -1;
-        }
-        out[e] = v;
-    }
-    if (threadIdx.x == 0) a.cnt[row] = (int32_t)total;
+    emit_row<THREADS>(bi, bp, nsel, pos, a.sink, a.window, a.pool, a.max_sel, a.idx + row * a.max_sel,
+                      a.cnt + row);
     if (COUNT) {
-        unsigned long long w = nscored;
+        unsigned long long wn = nsc_node, wb = nsc_blk;
 #pragma unroll
-        for (int o = 16; o >= 1; o >>= 1) w += __shfl_xor_sync(0xffffffffu, w, o);
-        if (lane == 0) atomicAdd(a.work, w);
+        for (int o = 16; o >= 1; o >>= 1) {
+            wn += __shfl_xor_sync(0xffffffffu, wn, o);
+            wb += __shfl_xor_sync(0xffffffffu, wb, o);
+        }
+        if (lane == 0) {
+            atomicAdd(a.work, wn);
+            atomicAdd(a.work + 1, wb);
+        }
     }
 }
 
@@ -742,7 +365,9 @@ template <int R, int THREADS>
 int launch_select_t(const SelArgs& a, int64_t nq, int64_t units, bool fullscan, cudaStream_t s) {
     const size_t smem = (size_t)a.cap * 12 + (size_t)(3 * a.beam + 1) * 4;
     auto kern = fullscan ? select_kernel<R, true, THREADS, false>
-                         : (a.work ? select_kernel<R, false, THREADS, true> : select_kernel<R, false, THREADS, false>);
+                         : (a.work ? select_kernel<R, false, THREADS, true>
+                                   : (a.out_score ? select_kernel<R, false, THREADS, false, true>
+                                                  : select_kernel<R, false, THREADS, false>));
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_status(e);
     if (THREADS == kSelThreads) {
@@ -777,11 +402,72 @@ int launch_select_r(const SelArgs& a, int64_t nq, int64_t units, bool fullscan, 
     return launch_select_t<R, kSelThreads>(a, nq, units, fullscan, s);
 }
 
+// ------------------------------------------------------------ shard merge
+// Selection rows from per-shard picks (context parallelism): per (query, KV
+// head) row, the union of every part's scored blocks, its top kb by (score
+// desc, block asc) with the same compaction as the tree search, then the row
+// of emit_row.  One CTA per row.
+constexpr int kMergeThreads = 256;
+
+struct MergeArgs {
+    int parts, kb_cap, kb, hkv, pool, sink, window, max_sel, cap;
+    int64_t rows, nq, q_pos0;
+    const float* score;
+    const int32_t* block;
+    const int32_t* count;
+    const int64_t* q_pos;
+    int32_t* idx;
+    int32_t* cnt;
+};
+
+__global__ __launch_bounds__(kMergeThreads) void merge_select_kernel(const MergeArgs m) {
+    extern __shared__ float4 dyn4[];
+    __shared__ SelShared sh;
+    __shared__ int part_off[65];
+    float* const bs = reinterpret_cast<float*>(dyn4);
+    int* const bi = reinterpret_cast<int*>(bs + m.cap);
+    int* const bp = reinterpret_cast<int*>(bs + 2 * m.cap);
+    const int64_t row = blockIdx.x;
+    const int64_t bseq = row / ((int64_t)m.nq * m.hkv);
+    const int64_t qi = (row / m.hkv) % m.nq;
+    const int64_t pos = m.q_pos ? m.q_pos[bseq * m.nq + qi] : m.q_pos0 + qi;
+    for (int e = threadIdx.x; e < 256; e += blockDim.x) sh.hist[e] = 0;
+    if (threadIdx.x == 0) {
+        int acc = 0;
+        for (int p = 0; p < m.parts; ++p) {
+            part_off[p] = acc;
+            const int c = m.count[(int64_t)p * m.rows + row];
+            acc += c < 0 ? 0 : (c > m.kb_cap ? m.kb_cap : c);
+        }
+        part_off[m.parts] = acc;
+    }
+    __syncthreads();
+    const int n = part_off[m.parts];
+    for (int t = threadIdx.x; t < m.parts * m.kb_cap; t += blockDim.x) {
+        const int p = t / m.kb_cap, e = t % m.kb_cap;
+        if (part_off[p] + e < part_off[p + 1]) {
+            const int64_t src = ((int64_t)p * m.rows + row) * m.kb_cap + e;
+            bs[part_off[p] + e] = m.score[src];
+            bi[part_off[p] + e] = m.block[src];
+            bp[part_off[p] + e] = 0;
+        }
+    }
+    __syncthreads();
+    int nsel = n;
+    if (n > m.kb) {
+        topk_compact(bs, bi, bp, n, m.kb, sh);
+        nsel = m.kb;
+    }
+    __syncthreads();
+    emit_row<kMergeThreads>(bi, bp, nsel, pos, m.sink, m.window, m.pool, m.max_sel, m.idx + row * m.max_sel,
+                            m.cnt + row);
+}
+
 }  // namespace
 
 int launch_select(const lsa_index* ix, const lsa_select_params* sp, const float* qbar, int64_t nq,
                   const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt, int max_sel, bool fullscan,
-                  cudaStream_t s, unsigned long long* work) {
+                  cudaStream_t s, unsigned long long* work, const ScoredOut* scored) {
     const lsa_build_params& p = ix->p;
     if (sp->beam > 1024) return LSA_ERR_INVALID_ARG;
     SelArgs a{};
@@ -814,6 +500,14 @@ int launch_select(const lsa_index* ix, const lsa_select_params* sp, const float*
     a.cnt = cnt;
     a.max_sel = max_sel;
     a.work = work;
+    if (scored) {
+        a.pos_shift = scored->pos_shift;
+        a.blk_shift = scored->blk_shift;
+        a.kb_cap = scored->kb_cap;
+        a.out_score = scored->score;
+        a.out_block = scored->block;
+        a.out_n = scored->n;
+    }
     const int kmax = a.kb > a.beam ? a.kb : a.beam;
     int cap = 1024;
     while (cap < 2 * kmax) cap <<= 1;
@@ -826,6 +520,43 @@ int launch_select(const lsa_index* ix, const lsa_select_params* sp, const float*
         case 128: return launch_select_r<128>(a, nq, ix->units, fullscan, s);
         default: return LSA_ERR_INVALID_ARG;
     }
+}
+
+}  // namespace lsa
+
+namespace lsa {
+
+int launch_merge_selection(int parts, const float* score, const int32_t* block, const int32_t* count, int kb_cap,
+                           int64_t batch, int64_t nq, int hkv, const int64_t* q_pos, int64_t q_pos0, int pool,
+                           int kb, int sink, int window, int32_t* idx, int32_t* cnt, int max_sel, cudaStream_t s) {
+    MergeArgs m{};
+    m.parts = parts;
+    m.kb_cap = kb_cap;
+    m.kb = kb;
+    m.hkv = hkv;
+    m.pool = pool;
+    m.sink = sink;
+    m.window = window;
+    m.max_sel = max_sel;
+    int cap = 1024;
+    while (cap < parts * kb_cap) cap <<= 1;
+    m.cap = cap;
+    m.rows = batch * nq * hkv;
+    m.nq = nq;
+    m.q_pos0 = q_pos0;
+    m.score = score;
+    m.block = block;
+    m.count = count;
+    m.q_pos = q_pos;
+    m.idx = idx;
+    m.cnt = cnt;
+    if (m.rows <= 0) return LSA_OK;
+    const size_t smem = (size_t)cap * 12;
+    cudaError_t e = cudaFuncSetAttribute(merge_select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_status(e);
+    note_launch();
+    merge_select_kernel<<<(unsigned)m.rows, kMergeThreads, smem, s>>>(m);
+    return cuda_status(cudaGetLastError());
 }
 
 }  // namespace lsa

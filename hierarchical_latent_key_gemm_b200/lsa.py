@@ -69,7 +69,7 @@ _SIGS = {
     "lsa_pca_map": (_i32, [_vp, _i64, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp, _vp]),
     "lsa_project_pool": (_i32, [_vp, _vp, _i64, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
     "lsa_query_latent": (_i32, [_vp, _vp, _i64, _i64, _i32, _i32, _i32, _i32, _i32, _vp, _vp]),
-    "lsa_kmeans": (_i32, [_vp, _i64, _i64, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp]),
+    "lsa_kmeans": (_i32, [_vp, _i64, _i64, _i32, _i32, _i32, _i32, _vp, _vp, _vp, _vp, _vp]),
     "lsa_index_get": (_i32, [_vp, _i32, _i32, _vp, _i64, _vp]),
     "lsa_index_info": (_i32, [_vp, C.POINTER(IndexInfo)]),
     "lsa_check": (_i32, [_vp, _vp]),
@@ -77,6 +77,12 @@ _SIGS = {
     "lsa_strerror": (C.c_char_p, [_i32]),
     "lsa_debug_fail_alloc_after": (None, [_i32]),
     "lsa_launch_count": (_i64, []),
+    "lsa_select_blocks": (_i32, [_vp, C.POINTER(SelectParams), _vp, _i64, _vp, _i64, _i64, _vp, _vp, _vp, _i32,
+                                 _vp]),
+    "lsa_merge_selection": (_i32, [_i32, _vp, _vp, _vp, _i32, _i64, _i64, _i32, _vp, _i64, _i32, _i32, _i32, _i32,
+                                   _vp, _vp, _i32, _vp]),
+    "lsa_localize_rows": (_i32, [_vp, _vp, _i64, _i32, _i64, _i64, _vp, _vp, _vp]),
+    "lsa_merge_attn": (_i32, [_i32, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp]),
 }
 
 _lib = None
@@ -309,16 +315,17 @@ def lsa_select_noalloc(index, sp, Q, idx, cnt, q_pos=None, q_pos0=0, stream=None
 
 
 def lsa_select_work(index, sp, Q, q_pos=None, q_pos0=0, idx=None, cnt=None, max_sel=None, stream=None):
-    """lsa_select plus the number of eligible nodes and blocks whose latent
-    rows were scored (a Python int; synchronises the stream)."""
-    scored = torch.zeros(1, dtype=torch.int64, device=Q.device)
+    """lsa_select plus the numbers of eligible tree nodes and of candidate
+    blocks whose latent rows were scored: returns (idx, cnt, nodes, blocks),
+    the counts as Python ints (synchronises the stream)."""
+    scored = torch.zeros(2, dtype=torch.int64, device=Q.device)
 
     def fn(h, spp, q, nq, qp, qp0, ii, cc, ms, st):
         return lib().lsa_select_work(h, spp, q, nq, qp, qp0, ii, cc, ms, _ptr(scored), st)
 
     idx, cnt = _select(fn, "lsa_select_work", index, sp, Q, q_pos=q_pos, q_pos0=q_pos0, idx=idx, cnt=cnt,
                        max_sel=max_sel, stream=stream)
-    return idx, cnt, int(scored.item())
+    return idx, cnt, int(scored[0].item()), int(scored[1].item())
 
 
 def lsa_fullscan_select(index, sp, Q, **kw):
@@ -426,14 +433,104 @@ def lsa_query_latent(Q, W, hkv, qbar=None, stream=None):
     return qbar
 
 
-def lsa_kmeans(X, k, iters, grid_log2=0, stream=None):
+def lsa_kmeans(X, k, iters, grid_log2=0, C_init=None, stream=None):
+    """Lloyd k-means of X [units, n, r] (float32); C_init [units, k, r] float32
+    or None for the stride init.  Returns (labels, centroids, objectives)."""
     U, n, r = X.shape
+    _typed(X, torch.float32, "X")
+    _shape(C_init, (U, k, r), "C_init")
     labels = torch.empty((U, n), dtype=torch.int32, device=X.device)
     Cc = torch.empty((U, k, r), dtype=torch.float32, device=X.device)
     obj = torch.empty((iters, U), dtype=torch.float64, device=X.device)
     _ok(lib().lsa_kmeans(_ptr(X), int(U), int(n), int(r), int(k), int(iters), int(grid_log2), _ptr(labels),
-                         _ptr(Cc), _ptr(obj), _stream(stream)), "lsa_kmeans")
+                         _ptr(Cc), _typed(C_init, torch.float32, "C_init"), _ptr(obj), _stream(stream)), "lsa_kmeans")
     return labels, Cc, obj
+
+
+# ------------------------------------------------------------ context parallelism
+def lsa_select_blocks(index, sp, Q, token_offset, q_pos=None, q_pos0=0, kb_cap=None, stream=None):
+    """A shard's tree search: (scores [B, nq, hkv, kb_cap] float32, blocks
+    [B, nq, hkv, kb_cap] int32 in whole-sequence block ids, count [B, nq, hkv]
+    int32); positions are whole-sequence positions."""
+    p = index.params
+    if Q.dim() != 4:
+        raise ValueError(f"Q must be [batch, nq, hq, d], got shape {tuple(Q.shape)}")
+    if dtype_code(Q) != p.dtype:
+        raise ValueError(f"Q is {Q.dtype} but the index was built for dtype {p.dtype}")
+    B, nq = p.batch, Q.shape[1]
+    _shape(Q, (B, nq, sp.hq, p.d), "Q")
+    _shape(q_pos, (B, nq), "q_pos")
+    kb = -(-sp.topk // p.pool)
+    kb_cap = kb if kb_cap is None else int(kb_cap)
+    scores = torch.empty((B, nq, p.hkv, kb_cap), dtype=torch.float32, device=Q.device)
+    blocks = torch.empty((B, nq, p.hkv, kb_cap), dtype=torch.int32, device=Q.device)
+    count = torch.empty((B, nq, p.hkv), dtype=torch.int32, device=Q.device)
+    _ok(lib().lsa_select_blocks(index.handle, C.byref(sp), _ptr(Q), int(nq), _typed(q_pos, torch.int64, "q_pos"),
+                                int(q_pos0), int(token_offset), _ptr(scores), _ptr(blocks), _ptr(count), int(kb_cap),
+                                _stream(stream)), "lsa_select_blocks")
+    return scores, blocks, count
+
+
+def lsa_merge_selection(scores, blocks, count, pool, topk, sink, window, q_pos=None, q_pos0=0, max_sel=None,
+                        idx=None, cnt=None, stream=None):
+    """Merge of the shards' picks (scores/blocks [parts, B, nq, hkv, kb_cap],
+    count [parts, B, nq, hkv]) into selection rows (idx, cnt) as lsa_select
+    writes them."""
+    parts, B, nq, hkv, kb_cap = scores.shape
+    _shape(blocks, scores.shape, "blocks")
+    _shape(count, scores.shape[:4], "count")
+    _shape(q_pos, (B, nq), "q_pos")
+    kb = -(-int(topk) // int(pool))
+    if max_sel is None:
+        max_sel = idx.shape[-1] if idx is not None else kb * pool + sink + window
+    _shape(idx, (B, nq, hkv, max_sel), "idx")
+    _shape(cnt, (B, nq, hkv), "cnt")
+    if idx is None:
+        idx = torch.empty((B, nq, hkv, max_sel), dtype=torch.int32, device=scores.device)
+    if cnt is None:
+        cnt = torch.empty((B, nq, hkv), dtype=torch.int32, device=scores.device)
+    _ok(lib().lsa_merge_selection(int(parts), _typed(scores, torch.float32, "scores"),
+                                  _typed(blocks, torch.int32, "blocks"), _typed(count, torch.int32, "count"),
+                                  int(kb_cap), int(B), int(nq), int(hkv), _typed(q_pos, torch.int64, "q_pos"),
+                                  int(q_pos0), int(pool), int(topk), int(sink), int(window),
+                                  _typed(idx, torch.int32, "idx"), _typed(cnt, torch.int32, "cnt"), int(max_sel),
+                                  _stream(stream)), "lsa_merge_selection")
+    return idx, cnt
+
+
+def lsa_localize_rows(idx, cnt, lo, hi, idx_out=None, cnt_out=None, stream=None):
+    """The entries of each selection row in [lo, hi), shifted by -lo."""
+    max_sel = idx.shape[-1]
+    rows = idx.numel() // max_sel
+    _shape(cnt, idx.shape[:-1], "cnt")
+    if idx_out is None:
+        idx_out = torch.empty_like(idx)
+    if cnt_out is None:
+        cnt_out = torch.empty_like(cnt)
+    _shape(idx_out, idx.shape, "idx_out")
+    _shape(cnt_out, cnt.shape, "cnt_out")
+    _ok(lib().lsa_localize_rows(_typed(idx, torch.int32, "idx"), _typed(cnt, torch.int32, "cnt"), int(rows),
+                                int(max_sel), int(lo), int(hi), _typed(idx_out, torch.int32, "idx_out"),
+                                _typed(cnt_out, torch.int32, "cnt_out"), _stream(stream)), "lsa_localize_rows")
+    return idx_out, cnt_out
+
+
+def lsa_merge_attn(O_parts, lse_parts, O=None, lse=None, want_lse=True, stream=None):
+    """Attention over the union of the parts' disjoint row sets: O_parts
+    [parts, B, nq, hq, d], lse_parts [parts, B, nq, hq] -> (O, lse)."""
+    parts, B, nq, hq, d = O_parts.shape
+    _shape(lse_parts, O_parts.shape[:4], "lse_parts")
+    if O is None:
+        O = torch.empty(O_parts.shape[1:], dtype=O_parts.dtype, device=O_parts.device)
+    if lse is None and want_lse:
+        lse = torch.empty((B, nq, hq), dtype=torch.float32, device=O_parts.device)
+    _shape(O, O_parts.shape[1:], "O")
+    _shape(lse, (B, nq, hq), "lse")
+    _same_dtype(O_parts, O)
+    _ok(lib().lsa_merge_attn(int(parts), _ptr(O_parts), _typed(lse_parts, torch.float32, "lse_parts"), int(B * nq),
+                             int(hq), int(d), dtype_code(O), _ptr(O), _typed(lse, torch.float32, "lse"),
+                             _stream(stream)), "lsa_merge_attn")
+    return O, lse
 
 
 def lsa_check(index: Index | None = None, stream=None) -> int:

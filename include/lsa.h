@@ -190,12 +190,13 @@ int lsa_select_noalloc(const lsa_index* index, const lsa_select_params* params, 
                        int64_t nq, const int64_t* q_pos, int64_t q_pos0,
                        int32_t* idx, int32_t* cnt, int32_t max_sel, void* stream);
 
-/* lsa_select that also adds to *scored (a device uint64 the caller zeroes)
- * the number of eligible tree nodes and candidate blocks whose latent rows it
- * scored, summed over all (query, KV head) pairs: the work count behind a
- * bytes-moved figure (each scored row is r floats).  Same results as
- * lsa_select; costs one atomic add per warp.  The pages give no counterpart:
- * it exists for measurement. */
+/* lsa_select that also counts the latent rows it scored, summed over all
+ * (query, KV head) pairs: scored is a device uint64[2] the caller zeroes;
+ * scored[0] += eligible tree nodes scored (centroid rows), scored[1] +=
+ * candidate blocks scored (latent key rows).  These are the work counts behind
+ * a bytes-moved figure (each scored row is r values).  Same results as
+ * lsa_select; costs two atomic adds per warp.  The pages give no
+ * counterpart: it exists for measurement. */
 int lsa_select_work(const lsa_index* index, const lsa_select_params* params, const void* Q,
                     int64_t nq, const int64_t* q_pos, int64_t q_pos0,
                     int32_t* idx, int32_t* cnt, int32_t max_sel, unsigned long long* scored,
@@ -227,6 +228,75 @@ int lsa_pca_map(const void* K, int64_t batch, int64_t n_tokens, int64_t ld_token
 int lsa_fullscan_select(const lsa_index* index, const lsa_select_params* params, const void* Q,
                         int64_t nq, const int64_t* q_pos, int64_t q_pos0,
                         int32_t* idx, int32_t* cnt, int32_t max_sel, void* stream);
+
+/* ---------------------------------------------------------------------
+ * Context parallelism: one sequence's context split over shards (GPUs).
+ * The pages say only that the 10M-token runs split one sequence over several
+ * GPUs ([p5] "What do 22.7x and 72.4x actually compare?", "Can I run
+ * LSA?").  Reading used here: shard s holds the block-aligned token range
+ * [t0_s, t1_s) of K and V and its own index over it (built with
+ * sink = max(0, S - t0_s), so the sink rule stays the global one); every
+ * shard picks its local top ceil(K/P) blocks with their scores
+ * (lsa_select_blocks); the picks of all shards are merged into the global top
+ * ceil(K/P) by (score desc, block asc), and the selection row is written as
+ * lsa_select writes it (lsa_merge_selection); each shard attends the rows of
+ * that selection it holds (lsa_localize_rows + lsa_sparse_attn, with lse) and
+ * the parts are combined by their log-sum-exps (lsa_merge_attn).  The
+ * collectives between the steps (an all-gather of the picks, an all-gather of
+ * the attention parts) are the caller's (NCCL through torch.distributed in
+ * the Python package). */
+
+/* The tree search of lsa_select on one shard, returning the chosen blocks
+ * with their scores instead of a selection row.
+ *  index: the shard's index (tokens of the shard in its own positions 0..).
+ *  Q, nq, q_pos, q_pos0: as lsa_select, positions in the WHOLE sequence.
+ *  token_offset: the shard's first token t0 (a multiple of the pool size); a
+ *      query at position i is searched at index position i - token_offset
+ *      (negative: nothing is chosen).
+ *  scores: device float [batch][nq][hkv][kb_cap], blocks: device int32
+ *      [batch][nq][hkv][kb_cap] (block ids in the whole sequence, i.e. index
+ *      block + t0/P), count: device int32 [batch][nq][hkv]: entries
+ *      [0, count) hold the chosen blocks in no particular order; the rest
+ *      are -inf / -1.  kb_cap >= ceil(K/P).
+ * Same rules, arithmetic and ties as lsa_select.  Stream-ordered scratch as
+ * lsa_select. */
+int lsa_select_blocks(const lsa_index* index, const lsa_select_params* params, const void* Q, int64_t nq,
+                      const int64_t* q_pos, int64_t q_pos0, int64_t token_offset, float* scores, int32_t* blocks,
+                      int32_t* count, int32_t kb_cap, void* stream);
+
+/* Merge of the shards' picks into selection rows.
+ *  scores, blocks, count: device, parts x the layouts of lsa_select_blocks
+ *      (part p at offset p * batch * nq * hkv rows); 1 <= parts <= 64,
+ *      parts * kb_cap <= 16384.  Block ids must be distinct within a row.
+ *  q_pos / q_pos0: positions of the queries in the whole sequence.
+ *  idx, cnt, max_sel: as lsa_select (max_sel >= ceil(K/P)*P + S + W).
+ * Per (query, KV head): the top ceil(K/P) of the union of the parts by
+ * (score desc, block asc), then the row sink | tokens of the chosen blocks |
+ * window, ascending, -1 after, as lsa_select. */
+int lsa_merge_selection(int32_t parts, const float* scores, const int32_t* blocks, const int32_t* count,
+                        int32_t kb_cap, int64_t batch, int64_t nq, int32_t hkv, const int64_t* q_pos, int64_t q_pos0,
+                        int32_t pool, int32_t topk, int32_t sink, int32_t window, int32_t* idx, int32_t* cnt,
+                        int32_t max_sel, void* stream);
+
+/* The entries of selection rows that fall in [lo, hi), shifted by -lo, in
+ * order: rows of the caller's shard in the shard's own token positions.
+ *  idx, cnt: device [rows][max_sel] and [rows] (entries past cnt ignored);
+ *  idx_out, cnt_out: device, same shapes; idx_out may be idx itself, or must
+ *  not overlap it.  Rows left without entries get cnt_out = 0 (lsa_sparse_attn
+ *  then gives O = 0 and lse = -inf for them). */
+int lsa_localize_rows(const int32_t* idx, const int32_t* cnt, int64_t rows, int32_t max_sel, int64_t lo, int64_t hi,
+                      int32_t* idx_out, int32_t* cnt_out, void* stream);
+
+/* Attention over a union of disjoint row sets from its parts:
+ *  O_parts: device [parts][rows][hq][d] of dtype (each part normalised over
+ *  its own rows), lse_parts: device float [parts][rows][hq] (natural log of
+ *  the part's softmax denominator, -inf for an empty part).
+ *  O: device [rows][hq][d]; lse: device float [rows][hq] or NULL.
+ * O = sum_s e^(lse_s - m) O_s / sum_s e^(lse_s - m), lse = m + log(sum_s
+ * e^(lse_s - m)), m = max_s lse_s (parts in order, fp32); all parts empty ->
+ * O = 0, lse = -inf.  rows = batch * nq of the attention calls. */
+int lsa_merge_attn(int32_t parts, const void* O_parts, const float* lse_parts, int64_t rows, int32_t hq, int32_t d,
+                   int32_t dtype, void* O, float* lse, void* stream);
 
 /* Exact softmax attention over selected tokens.
  *  Q: device [batch][nq][hq][d]; K, V: device [batch][ld_tokens][hkv][d];
@@ -327,12 +397,21 @@ int lsa_query_latent(const void* Q, const float* W, int64_t batch, int64_t nq, i
  *  X: device float [units][n][r]; labels: device int32 [units][n];
  *  C: device float [units][k][r] (output); objective: device double
  *  [iters][units] (sum of squared distances after each assign) or NULL.
- * Same rules as the build (stride init, ties low, empty keeps, grid). */
+ *  C_init: device float [units][k][r], the centroids the first round assigns
+ *  against, or NULL for the build's stride init (centroid j = point
+ *  floor(j*n/k)); it may not overlap C.  Starting from given centroids lets a
+ *  caller run any single Lloyd round of a longer run.
+ * Same rules as the build (ties low, empty keeps, grid). */
 int lsa_kmeans(const float* X, int64_t units, int64_t n, int32_t r, int32_t k, int32_t iters,
-               int32_t grid_log2, int32_t* labels, float* C, double* objective, void* stream);
+               int32_t grid_log2, int32_t* labels, float* C, const float* C_init, double* objective,
+               void* stream);
 
 /* Copy one array of the index to `dst` (device or host memory, dst_bytes
- * large enough; see lsa_get_what for shapes).  Synchronises `stream`. */
+ * large enough; see lsa_get_what for shapes).  Synchronises `stream`.
+ * Index statistics are read through this call and lsa_index_info: the
+ * objective after every Lloyd round of every level (LSA_GET_OBJECTIVE), the
+ * bucket sizes (LSA_GET_LEAF_COUNT), the device bytes held
+ * (lsa_index_info_t.device_bytes), and every array of the tree. */
 int lsa_index_get(const lsa_index* index, int32_t what, int32_t level, void* dst,
                   int64_t dst_bytes, void* stream);
 

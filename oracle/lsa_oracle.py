@@ -149,18 +149,23 @@ def squared_distances(X: np.ndarray, C: np.ndarray) -> np.ndarray:
     return xx - 2.0 * (X @ C.T) + cc
 
 
-def kmeans_assign(X: np.ndarray, C: np.ndarray, chunk: int = 4096):
+def kmeans_assign(X: np.ndarray, C: np.ndarray, chunk: int = 0):
     """Nearest centroid of every point, ties to the lower centroid id (R7).
-    Returns (labels int64 [n], objective = sum of the chosen squared distances)."""
+    Returns (labels int64 [n], objective = sum of the chosen squared distances).
+    Points are taken ``chunk`` at a time only to bound the size of the
+    distance matrix (default: about 4 M entries); each point's distances, its
+    argmin and the final sum do not depend on the chunking."""
     n = X.shape[0]
+    if chunk <= 0:
+        chunk = max(1, (1 << 22) // max(1, C.shape[0]))
     labels = np.empty(n, dtype=np.int64)
-    obj = 0.0
+    dmin = np.empty(n, dtype=np.float64)
     for s in range(0, n, chunk):
         d2 = squared_distances(X[s : s + chunk], C)
         lab = np.argmin(d2, axis=1)  # first minimum = lower id
         labels[s : s + chunk] = lab
-        obj += float(d2[np.arange(d2.shape[0]), lab].sum())
-    return labels, obj
+        dmin[s : s + chunk] = d2[np.arange(d2.shape[0]), lab]
+    return labels, float(dmin.sum())
 
 
 def _round_half_even_div(s: np.ndarray, n: np.ndarray) -> np.ndarray:
@@ -215,8 +220,10 @@ class KMeansResult:
     objectives: list            # objective after every assign, len = iters
 
 
-def kmeans(X: np.ndarray, k: int, iters: int, grid_log2: int = 0) -> KMeansResult:
-    """``iters`` Lloyd rounds of (assign, update) from the stride init (R9, R10)."""
+def kmeans(X: np.ndarray, k: int, iters: int, grid_log2: int = 0, history: list | None = None) -> KMeansResult:
+    """``iters`` Lloyd rounds of (assign, update) from the stride init (R9, R10).
+    With ``history`` (a list), every round appends (centroids it assigned
+    against, labels, centroids after the update), for round-by-round checks."""
     X = np.asarray(X, dtype=np.float64)
     C = kmeans_init(X, k)
     objectives = []
@@ -224,7 +231,10 @@ def kmeans(X: np.ndarray, k: int, iters: int, grid_log2: int = 0) -> KMeansResul
     for _ in range(iters):
         labels, obj = kmeans_assign(X, C)
         objectives.append(obj)
-        C = kmeans_update(X, labels, C, grid_log2)
+        C_next = kmeans_update(X, labels, C, grid_log2)
+        if history is not None:
+            history.append((C, labels, C_next))
+        C = C_next
     return KMeansResult(labels, C, objectives)
 
 
@@ -289,12 +299,13 @@ class Tree:
 
 
 def build_tree(Kl: np.ndarray, level_sizes, iters: int, grid_log2: int,
-               sink: int, pool: int) -> Tree:
+               sink: int, pool: int, leaf_history: list | None = None) -> Tree:
     """Leaf k-means over the latent keys, then k-means of each level's
-    centroids into the level above (R10).  ``level_sizes`` is top first."""
+    centroids into the level above (R10).  ``level_sizes`` is top first.
+    ``leaf_history``: see ``kmeans`` (the leaf level's rounds)."""
     level_sizes = list(level_sizes)
     L = len(level_sizes)
-    res = kmeans(Kl, level_sizes[-1], iters, grid_log2)
+    res = kmeans(Kl, level_sizes[-1], iters, grid_log2, leaf_history)
     centroids = [None] * L
     parent = [None] * L
     objectives = [None] * L
@@ -455,3 +466,85 @@ def append_block(tree: Tree, Kl_rows: list, x: np.ndarray) -> int:
             if l > 0:
                 node = int(tree.parent[l][node])
     return leaf
+
+
+# ---------------------------------------------------------------------------
+# Context parallelism over shards of one sequence  [p5 "What do 22.7x and
+# 72.4x actually compare?" and "Can I run LSA?": the 10M-token runs split one
+# sequence's context over several GPUs]
+#
+# Reading R20 (the pages give no algorithm for it): shard s holds the
+# contiguous token range [t0_s, t1_s) (block-aligned) and its own tree, built
+# from its latent keys alone with the sink rule in global positions (a block is
+# a candidate iff it starts at or after S globally).  A query selects in every
+# shard the local top ceil(K/P) blocks by the tree search of ``select_blocks``
+# (positions shifted by t0_s); the selection is the top ceil(K/P) of the union
+# of the shards' picks by (score desc, global block asc), expanded to tokens
+# with the sink and the window as in ``selection_tokens``.  Attention over it
+# is computed per shard on the shard's rows and merged by the log-sum-exp
+# rule, which equals attention over the whole selection.
+# ---------------------------------------------------------------------------
+def shard_ranges(n_tokens: int, world: int, pool: int):
+    """Contiguous token ranges [t0, t1) of ``world`` shards, each starting on a
+    block boundary; the first shards get one block more when blocks do not
+    divide evenly, and the last one also takes the partial block at the end."""
+    nb = n_tokens // pool
+    out = []
+    b0 = 0
+    for s in range(world):
+        nbs = nb // world + (1 if s < nb % world else 0)
+        t0 = b0 * pool
+        t1 = (b0 + nbs) * pool if s < world - 1 else n_tokens
+        out.append((t0, t1))
+        b0 += nbs
+    return out
+
+
+def local_sink(sink: int, t0: int) -> int:
+    """The sink rule of a shard starting at token t0, in its own positions."""
+    return max(0, sink - t0)
+
+
+def scored_blocks(tree: Tree, Kl: np.ndarray, qbar: np.ndarray, i: int, beam: int, topk: int,
+                  window: int):
+    """``select_blocks`` with the scores of the chosen blocks: returns (blocks,
+    scores), blocks ascending.  A position before the tree's first block (i < 0
+    in a shard's coordinates) chooses nothing."""
+    blocks = select_blocks(tree, Kl, qbar, i, beam, topk, window)
+    scores = np.asarray(Kl, dtype=np.float64)[blocks] @ np.asarray(qbar, dtype=np.float64)
+    return blocks, scores
+
+
+def cp_select_blocks(shards, qbar: np.ndarray, i: int, beam: int, topk: int, window: int, pool: int):
+    """R20 selection of the query at global position i.  ``shards``: list of
+    (t0, tree, Kl) with the tree over that shard's latent keys.  Returns the
+    chosen global block ids, ascending."""
+    ids, scs = [], []
+    for t0, tree, Kl in shards:
+        b, s = scored_blocks(tree, Kl, qbar, i - t0, beam, topk, window)
+        ids.append(b + t0 // pool)
+        scs.append(s)
+    ids = np.concatenate(ids) if ids else np.zeros(0, np.int64)
+    scs = np.concatenate(scs) if scs else np.zeros(0)
+    return np.sort(top_by_score(ids, scs, blocks_per_topk(topk, pool)))
+
+
+def merge_attention(outs, lses):
+    """Attention over a union of disjoint row sets from the parts computed on
+    each set: outs[s] [G, d] normalised outputs, lses[s] [G] natural-log
+    denominators (-inf for an empty part).  Returns (O [G, d], lse [G]); a query
+    whose parts are all empty gets O = 0 and lse = -inf."""
+    L = np.stack([np.asarray(x, dtype=np.float64) for x in lses])          # [S, G]
+    Os = np.stack([np.asarray(x, dtype=np.float64) for x in outs])         # [S, G, d]
+    m = L.max(axis=0)
+    G, d = Os.shape[1], Os.shape[2]
+    O = np.zeros((G, d))
+    lse = np.full(G, -INF)
+    for g in range(G):
+        if m[g] == -INF:
+            continue
+        wts = np.exp(L[:, g] - m[g])
+        den = wts.sum()
+        O[g] = (wts[:, None] * Os[:, g, :]).sum(axis=0) / den
+        lse[g] = m[g] + math.log(den)
+    return O, lse

@@ -509,3 +509,83 @@ def test_refresh_makes_each_centroid_the_mean_of_its_members():
                 np.testing.assert_array_equal(t.centroids[l][j], old[l][j])
     # the appended blocks moved some leaf: the refresh did something
     assert any(not np.array_equal(a, b) for a, b in zip(old, t.centroids))
+
+
+# ------------------------------------------------------- context parallelism
+def test_shard_ranges_worked_examples():
+    # 5 blocks of 2 over 3 shards: 2, 2, 1 blocks
+    assert O.shard_ranges(10, 3, 2) == [(0, 4), (4, 8), (8, 10)]
+    # 2 whole blocks of 4 over 2 shards; the last shard keeps the 3 trailing tokens
+    assert O.shard_ranges(11, 2, 4) == [(0, 4), (4, 11)]
+    assert O.shard_ranges(7, 1, 4) == [(0, 7)]
+    for n, world, pool in ((1000, 4, 4), (1003, 3, 2), (64, 8, 8)):
+        rs = O.shard_ranges(n, world, pool)
+        assert rs[0][0] == 0 and rs[-1][1] == n
+        assert all(a[1] == b[0] for a, b in zip(rs[:-1], rs[1:]))
+        assert all(t0 % pool == 0 for t0, _ in rs)
+        sizes = [(t1 - t0) // pool for t0, t1 in rs]
+        assert max(sizes) - min(sizes) <= 1
+
+
+def _shards(Kl_tokens_blocks, n_tokens, world, pool, sink, sizes, iters, seed_shift=0):
+    """Per-shard trees over the shards' latent keys (block rows of Kl)."""
+    out = []
+    for t0, t1 in O.shard_ranges(n_tokens, world, pool):
+        b0, b1 = t0 // pool, t1 // pool
+        Kl_s = Kl_tokens_blocks[b0:b1]
+        tree = O.build_tree(Kl_s, sizes, iters, 0, O.local_sink(sink, t0), pool)
+        out.append((t0, tree, Kl_s))
+    return out
+
+
+def test_cp_one_shard_equals_tree_selection():
+    Kl, t = _random_tree(21, nb=150, sizes=(3, 12), pool=2, sink=4)
+    rng = np.random.default_rng(5)
+    for i in (0, 9, 40, 150, 299):
+        q = rng.standard_normal(Kl.shape[1])
+        want = O.select_blocks(t, Kl, q, i, 4, 40, 8)
+        got = O.cp_select_blocks([(0, t, Kl)], q, i, 4, 40, 8, 2)
+        np.testing.assert_array_equal(got, want)
+
+
+@pytest.mark.parametrize("world,pool,sink", [(2, 2, 6), (3, 1, 0), (4, 4, 9)])
+def test_cp_full_beam_equals_global_fullscan(world, pool, sink):
+    """With a beam that keeps every node, each shard returns its own exact
+    top-K, and the merge is then the full scan over the whole sequence."""
+    rng = np.random.default_rng(world * 10 + pool)
+    n_tokens = 400 + pool - 1
+    nb = n_tokens // pool
+    Kl = rng.standard_normal((nb, 4))
+    shards = _shards(Kl, n_tokens, world, pool, sink, (2, 6), 3)
+    window, topk = 5, 24
+    for i in list(range(0, n_tokens, 37)) + [n_tokens - 1]:
+        q = rng.standard_normal(4)
+        got = O.cp_select_blocks(shards, q, i, 1000, topk, window, pool)
+        want = O.fullscan_blocks(Kl, q, i, topk, sink, window, pool)
+        np.testing.assert_array_equal(got, want)
+
+
+def test_merge_attention_equals_attention_over_the_union():
+    rng = np.random.default_rng(3)
+    N, d, G = 90, 8, 3
+    K = rng.standard_normal((N, d))
+    V = rng.standard_normal((N, d))
+    q = rng.standard_normal((G, d))
+    sel = np.sort(rng.choice(N, 50, replace=False))
+    want_o, want_l = O.sparse_attention(q, K, V, sel)
+    # split into 4 disjoint parts, one of them empty
+    cuts = [sel[sel < 20], sel[(sel >= 20) & (sel < 20)], sel[(sel >= 20) & (sel < 61)], sel[sel >= 61]]
+    outs, lses = [], []
+    for part in cuts:
+        if part.size:
+            o, l = O.sparse_attention(q, K, V, part)
+        else:
+            o, l = np.zeros((G, d)), np.full(G, -np.inf)
+        outs.append(o)
+        lses.append(l)
+    got_o, got_l = O.merge_attention(outs, lses)
+    np.testing.assert_allclose(got_o, want_o, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(got_l, want_l, rtol=0, atol=1e-12)
+    # every part empty: O = 0, lse = -inf
+    o, l = O.merge_attention([np.zeros((G, d))] * 2, [np.full(G, -np.inf)] * 2)
+    assert np.all(o == 0) and np.all(l == -np.inf)
