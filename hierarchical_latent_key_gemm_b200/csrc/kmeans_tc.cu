@@ -3,13 +3,16 @@
 // distance(x, c_j) = ||c_j||^2 - 2 x.c_j (||x||^2 is common to a row); the
 // x.c products of a 128-point tile against 256-centroid tiles are one dense
 // GEMM per tile.  Operands are fp32; each is scaled by one power of two
-// (exact; chosen from the largest magnitude so that every value fits fp16)
-// and split into two fp16 parts (x = xh + xl, c = ch + cl), and the GEMM runs
-// over K = 3r with A = [xh | xh | xl], B = [ch | cl | ch] (zero-padded to a
-// multiple of 64), so the accumulator holds xh.ch + xh.cl + xl.ch: fp16 keeps
-// 11 significant bits like tf32, so the dropped xl.cl term and the roundings
-// leave an error near 2^-21 of |x||c| (fp32-like assignments), at the f16 MMA
-// rate, twice the tf32 one.
+// (exact; chosen from the largest magnitude so that every value is below
+// 2^10) and split into two fp16 parts (x = xh + xl, c = ch + cl).  The GEMM
+// runs over K = 3r + 2 (zero-padded to a multiple of 64) with
+// A = [xh | xh | xl | 2^12 | 2^12], B = [ch | cl | ch | -nh | -nl], nh + nl =
+// |c|^2 / 2^13 split the same way, so the accumulator holds
+// x.c - |c|^2 / 2 (scaled) and the nearest centroid is the largest entry: the
+// norms ride in the product and the epilogue is one compare per entry.  fp16
+// keeps 11 significant bits like tf32, so the dropped xl.cl term and the
+// roundings leave an error near 2^-21 of |x||c| (fp32-like assignments), at
+// the f16 MMA rate, twice the tf32 one.
 //
 // One CTA per 128 points, persistent over all centroid tiles of its unit:
 //   warp 0    TMA producer: the point tile once (all K-chunks resident), then
@@ -17,8 +20,10 @@
 //   warp 1    TMEM owner and MMA issuer (one thread): tcgen05.mma kind::f16
 //             (fp16 A and B), M=128, N=256, K=16 per instruction, into one of
 //             two TMEM accumulators (2 x 256 columns)
-//   warps 2-5 epilogue: tcgen05.ld of the accumulator rows, running
-//             (distance, id) minimum per point, ties to the lower id
+//   warps 2-9 epilogue: tcgen05.ld of the accumulator rows, two warps per
+//             TMEM lane quarter (each on half of the columns), running
+//             (value, id) maximum per point, ties to the lower id, the two
+//             halves merged at the end
 // Every mbarrier wait is bounded; a timeout latches kErrTimeout and the CTA
 // winds down (TMEM is always released).
 #include <cuda_fp16.h>
@@ -35,7 +40,7 @@ constexpr int kTM = 128;          // points per CTA (UMMA M)
 constexpr int kTN = 256;          // centroids per tile (UMMA N)
 constexpr int kKC = 64;           // fp16 per K-chunk: one 128-byte swizzle row
 constexpr int kStagesB = 3;
-constexpr int kThreadsTC = 192;
+constexpr int kThreadsTC = 320;   // producer, MMA issuer, 8 epilogue warps
 // K-major operand, 128-byte swizzle: 8-row x 128-byte atoms, 1024 bytes apart.
 __device__ __forceinline__ uint64_t umma_desc(const void* p) {
     const uint64_t addr = su32(p);
@@ -60,8 +65,8 @@ __device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t a, uint64_t b
         "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate), "r"(0u));
 }
 
-// K extent of the split operands: 3r rounded up to whole 64-element chunks.
-__host__ __device__ constexpr int split_k(int r) { return (3 * r + kKC - 1) / kKC * kKC; }
+// K extent of the split operands: 3r + 2 rounded up to whole 64-element chunks.
+__host__ __device__ constexpr int split_k(int r) { return (3 * r + 2 + kKC - 1) / kKC * kKC; }
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(bar))
                  : "memory");
@@ -103,16 +108,16 @@ __global__ void absmax_kernel(const float* __restrict__ X, int64_t ldx, int64_t 
     if ((threadIdx.x & 31) == 0) atomicMax(out, m);
 }
 
-// The power of two 2^-e that brings the largest magnitude into [2^13, 2^14)
-// (|scaled value| < 2^14 fits fp16 with room for sums of parts).
+// The power of two 2^-e that brings the largest magnitude into [2^9, 2^10):
+// scaled coordinates fit fp16, and |scaled c|^2 / 2^13 <= r 2^7 does too.
 __device__ __forceinline__ int scale_exp(const uint32_t* absmax) {
     const float m = __uint_as_float(*absmax);
     if (!(m > 0.f) || isinf(m)) return 0;
-    // (clamped so that 2^(2e+1), the epilogue's factor, stays a normal float)
-    return max(-60, min(60, ilogbf(m) - 13));
+    return max(-60, min(60, ilogbf(m) - 9));
 }
 
-// Xs[u*n_pad + p] = [xh | xh | xl | 0], x scaled by 2^-e, zero rows past n.
+// Xs[u*n_pad + p] = [xh | xh | xl | 2^12 | 2^12 | 0], x scaled by 2^-e, zero
+// rows past n.
 __global__ void split_points_kernel(const float* __restrict__ X, int64_t ldx, int64_t n, int64_t n_pad, int r,
                                     int64_t units, const uint32_t* __restrict__ absmax, __half* __restrict__ Xs) {
     const int kp = split_k(r);
@@ -127,25 +132,41 @@ __global__ void split_points_kernel(const float* __restrict__ X, int64_t ldx, in
     if (p < n && src >= 0) x = ldexpf(X[(u * ldx + p) * r + src], sc);
     const __half xh = __float2half_rn(x);
     const __half xl = __float2half_rn(x - __half2float(xh));
-    Xs[row * kp + c] = (c < 2 * r) ? xh : (c < 3 * r ? xl : __float2half_rn(0.f));
+    __half out = __float2half_rn(0.f);
+    if (c < 2 * r) out = xh;
+    else if (c < 3 * r) out = xl;
+    else if (c < 3 * r + 2 && p < n) out = __float2half_rn(4096.f);
+    Xs[row * kp + c] = out;
 }
 
-// Cs[u*k_pad + j] = [ch | cl | ch | 0], c scaled by 2^-e, zero rows past k.
+// Cs[u*k_pad + j] = [ch | cl | ch | -nh | -nl | 0], c scaled by 2^-e,
+// nh + nl = |scaled c|^2 / 2^13 (summed in fp64, split in two fp16 parts);
+// zero rows past k.  One thread per row.
 __global__ void split_centroids_kernel(const float* __restrict__ C, int k, int k_pad, int r, int64_t units,
                                        const uint32_t* __restrict__ absmax, __half* __restrict__ Cs) {
     const int kp = split_k(r);
-    const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-    if (e >= units * k_pad * kp) return;
-    const int c = (int)(e % kp);
-    const int64_t row = e / kp;
+    const int64_t row = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (row >= units * k_pad) return;
     const int64_t u = row / k_pad, j = row % k_pad;
     const int sc = -scale_exp(absmax);
-    const int src = c < r ? c : (c < 2 * r ? c - r : (c < 3 * r ? c - 2 * r : -1));
-    float x = 0.f;
-    if (j < k && src >= 0) x = ldexpf(C[(u * k + j) * r + src], sc);
-    const __half xh = __float2half_rn(x);
-    const __half xl = __float2half_rn(x - __half2float(xh));
-    Cs[row * kp + c] = (c < 3 * r && c >= r && c < 2 * r) ? xl : (c < 3 * r ? xh : __float2half_rn(0.f));
+    __half* o = Cs + row * kp;
+    double nrm = 0.0;   // (in fp64: the norm then carries only the split's error)
+    for (int c = 0; c < r; ++c) {
+        float x = 0.f;
+        if (j < k) x = ldexpf(C[(u * k + j) * r + c], sc);
+        nrm = fma((double)x, (double)x, nrm);
+        const __half xh = __float2half_rn(x);
+        const __half xl = __float2half_rn(x - __half2float(xh));
+        o[c] = xh;
+        o[r + c] = xl;
+        o[2 * r + c] = xh;
+    }
+    const double hn = ldexp(nrm, -13);
+    const __half nh = __double2half(hn);
+    const __half nl = __double2half(hn - (double)__half2float(nh));
+    o[3 * r] = __hneg(nh);
+    o[3 * r + 1] = __hneg(nl);
+    for (int c = 3 * r + 2; c < kp; ++c) o[c] = __float2half_rn(0.f);
 }
 
 template <int R>
@@ -182,7 +203,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(acc_full + b, 1);
-            mbar_init(acc_empty + b, 128);
+            mbar_init(acc_empty + b, 256);
         }
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
@@ -249,43 +270,48 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
             if (!ok) latch(err, kErrTimeout);
         }
     } else {
-        // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31, one point per thread
+        // epilogue: warp w reads TMEM lanes 32*(w%4) .. +31, one point per
+        // thread; warps 2-5 take columns [0, 128) of every tile, warps 6-9
+        // columns [128, 256)
         const int q = warp & 3;
+        const int half = (warp - 2) >> 2;
         const int row = 32 * q + lane;
         const int64_t p = p0 + row;
-        float best = INFINITY;
-        int bestj = 0;
-        const float* ccu = cc + (int64_t)u * k;
-        // x.c = 2^(2e) (scaled x).(scaled c): -2 x.c is one exact power-of-two multiple
-        const float m2 = -ldexpf(2.f, 2 * scale_exp(absmax));
+        float best = -INFINITY;
+        int bestj = INT32_MAX;
         for (int t = 0; t < ntile; ++t) {
             const int buf = t & 1;
-            // the tile's centroid norms, one per lane per 32-column chunk, read
-            // before the wait and handed to every lane by shuffles
-            float ccr[kTN / 32];
-#pragma unroll
-            for (int cb = 0; cb < kTN / 32; ++cb) {
-                const int j = t * kTN + cb * 32 + lane;
-                ccr[cb] = j < k ? __ldg(ccu + j) : 0.f;
-            }
             if (!mbar_wait(acc_full + buf, (uint32_t)(t >> 1) & 1u)) { ok = false; latch(err, kErrTimeout); break; }
             asm volatile("tcgen05.fence::after_thread_sync;");
 #pragma unroll
-            for (int cb = 0; cb < kTN / 32; ++cb) {
+            for (int cb = 0; cb < kTN / 64; ++cb) {
                 float v[32];
-                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + buf * kTN + cb * 32, v);
-                const int j0 = t * kTN + cb * 32;
+                const int col = half * (kTN / 2) + cb * 32;
+                tmem_ld32(tmem + ((uint32_t)(32 * q) << 16) + buf * kTN + col, v);
+                const int j0 = t * kTN + col;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
-                    const int j = j0 + i;
-                    const float dist = __fmaf_rn(m2, v[i], __shfl_sync(0xffffffffu, ccr[cb], i));
-                    if (j < k && dist < best) { best = dist; bestj = j; }
+                    if (v[i] > best && j0 + i < k) { best = v[i]; bestj = j0 + i; }
                 }
             }
             asm volatile("tcgen05.fence::before_thread_sync;");
             mbar_arrive(acc_empty + buf);
         }
-        if (ok && p < n) labels[(int64_t)u * ldl + p] = bestj;
+        // the two halves of each point: the larger value, ties to the lower id
+        float* mv = reinterpret_cast<float*>(tmem_slot + 4);    // [128] values of the second half
+        int* mj = reinterpret_cast<int*>(mv + kTM);            // [128] their ids
+        if (half == 1) {
+            mv[row] = best;
+            mj[row] = bestj;
+        }
+        asm volatile("bar.sync 1, 256;" ::: "memory");   // the 8 epilogue warps only
+        if (half == 0) {
+            const float ob = mv[row];
+            const int oj = mj[row];
+            if (ob > best || (ob == best && oj < bestj)) { best = ob; bestj = oj; }
+            if (bestj == INT32_MAX) bestj = 0;
+            if (ok && p < n) labels[(int64_t)u * ldl + p] = bestj;
+        }
     }
     asm volatile("tcgen05.fence::before_thread_sync;");
     __syncthreads();
@@ -295,7 +321,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
 
 template <int R>
 size_t tc_smem_bytes() {
-    return (size_t)(split_k(R) / kKC) * kTM * 128 + (size_t)kStagesB * kTN * 128 + 256 + 1024;
+    // operand tiles + barriers and TMEM slot (256 B) + the halves' merge (1 KB) + alignment
+    return (size_t)(split_k(R) / kKC) * kTM * 128 + (size_t)kStagesB * kTN * 128 + 256 + 1024 + 1024;
 }
 
 }  // namespace
@@ -343,9 +370,9 @@ int assign_tc_run(void* work, const float* C, const float* cc, int64_t units, in
                   int32_t* labels, int64_t ldl, int32_t* err, cudaStream_t s) {
     AssignTcWork* w = static_cast<AssignTcWork*>(work);
     const int kp = split_k(r);
-    const int64_t tot = units * (int64_t)w->k_pad * kp;
+    const int64_t tot = units * (int64_t)w->k_pad;
     note_launch();
-    split_centroids_kernel<<<(unsigned)((tot + 255) / 256), 256, 0, s>>>(C, k, w->k_pad, r, units, w->absmax,
+    split_centroids_kernel<<<(unsigned)((tot + 127) / 128), 128, 0, s>>>(C, k, w->k_pad, r, units, w->absmax,
                                                                          w->Cs);
     CUtensorMap mx, mc;
     if (!make_tensor_map_2d(&mx, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, w->Xs, units * w->n_pad, kp, kp * 2, kKC, kTM) ||
