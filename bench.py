@@ -492,20 +492,32 @@ def run_extra(w, inp, bp, sp, dev, select_ms, idx, cnt):
     N = w.n_tokens
     ix = lsa.lsa_build_index(bp, K, inp["W"])
     info = ix.info()
+    # full-scan time: 8 runs of 4,096 consecutive queries, one in the middle
+    # of every eighth of the sequence (the causal cost grows with the
+    # position), timed in one call and scaled to all N queries
+    runs = 8
+    run_len = min(4096, max(1, N // (2 * runs)))
+    tpos = torch.cat([torch.arange(run_len, device=dev) + (2 * j + 1) * N // (2 * runs) - run_len // 2
+                      for j in range(runs)]).clamp_(0, N - 1).unique()
+    tq = Q[:, tpos].contiguous()
+    tqpos = tpos[None, :].repeat(w.batch, 1).contiguous()
+    lsa.lsa_fullscan_select(ix, sp, tq, q_pos=tqpos)  # warm-up
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    lsa.lsa_fullscan_select(ix, sp, tq, q_pos=tqpos)
+    e1.record()
+    torch.cuda.synchronize()
+    full_ms_sample = e0.elapsed_time(e1)
+    full_ms_est = full_ms_sample * N / tpos.numel()
+    del tq, tqpos
+    # recall and needles: 2,048 queries spread over the sequence
     ns = 2048
     pos = torch.linspace(0, N - 1, ns, device=dev).round().to(torch.int64)
     pos = torch.unique(pos)
     qs = Q[:, pos].contiguous()
     qpos = pos[None, :].repeat(w.batch, 1).contiguous()
-    lsa.lsa_fullscan_select(ix, sp, qs, q_pos=qpos)  # warm-up
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
     fidx, fcnt = lsa.lsa_fullscan_select(ix, sp, qs, q_pos=qpos)
-    e1.record()
-    torch.cuda.synchronize()
-    full_ms_sample = e0.elapsed_time(e1)
-    full_ms_est = full_ms_sample * N / pos.numel()
     tidx = idx[:, pos]
     tcnt = cnt[:, pos]
 
@@ -592,7 +604,9 @@ def run_extra(w, inp, bp, sp, dev, select_ms, idx, cnt):
                "tree_recall_vs_fullscan_topk": recall(psi, psc),
                "needle_hit_rate_tree": nh_pca / max(1, len(needles))}
         ixp.free()
-    return {"fullscan_ms_estimate": full_ms_est, "fullscan_sample_queries": int(pos.numel()),
+    return {"fullscan_ms_estimate": full_ms_est, "fullscan_sample_queries": int(tpos.numel()),
+            "fullscan_sample": f"{runs} runs of {run_len} consecutive queries, one in the middle of every "
+                               f"eighth of the sequence, timed in one call, scaled to {N} queries",
             "pca_map": pca,
             "tree_select_ms": select_ms, "tree_vs_fullscan_speedup": full_ms_est / select_ms,
             "tree_recall_vs_fullscan_topk": tree_recall, "flat_vs_tree": flat,

@@ -339,6 +339,10 @@ int check_select(const lsa_index* ix, const lsa_select_params* sp, const void* Q
     return LSA_OK;
 }
 
+// Full scans of this many (query, KV head) pairs or more take the tensor-core
+// filter (fewer: the per-query kernel scores every block directly).
+constexpr int64_t kFullscanTcMinPairs = 512;
+
 int do_select(const lsa_index* ix, const lsa_select_params* sp, const void* Q, int64_t nq, const int64_t* q_pos,
               int64_t q_pos0, int32_t* idx, int32_t* cnt, int32_t max_sel, void* stream, bool fullscan,
               unsigned long long* work = nullptr) {
@@ -353,7 +357,10 @@ int do_select(const lsa_index* ix, const lsa_select_params* sp, const void* Q, i
     float* qbar = scratch.alloc<float>(p.batch * nq * p.hkv * p.r);
     if (scratch.status != LSA_OK) return scratch.status;
     st = launch_query_latent(Q, ix->W, p.batch, nq, sp->hq, p.hkv, p.d, p.r, p.dtype, qbar, s);
-    if (st == LSA_OK) st = launch_select(ix, sp, qbar, nq, q_pos, q_pos0, idx, cnt, max_sel, fullscan, s, work);
+    if (st == LSA_OK && fullscan && nq * ix->units >= kFullscanTcMinPairs && fullscan_tc_applies(ix, sp))
+        st = launch_fullscan_tc(ix, sp, qbar, nq, q_pos, q_pos0, idx, cnt, max_sel, s, scratch);
+    else if (st == LSA_OK)
+        st = launch_select(ix, sp, qbar, nq, q_pos, q_pos0, idx, cnt, max_sel, fullscan, s, work);
     scratch.release();
     return st;
 }

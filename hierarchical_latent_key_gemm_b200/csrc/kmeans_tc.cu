@@ -31,60 +31,18 @@
 #include <mutex>
 #include <new>
 
-#include "tma_util.cuh"
+#include "tc_common.cuh"
 
 namespace lsa {
 namespace {
 
-constexpr int kTM = 128;          // points per CTA (UMMA M)
-constexpr int kTN = 256;          // centroids per tile (UMMA N)
+constexpr int kTM = kTcM;         // points per CTA (UMMA M)
+constexpr int kTN = kTcN;         // centroids per tile (UMMA N)
 constexpr int kKC = 64;           // fp16 per K-chunk: one 128-byte swizzle row
 constexpr int kStagesB = 3;
 constexpr int kThreadsTC = 320;   // producer, MMA issuer, 8 epilogue warps
-// K-major operand, 128-byte swizzle: 8-row x 128-byte atoms, 1024 bytes apart.
-__device__ __forceinline__ uint64_t umma_desc(const void* p) {
-    const uint64_t addr = su32(p);
-    uint64_t d = 0;
-    d |= (addr >> 4) & 0x3FFFull;          // start address
-    d |= (uint64_t)1 << 16;                // leading byte offset (unused for swizzled K-major)
-    d |= (uint64_t)(1024 >> 4) << 32;      // stride byte offset: next 8-row group
-    d |= (uint64_t)1 << 46;                // descriptor version
-    d |= (uint64_t)2 << 61;                // 128-byte swizzle
-    return d;
-}
-// kind::f16 with fp16 A and B (format 0), fp32 accumulate, K-major A and B,
-// M = 128, N = 256.
-constexpr uint32_t kIdesc = (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(kTN >> 3) << 17) |
-                            ((uint32_t)(kTM >> 4) << 24);
-
-__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n\t}" ::"r"(tmem_d),
-        "l"(a), "l"(b), "r"(kIdesc), "r"(accumulate), "r"(0u));
-}
-
 // K extent of the split operands: 3r + 2 rounded up to whole 64-element chunks.
 __host__ __device__ constexpr int split_k(int r) { return (3 * r + 2 + kKC - 1) / kKC * kKC; }
-__device__ __forceinline__ void umma_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(su32(bar))
-                 : "memory");
-}
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float* v) {
-    uint32_t r[32];
-    asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,"
-        "%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
-        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-          "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
-          "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
-          "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
-        : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
 
 // Largest |value| of the points and the starting centroids, as float bits
 // (non-negative floats order like their bit patterns).

@@ -179,6 +179,21 @@ int launch_select(const lsa_index* ix, const lsa_select_params* sp, const float*
                   const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt, int max_sel,
                   bool fullscan, cudaStream_t s, unsigned long long* work = nullptr,
                   const ScoredOut* scored = nullptr);
+// Full scan on the tensor cores (fullscan_tc.cu): candidate lists from a
+// filtering GEMM, ranked exactly by the per-query kernel (select.cu).
+struct ListIn {
+    const int32_t* cand;
+    const int32_t* count;
+    int64_t npad;
+    int cap;
+};
+bool fullscan_tc_applies(const lsa_index* ix, const lsa_select_params* sp);
+int launch_fullscan_tc(const lsa_index* ix, const lsa_select_params* sp, const float* qbar, int64_t nq,
+                       const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt, int max_sel,
+                       cudaStream_t s, Arena& A);
+int launch_select_lists(const lsa_index* ix, const lsa_select_params* sp, const float* qbar, int64_t nq_stride,
+                        int64_t nq_grid, const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt,
+                        int max_sel, const ListIn& li, cudaStream_t s);
 // Merge of per-shard scored blocks into selection rows (select.cu).
 int launch_merge_selection(int parts, const float* score, const int32_t* block, const int32_t* count, int kb_cap,
                            int64_t batch, int64_t nq, int hkv, const int64_t* q_pos, int64_t q_pos0, int pool,

@@ -69,6 +69,13 @@ struct SelArgs {
     float* out_score;
     int32_t* out_block;
     int32_t* out_n;
+    // full scan over candidate lists (fullscan_tc.cu): for query qi of unit u,
+    // two lists at l_cand + ((u * l_npad + qi) * 2 + half) * l_cap with
+    // l_cnt entries each; a list longer than l_cap means "scan every block"
+    const int32_t* l_cand;
+    const int32_t* l_cnt;
+    int64_t l_npad;
+    int l_cap;
 };
 
 // THREADS = kSelThreads for large grids; small grids (decode: a few queries)
@@ -324,14 +331,35 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
         const int64_t hi = min(a.nb - 1, b_hi);
         const int total = hi >= b_lo ? (int)(hi - b_lo + 1) : 0;
         const float* kl = a.Kl + (int64_t)u * a.nb_cap * R;
-        stream_topk(total, a.kb, [&](int t, OwnerState* state, bool* el, int* id, int* p, float* y) {
-            (void)state;
-            const int64_t b = b_lo + t;
-            load_row(kl + b * R, y);
-            *id = (int)b;
-            *p = 0;
-            *el = true;
-        });
+        bool listed = false;
+        if (a.l_cand) {
+            const int64_t gr = (int64_t)u * a.l_npad + qi;
+            const int n0 = a.l_cnt[gr * 2], n1 = a.l_cnt[gr * 2 + 1];
+            if (n0 <= a.l_cap && n1 <= a.l_cap) {
+                // every block that can be in the top K is in the two lists
+                listed = true;
+                const int32_t* L0 = a.l_cand + gr * 2 * a.l_cap;
+                const int32_t* L1 = L0 + a.l_cap;
+                stream_topk(n0 + n1, a.kb, [&](int t, OwnerState* state, bool* el, int* id, int* p, float* y) {
+                    (void)state;
+                    const int64_t b = t < n0 ? __ldg(L0 + t) : __ldg(L1 + (t - n0));
+                    load_row(kl + b * R, y);
+                    *id = (int)b;
+                    *p = 0;
+                    *el = true;
+                });
+            }
+        }
+        if (!listed) {
+            stream_topk(total, a.kb, [&](int t, OwnerState* state, bool* el, int* id, int* p, float* y) {
+                (void)state;
+                const int64_t b = b_lo + t;
+                load_row(kl + b * R, y);
+                *id = (int)b;
+                *p = 0;
+                *el = true;
+            });
+        }
     }
     const int nsel = sh.count;
     if (SCORED) {
@@ -557,6 +585,48 @@ int launch_merge_selection(int parts, const float* score, const int32_t* block, 
     note_launch();
     merge_select_kernel<<<(unsigned)m.rows, kMergeThreads, smem, s>>>(m);
     return cuda_status(cudaGetLastError());
+}
+
+}  // namespace lsa
+
+namespace lsa {
+
+int launch_select_lists(const lsa_index* ix, const lsa_select_params* sp, const float* qbar, int64_t nq_stride,
+                        int64_t nq_grid, const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt,
+                        int max_sel, const ListIn& li, cudaStream_t s) {
+    const lsa_build_params& p = ix->p;
+    SelArgs a{};
+    a.levels = p.levels;
+    a.Kl = ix->Kl;
+    a.nb_cap = ix->nb_cap;
+    a.nb = ix->nb;
+    a.pool = p.pool;
+    a.sink = p.sink;
+    a.window = sp->window;
+    a.beam = sp->beam;
+    a.kb = (sp->topk + p.pool - 1) / p.pool;
+    a.hkv = p.hkv;
+    a.nq = nq_stride;
+    a.qbar = qbar;
+    a.q_pos = q_pos;
+    a.q_pos0 = q_pos0;
+    a.idx = idx;
+    a.cnt = cnt;
+    a.max_sel = max_sel;
+    a.l_cand = li.cand;
+    a.l_cnt = li.count;
+    a.l_npad = li.npad;
+    a.l_cap = li.cap;
+    const int kmax = a.kb > a.beam ? a.kb : a.beam;
+    int cap = 1024;
+    while (cap < 2 * kmax) cap <<= 1;
+    a.cap = cap;
+    if (nq_grid <= 0) return LSA_OK;
+    switch (p.r) {
+        case 16: return launch_select_t<16, kSelThreads>(a, nq_grid, ix->units, true, s);
+        case 32: return launch_select_t<32, kSelThreads>(a, nq_grid, ix->units, true, s);
+        default: return launch_select_t<64, kSelThreads>(a, nq_grid, ix->units, true, s);
+    }
 }
 
 }  // namespace lsa

@@ -224,6 +224,14 @@ int lsa_pca_map(const void* K, int64_t batch, int64_t n_tokens, int64_t ld_token
 
 /* The quadratic baseline indexer: every candidate block is scored, no tree.
  * Same arguments and output format as lsa_select (beam is ignored).
+ * Calls of 512 or more (query, KV head) pairs with r <= 64 first filter on the
+ * tensor cores (fp16 scores of 128 queries x 256 blocks per tile; a per-query
+ * histogram gives a threshold that provably keeps every block of the exact
+ * top ceil(K/P)), then rank the survivors with the exact fp32 arithmetic of
+ * the per-query kernel, so the selected blocks are the same bits as scoring
+ * every block exactly.  Stream-ordered scratch: the fp16 keys (2 B x 64 per
+ * block), and for each chunk of up to ~2 GiB/(16 KB x KV heads) queries,
+ * 16 KB of candidate lists per (query, KV head).
  * [p3 flowchart, red path: the full key scan] */
 int lsa_fullscan_select(const lsa_index* index, const lsa_select_params* params, const void* Q,
                         int64_t nq, const int64_t* q_pos, int64_t q_pos0,
