@@ -359,8 +359,10 @@ int do_select(const lsa_index* ix, const lsa_select_params* sp, const void* Q, i
     st = launch_query_latent(Q, ix->W, p.batch, nq, sp->hq, p.hkv, p.d, p.r, p.dtype, qbar, s);
     if (st == LSA_OK && fullscan && nq * ix->units >= kFullscanTcMinPairs && fullscan_tc_applies(ix, sp))
         st = launch_fullscan_tc(ix, sp, qbar, nq, q_pos, q_pos0, idx, cnt, max_sel, s, scratch);
+    else if (st == LSA_OK && fullscan)
+        st = launch_select(ix, sp, qbar, nq, q_pos, q_pos0, idx, cnt, max_sel, true, s, work);
     else if (st == LSA_OK)
-        st = launch_select(ix, sp, qbar, nq, q_pos, q_pos0, idx, cnt, max_sel, fullscan, s, work);
+        st = launch_select_tree(ix, sp, qbar, nq, q_pos, q_pos0, idx, cnt, max_sel, s, work, nullptr, scratch);
     scratch.release();
     return st;
 }
@@ -434,7 +436,7 @@ int lsa_select_blocks(const lsa_index* index, const lsa_select_params* params, c
     ScoredOut so{token_offset, (int32_t)(token_offset / p.pool), kb_cap, scores, blocks, count};
     int st = launch_query_latent(Q, index->W, p.batch, nq, sp.hq, p.hkv, p.d, p.r, p.dtype, qbar, s);
     if (st == LSA_OK)
-        st = launch_select(index, params, qbar, nq, q_pos, q_pos0, nullptr, nullptr, 0, false, s, nullptr, &so);
+        st = launch_select_tree(index, params, qbar, nq, q_pos, q_pos0, nullptr, nullptr, 0, s, nullptr, &so, scratch);
     scratch.release();
     return st;
 }

@@ -179,6 +179,29 @@ int launch_select(const lsa_index* ix, const lsa_select_params* sp, const float*
                   const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt, int max_sel,
                   bool fullscan, cudaStream_t s, unsigned long long* work = nullptr,
                   const ScoredOut* scored = nullptr);
+// Dense upper levels scored ahead of the search (node_scores.cu): the
+// leading `levels` levels' scores for every node, row-major per (query, KV
+// head) row, level l from column off[l]; launch_select_rows runs the search
+// over nq rows whose queries, positions and outputs start at the given
+// pointers (sequence stride nq_stride) and takes those levels' scores from S.
+struct PreScores {
+    const float* S;
+    int64_t ld;
+    int levels;
+    int off[LSA_MAX_LEVELS];
+};
+int launch_select_rows(const lsa_index* ix, const lsa_select_params* sp, const float* qbar, int64_t nq_stride,
+                       int64_t nq, const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt, int max_sel,
+                       bool fullscan, cudaStream_t s, unsigned long long* work, const ScoredOut* scored,
+                       const PreScores* pre);
+int dense_levels(const lsa_index* ix, int beam, int max_cols, int* col_off);
+int launch_node_scores(const lsa_index* ix, const float* qbar, int64_t nq_stride, int64_t nqc, int levels,
+                       const int* col_off, float* S, int64_t ld, cudaStream_t s);
+// The tree search of nq queries: dense levels first when the call is large
+// enough, in chunks of queries whose scores fit a bounded buffer.
+int launch_select_tree(const lsa_index* ix, const lsa_select_params* sp, const float* qbar, int64_t nq,
+                       const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt, int max_sel,
+                       cudaStream_t s, unsigned long long* work, const ScoredOut* scored, Arena& A);
 // Full scan on the tensor cores (fullscan_tc.cu): candidate lists from a
 // filtering GEMM, ranked exactly by the per-query kernel (select.cu).
 struct ListIn {

@@ -22,6 +22,8 @@
 // order in which warps append.  One buffer instead of two halves the shared
 // memory of a CTA, which leaves more of each SM's L1 for the centroid rows
 // that every query of a unit reads.
+#include <type_traits>
+
 #include "select_common.cuh"
 
 namespace lsa {
@@ -76,6 +78,14 @@ struct SelArgs {
     const int32_t* l_cnt;
     int64_t l_npad;
     int l_cap;
+    // scores of the leading pre_levels tree levels, computed for all of their
+    // nodes by the dense-level kernel (node_scores.cu) with this kernel's own
+    // arithmetic: row (bseq * pre_nq + qi) * hkv + h, level l's node at
+    // position q in column pre_off[l] + q
+    const float* pre;
+    int64_t pre_nq, pre_ld;
+    int pre_levels;
+    int pre_off[LSA_MAX_LEVELS];
 };
 
 // THREADS = kSelThreads for large grids; small grids (decode: a few queries)
@@ -162,8 +172,14 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
     // buffer has been compacted, a candidate whose key is below the k-th kept
     // key cannot enter the top k and is not appended.  The buffer is compacted
     // only when the next chunk might not fit, and at the end.  Appends are
-    // aggregated per warp: one shared-memory atomic per batch.
-    auto stream_topk = [&](int total, int k, auto&& fetch) {
+    // aggregated per warp: one shared-memory atomic per batch.  With LANE
+    // (scores given, no rows to load), every lane is a group of its own and
+    // fetch puts the candidate's score in y[0].
+    auto stream_topk = [&](int total, int k, auto lane_mode, auto&& fetch) {
+        constexpr bool LANE = decltype(lane_mode)::value;
+        constexpr int NGx = LANE ? THREADS : NG;
+        const int gidx = LANE ? (int)threadIdx.x : gid;
+        const bool lead = LANE || gl == 0;
         if (k <= 0) return;  // nothing is kept; the buffer stays empty
         // entered with an empty buffer; nbuf mirrors sh.count between chunks
         if (threadIdx.x == 0) sh.thr = 0u;
@@ -172,8 +188,8 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
         while (t0 < total) {
             const uint32_t thr = sh.thr;
             const int t1 = min(total, t0 + (a.cap - nbuf));
-            const int span = (t1 - t0 + NG - 1) / NG;
-            const int tb = t0 + gid * span;
+            const int span = (t1 - t0 + NGx - 1) / NGx;
+            const int tb = t0 + gidx * span;
             const int te = min(t1, tb + span);
             OwnerState state{-1, 0, 0};
             for (int s0 = 0; s0 < span; s0 += kUnroll) {
@@ -192,14 +208,15 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
 #pragma unroll
                 for (int v = 0; v < kUnroll; ++v) {
                     if (ok[v]) {
-                        sc[v] = dot(y[v]);
+                        if constexpr (LANE) sc[v] = y[v][0];
+                        else sc[v] = dot(y[v]);
                         if (COUNT) {
-                            if (phase) nsc_blk += (gl == 0);
-                            else nsc_node += (gl == 0);
+                            if (phase) nsc_blk += lead;
+                            else nsc_node += lead;
                         }
                         ok[v] = fkey(sc[v]) >= thr;
                     }
-                    bal[v] = __ballot_sync(0xffffffffu, ok[v] && gl == 0);
+                    bal[v] = __ballot_sync(0xffffffffu, ok[v] && lead);
                     nb_warp += __popc(bal[v]);
                 }
                 int base = 0;
@@ -207,7 +224,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
                 base = __shfl_sync(0xffffffffu, base, 0);
 #pragma unroll
                 for (int v = 0; v < kUnroll; ++v) {
-                    if (ok[v] && gl == 0) {
+                    if (ok[v] && lead) {
                         const int p = base + __popc(bal[v] & lt_mask);
                         bs[p] = sc[v];
                         bi[p] = idv[v];
@@ -260,18 +277,26 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
             const int total = (l == 0) ? nl : pre[nk];
             if (threadIdx.x == 0) sh.count = 0;
             __syncthreads();
-            stream_topk(total, a.beam, [&](int t, OwnerState* state, bool* el, int* id, int* p, float* y) {
-                int q;
-                if (l == 0) {
-                    q = t;
-                } else {
-                    q = slot_of(t, nk, state);
-                }
-                load_row(cent + (int64_t)q * R, y);
-                *id = __ldg(oid + q);
-                *p = q;
-                *el = __ldg(mp + q) <= bound;
-            });
+            if (l < a.pre_levels) {
+                const float* ps = a.pre + ((bseq * a.pre_nq + qi) * a.hkv + h) * a.pre_ld + a.pre_off[l];
+                stream_topk(total, a.beam, std::true_type{},
+                            [&](int t, OwnerState* state, bool* el, int* id, int* p, float* y) {
+                                const int q = (l == 0) ? t : slot_of(t, nk, state);
+                                y[0] = __ldg(ps + q);
+                                *id = __ldg(oid + q);
+                                *p = q;
+                                *el = __ldg(mp + q) <= bound;
+                            });
+            } else {
+                stream_topk(total, a.beam, std::false_type{},
+                            [&](int t, OwnerState* state, bool* el, int* id, int* p, float* y) {
+                                const int q = (l == 0) ? t : slot_of(t, nk, state);
+                                load_row(cent + (int64_t)q * R, y);
+                                *id = __ldg(oid + q);
+                                *p = q;
+                                *el = __ldg(mp + q) <= bound;
+                            });
+            }
             const int n = sh.count;
             for (int e = threadIdx.x; e < n; e += blockDim.x) kk[e] = bp[e];
             __syncthreads();
@@ -320,7 +345,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
         if (threadIdx.x == 0) sh.count = 0;
         __syncthreads();
         phase = 1;
-        stream_topk(pre[nk], a.kb, [&](int t, OwnerState* state, bool* el, int* id, int* p, float* y) {
+        stream_topk(pre[nk], a.kb, std::false_type{}, [&](int t, OwnerState* state, bool* el, int* id, int* p, float* y) {
             const int64_t slot = slot_of(t, nk, state);
             load_row(a.Klp + slot * R, y);
             *id = __ldg(a.blk + slot);
@@ -340,7 +365,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
                 listed = true;
                 const int32_t* L0 = a.l_cand + gr * 2 * a.l_cap;
                 const int32_t* L1 = L0 + a.l_cap;
-                stream_topk(n0 + n1, a.kb, [&](int t, OwnerState* state, bool* el, int* id, int* p, float* y) {
+                stream_topk(n0 + n1, a.kb, std::false_type{}, [&](int t, OwnerState* state, bool* el, int* id, int* p, float* y) {
                     (void)state;
                     const int64_t b = t < n0 ? __ldg(L0 + t) : __ldg(L1 + (t - n0));
                     load_row(kl + b * R, y);
@@ -351,7 +376,7 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
             }
         }
         if (!listed) {
-            stream_topk(total, a.kb, [&](int t, OwnerState* state, bool* el, int* id, int* p, float* y) {
+            stream_topk(total, a.kb, std::false_type{}, [&](int t, OwnerState* state, bool* el, int* id, int* p, float* y) {
                 (void)state;
                 const int64_t b = b_lo + t;
                 load_row(kl + b * R, y);
@@ -493,9 +518,10 @@ __global__ __launch_bounds__(kMergeThreads) void merge_select_kernel(const Merge
 
 }  // namespace
 
-int launch_select(const lsa_index* ix, const lsa_select_params* sp, const float* qbar, int64_t nq,
-                  const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt, int max_sel, bool fullscan,
-                  cudaStream_t s, unsigned long long* work, const ScoredOut* scored) {
+int launch_select_rows(const lsa_index* ix, const lsa_select_params* sp, const float* qbar, int64_t nq_stride,
+                       int64_t nq, const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt, int max_sel,
+                       bool fullscan, cudaStream_t s, unsigned long long* work, const ScoredOut* scored,
+                       const PreScores* pre) {
     const lsa_build_params& p = ix->p;
     if (sp->beam > 1024) return LSA_ERR_INVALID_ARG;
     SelArgs a{};
@@ -520,7 +546,7 @@ int launch_select(const lsa_index* ix, const lsa_select_params* sp, const float*
     a.beam = sp->beam;
     a.kb = (sp->topk + p.pool - 1) / p.pool;
     a.hkv = p.hkv;
-    a.nq = nq;
+    a.nq = nq_stride;
     a.qbar = qbar;
     a.q_pos = q_pos;
     a.q_pos0 = q_pos0;
@@ -528,6 +554,13 @@ int launch_select(const lsa_index* ix, const lsa_select_params* sp, const float*
     a.cnt = cnt;
     a.max_sel = max_sel;
     a.work = work;
+    if (pre && !fullscan) {
+        a.pre = pre->S;
+        a.pre_nq = nq;
+        a.pre_ld = pre->ld;
+        a.pre_levels = pre->levels;
+        for (int l = 0; l < pre->levels; ++l) a.pre_off[l] = pre->off[l];
+    }
     if (scored) {
         a.pos_shift = scored->pos_shift;
         a.blk_shift = scored->blk_shift;
@@ -548,6 +581,13 @@ int launch_select(const lsa_index* ix, const lsa_select_params* sp, const float*
         case 128: return launch_select_r<128>(a, nq, ix->units, fullscan, s);
         default: return LSA_ERR_INVALID_ARG;
     }
+}
+
+int launch_select(const lsa_index* ix, const lsa_select_params* sp, const float* qbar, int64_t nq,
+                  const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt, int max_sel, bool fullscan,
+                  cudaStream_t s, unsigned long long* work, const ScoredOut* scored) {
+    return launch_select_rows(ix, sp, qbar, nq, nq, q_pos, q_pos0, idx, cnt, max_sel, fullscan, s, work, scored,
+                              nullptr);
 }
 
 }  // namespace lsa

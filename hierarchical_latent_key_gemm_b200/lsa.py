@@ -76,6 +76,7 @@ _SIGS = {
     "lsa_free_index": (None, [_vp]),
     "lsa_strerror": (C.c_char_p, [_i32]),
     "lsa_debug_fail_alloc_after": (None, [_i32]),
+    "lsa_debug_dense_config": (None, [_i64, _i64]),
     "lsa_launch_count": (_i64, []),
     "lsa_select_blocks": (_i32, [_vp, C.POINTER(SelectParams), _vp, _i64, _vp, _i64, _i64, _vp, _vp, _vp, _i32,
                                  _vp]),
@@ -543,6 +544,13 @@ def lsa_launch_count() -> int:
 
 def lsa_debug_fail_alloc_after(n: int):
     lib().lsa_debug_fail_alloc_after(int(n))
+
+
+def lsa_debug_dense_config(min_pairs: int = 0, chunk_bytes: int = 0):
+    """Test hook: min_pairs < 0 turns the dense-level scoring of large
+    selections off, 0 restores its default threshold; chunk_bytes bounds its
+    score buffer (0: default)."""
+    lib().lsa_debug_dense_config(int(min_pairs), int(chunk_bytes))
 
 
 def exported_symbols_from_header(header_path: str) -> list:

@@ -441,6 +441,15 @@ const char* lsa_strerror(int status);
  * (n >= 1), to exercise the LSA_ERR_OOM path; n = 0 disarms it. */
 void lsa_debug_fail_alloc_after(int32_t n);
 
+/* Test hook for the dense-level scoring of large selections (the scores of
+ * the upper tree levels whose parents all fit in the beam, computed for a
+ * tile of queries at a time before the per-query search; the selection is
+ * bit-identical either way): min_pairs < 0 turns it off, 0 restores the
+ * default threshold of (query, KV head) pairs per call, > 0 sets it;
+ * chunk_bytes > 0 bounds the score buffer (queries run in chunks that fit),
+ * 0 restores the default of 1 GiB. */
+void lsa_debug_dense_config(int64_t min_pairs, int64_t chunk_bytes);
+
 /* Number of kernels the library has launched in this process (a host-side
  * counter, incremented at every launch; for accounting in benchmarks). */
 int64_t lsa_launch_count(void);

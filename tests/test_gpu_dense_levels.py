@@ -1,0 +1,102 @@
+"""Dense-level scoring of large selections (node_scores.cu).  The upper tree
+levels whose parents all fit in the beam are scored for tiles of queries
+before the per-query search, which then reads one score per node of those
+levels.  The selection must be the same, bit for bit, as that of the
+per-query search scoring every node itself (the scores are the same fp32
+values), with one buffer of scores and with the buffer forced small so that
+the queries run in several chunks.  The per-query search is the path the
+other parity tests check against the oracle; this pins the dense form to it
+on every tree shape the workloads use."""
+import pytest
+import torch
+
+from hierarchical_latent_key_gemm_b200 import lsa
+from hierarchical_latent_key_gemm_b200.workloads import WORKLOADS, make_inputs
+
+import lsa_testutil as TU
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    lsa.lib()
+    yield
+    lsa.lsa_debug_dense_config(0, 0)
+    torch.cuda.synchronize()
+
+
+def _three_ways(ix, sp, Q, **kw):
+    out = []
+    try:
+        for min_pairs, chunk in ((-1, 0), (1, 0), (1, 1 << 20)):
+            lsa.lsa_debug_dense_config(min_pairs, chunk)
+            out.append(lsa.lsa_select(ix, sp, Q, **kw))
+    finally:
+        lsa.lsa_debug_dense_config(0, 0)
+    return out
+
+
+@pytest.mark.parametrize("name,over,beam", [
+    ("int_exact_16k", {}, None),                                        # 16 x 256, r = 16, beam 16: both levels dense
+    ("flat_4k_f32", {}, None),                                          # one level of 64, r = 32
+    ("gqa_128k", dict(n_tokens=16384 + 5, needles=0, components=512), None),   # 32 x 1024, beam 32, 4 KV heads
+    ("gqa_128k", dict(n_tokens=16384 + 5, needles=0, components=512), 31),     # beam below the top level: one level
+    ("prefill_1m", dict(n_tokens=65536 + 7, level_sizes=(16, 128, 1024), needles=0, components=1024,
+                        drift_every=1 << 14), None),                    # three levels, the leaves per query
+])
+def test_dense_levels_match_the_per_query_search(name, over, beam):
+    w = WORKLOADS[name].scaled(**over)
+    inp = make_inputs(w, seed=31, device="cuda")
+    ix = lsa.lsa_build_index(TU.build_params(w), inp["K"], inp["W"])
+    sp = TU.select_params(w, beam=beam)
+    (i0, c0), (i1, c1), (i2, c2) = _three_ways(ix, sp, inp["Q"])
+    assert lsa.lsa_check(ix) == lsa.LSA_OK
+    assert torch.equal(c0, c1) and torch.equal(i0, i1)
+    assert torch.equal(c0, c2) and torch.equal(i0, i2)
+    ix.free()
+
+
+def test_dense_levels_batch_and_given_positions():
+    """Several sequences (row index (b * nq + qi) * hkv + h in the score
+    buffer) and query positions given per query."""
+    w = WORKLOADS["decode_10m_x4"].scaled(n_tokens=8192 + 3, level_sizes=(8, 64, 512), needles=0, components=512,
+                                          decode_steps=0)
+    inp = make_inputs(w, seed=32, device="cuda")
+    ix = lsa.lsa_build_index(TU.build_params(w), inp["K"], inp["W"])
+    sp = TU.select_params(w)
+    nq = 1500
+    g = torch.Generator().manual_seed(5)
+    pos = torch.randint(0, w.n_tokens, (w.batch, nq), generator=g).to(torch.int64).cuda()
+    Q = inp["Q"][:, :nq].contiguous()
+    (i0, c0), (i1, c1), (i2, c2) = _three_ways(ix, sp, Q, q_pos=pos)
+    assert lsa.lsa_check(ix) == lsa.LSA_OK
+    assert torch.equal(c0, c1) and torch.equal(i0, i1)
+    assert torch.equal(c0, c2) and torch.equal(i0, i2)
+    ix.free()
+
+
+def test_dense_levels_scored_blocks():
+    """The scored-blocks form (context-parallel shards) through the dense path."""
+    w = WORKLOADS["gqa_128k"].scaled(n_tokens=8192 + 1, needles=0, components=256)
+    inp = make_inputs(w, seed=33, device="cuda")
+    ix = lsa.lsa_build_index(TU.build_params(w), inp["K"], inp["W"])
+    sp = TU.select_params(w)
+    outs = []
+    try:
+        for min_pairs, chunk in ((-1, 0), (1, 0), (1, 1 << 18)):
+            lsa.lsa_debug_dense_config(min_pairs, chunk)
+            sc, bl, ct = lsa.lsa_select_blocks(ix, sp, inp["Q"], 0)
+            # the kept blocks come in no particular order: sort each row by block id
+            key = torch.where(bl >= 0, bl, torch.full_like(bl, 2 ** 31 - 1))
+            key, order = torch.sort(key, dim=-1)
+            outs.append((torch.gather(sc, -1, order), key, ct))
+    finally:
+        lsa.lsa_debug_dense_config(0, 0)
+    assert lsa.lsa_check(ix) == lsa.LSA_OK
+    for o in outs[1:]:
+        for a, b in zip(outs[0], o):
+            assert torch.equal(a, b)
+    ix.free()
