@@ -155,10 +155,13 @@ def measured_peaks() -> dict:
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
-def kernel_source_sha(fname: str) -> str:
-    path = os.path.join(ROOT, "hierarchical_latent_key_gemm_b200", "csrc", fname)
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def kernel_source_sha(fnames: str) -> str:
+    """sha256[:16] of the kernel's source files ("a.cu+b.cuh": concatenated in that order)."""
+    h = hashlib.sha256()
+    for fname in fnames.split("+"):
+        with open(os.path.join(ROOT, "hierarchical_latent_key_gemm_b200", "csrc", fname), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def recorded_traffic(kernel: str, workload: str, src: str):
@@ -282,7 +285,7 @@ def run_ours(args):
     sel = stages["select"]
     roofline = {"bound": "hbm", "kernel": "select_kernel<64, tree> (select stage: query latents + select)",
                 "achieved": sel["achieved_GBps"], "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": sel["frac"],
-                "traffic": recorded_traffic("select_kernel<64, tree>", w.name, "select.cu"),
+                "traffic": recorded_traffic("select_kernel<64, tree>", w.name, "select.cu+select_common.cuh"),
                 "algorithmic_bytes_per_launch": sel["algorithmic_bytes"], "peak_source": peaks["source"],
                 "note": sel["formula"]}
 

@@ -339,9 +339,11 @@ int check_select(const lsa_index* ix, const lsa_select_params* sp, const void* Q
     return LSA_OK;
 }
 
-// Full scans of this many (query, KV head) pairs or more take the tensor-core
-// filter (fewer: the per-query kernel scores every block directly).
-constexpr int64_t kFullscanTcMinPairs = 512;
+// Full scans of this many (query, KV head) pairs or more take the
+// tensor-core filter (its CTAs split the block range when the query tiles
+// alone would not fill the GPU); fewer pairs are scanned by the per-query
+// kernel directly.
+constexpr int64_t kFullscanTcMinPairs = 64;
 
 int do_select(const lsa_index* ix, const lsa_select_params* sp, const void* Q, int64_t nq, const int64_t* q_pos,
               int64_t q_pos0, int32_t* idx, int32_t* cnt, int32_t max_sel, void* stream, bool fullscan,

@@ -61,6 +61,12 @@ struct FsArgs {
     int32_t* cand;            // [units][nq_pad][2][kHalfCap] block ids
     int32_t* ccount;          // [units][nq_pad][2]
     int32_t* err;
+    // split of each tile's block range over gridDim.z CTAs (small calls):
+    // pass 0 adds its counts into ghist [units][nq_pad][kBins] and the
+    // thresholds come from fs_thr_kernel; pass 1 appends through atomics on
+    // ccount (zeroed before)
+    int nsplit;
+    int32_t* ghist;
 };
 
 __device__ __forceinline__ int64_t fs_bhi(const FsArgs& a, int u, int64_t qi) {
@@ -139,6 +145,30 @@ __global__ void fs_kmax_kernel(const float* __restrict__ knorm, int64_t n, int64
     }
 }
 
+// Thresholds of a split pass 0: the same rule as in the kernel, on the summed
+// histogram of every row.
+__global__ void fs_thr_kernel(const int32_t* __restrict__ ghist, const float* __restrict__ qnorm,
+                              const float* __restrict__ kmax, int64_t nq, int64_t nq_pad, int64_t units, int kb,
+                              float* __restrict__ thr) {
+    const int64_t gr = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (gr >= units * nq_pad) return;
+    const int64_t u = gr / nq_pad, qi = gr % nq_pad;
+    if (qi >= nq) return;
+    const float Rr = qnorm[gr] * kmax[u];
+    const int32_t* h = ghist + gr * kBins;
+    float t = -INFINITY;
+    int cum = 0;
+    for (int bin = kBins - 1; bin >= 0; --bin) {
+        cum += h[bin];
+        if (cum >= kb) {
+            const float L = -Rr + (float)bin * (2.f * Rr / (float)kBins);
+            t = L - 2.f * (kEpsRel * Rr + kEpsAbs);
+            break;
+        }
+    }
+    thr[gr] = t;
+}
+
 template <int R, int PASS>
 __global__ void __launch_bounds__(kFThreads, 1)
     fs_tc_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_k,
@@ -196,7 +226,11 @@ __global__ void __launch_bounds__(kFThreads, 1)
     __syncthreads();
     asm volatile("tcgen05.fence::after_thread_sync;");
     const uint32_t tmem = *tmem_slot;
-    const int ntile = *sh_tiles;
+    // this CTA's share of the tile's block range: tiles [t_beg, t_beg + ntile)
+    const int ntile_all = *sh_tiles;
+    const int per = (ntile_all + a.nsplit - 1) / a.nsplit;
+    const int t_beg = min(ntile_all, (int)blockIdx.z * per);
+    const int ntile = min(ntile_all, t_beg + per) - t_beg;
 
     bool ok = true;
     if (warp == 0) {
@@ -212,7 +246,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
                     if (!mbar_wait(b_empty + s, ph ^ 1u)) { ok = false; break; }
                     mbar_expect_tx(b_full + s, B_CHUNK);
                     tma_load_2d(Bs + s * B_CHUNK, &map_k, b_full + s, c * kFKC,
-                                (int)(u * a.nb_pad + a.b_lo + (int64_t)t * kFN));
+                                (int)(u * a.nb_pad + a.b_lo + (int64_t)(t_beg + t) * kFN));
                     ++issued;
                 }
             }
@@ -274,7 +308,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
                 float v[32];
                 const int col = half * (kFN / 2) + cb * 32;
                 tmem_ld32(tmem + ((uint32_t)(32 * qd) << 16) + buf * kFN + col, v);
-                const int64_t b0 = a.b_lo + (int64_t)t * kFN + col;
+                const int64_t b0 = a.b_lo + (int64_t)(t_beg + t) * kFN + col;
 #pragma unroll
                 for (int i = 0; i < 32; ++i) {
                     if (b0 + i <= bh) {
@@ -282,8 +316,13 @@ __global__ void __launch_bounds__(kFThreads, 1)
                             const int bin = min(kBins - 1, max(0, (int)((v[i] + Rr) * inv)));
                             atomicAdd(hr + bin, 1);
                         } else if (v[i] >= T) {
-                            if (n < kHalfCap) lst[n] = (int32_t)(b0 + i);
-                            ++n;
+                            if (a.nsplit == 1) {
+                                if (n < kHalfCap) lst[n] = (int32_t)(b0 + i);
+                                ++n;
+                            } else {
+                                const int pp = atomicAdd(a.ccount + gr * 2 + half, 1);
+                                if (pp < kHalfCap) lst[pp] = (int32_t)(b0 + i);
+                            }
                         }
                     }
                 }
@@ -291,7 +330,12 @@ __global__ void __launch_bounds__(kFThreads, 1)
             asm volatile("tcgen05.fence::before_thread_sync;");
             mbar_arrive(acc_empty + buf);
         }
-        if (PASS == 0) {
+        if (PASS == 0 && a.nsplit > 1) {
+            asm volatile("bar.sync 1, 256;" ::: "memory");   // both halves' counts are in
+            if (half == 0 && live)
+                for (int bin = 0; bin < kBins; ++bin)
+                    if (hr[bin]) atomicAdd(a.ghist + gr * kBins + bin, hr[bin]);
+        } else if (PASS == 0) {
             asm volatile("bar.sync 1, 256;" ::: "memory");   // both halves' counts are in
             if (half == 0 && live) {
                 float thr = -INFINITY;
@@ -308,7 +352,7 @@ __global__ void __launch_bounds__(kFThreads, 1)
                 }
                 a.thr[gr] = thr;
             }
-        } else if (live) {
+        } else if (live && a.nsplit == 1) {
             a.ccount[gr * 2 + half] = n;
         }
     }
@@ -326,18 +370,33 @@ size_t fs_smem_bytes() {
 
 template <int R>
 int fs_run_passes(const CUtensorMap& mq, const CUtensorMap& mk, const FsArgs& a, int64_t units, cudaStream_t s) {
-    dim3 grid((unsigned)(a.nq_pad / kFM), (unsigned)units);
+    dim3 grid((unsigned)(a.nq_pad / kFM), (unsigned)units, (unsigned)a.nsplit);
     const size_t s0 = fs_smem_bytes<R, 0>(), s1 = fs_smem_bytes<R, 1>();
     cudaError_t e = cudaFuncSetAttribute(fs_tc_kernel<R, 0>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s0);
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(fs_tc_kernel<R, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s1);
     if (e != cudaSuccess) return cuda_status(e);
+    const int64_t rows = units * a.nq_pad;
+    if (a.nsplit > 1) {
+        e = cudaMemsetAsync(a.ghist, 0, (size_t)rows * kBins * sizeof(int32_t), s);
+        if (e != cudaSuccess) return cuda_status(e);
+    }
     note_launch();
     fs_tc_kernel<R, 0><<<grid, kFThreads, s0, s>>>(mq, mk, a);
+    if (a.nsplit > 1) {
+        note_launch();
+        fs_thr_kernel<<<(unsigned)((rows + 255) / 256), 256, 0, s>>>(a.ghist, a.qnorm, a.kmax, a.nq, a.nq_pad, units,
+                                                                      a.kb, a.thr);
+        e = cudaMemsetAsync(a.ccount, 0, (size_t)rows * 2 * sizeof(int32_t), s);
+        if (e != cudaSuccess) return cuda_status(e);
+    }
     note_launch();
     fs_tc_kernel<R, 1><<<grid, kFThreads, s1, s>>>(mq, mk, a);
     return cuda_status(cudaGetLastError());
 }
+
+// first candidate block (the sink rule)
+int64_t a_b_lo(const lsa_build_params& p) { return (p.sink + p.pool - 1) / p.pool; }
 
 }  // namespace
 
@@ -368,6 +427,15 @@ int launch_fullscan_tc(const lsa_index* ix, const lsa_select_params* sp, const f
     float* thr = A.alloc<float>(U * nq_chunk_max);
     int32_t* cand = A.alloc<int32_t>(U * nq_chunk_max * 2 * kHalfCap);
     int32_t* ccount = A.alloc<int32_t>(U * nq_chunk_max * 2);
+    // small calls split each tile's block range so that about two CTAs run per SM
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int64_t tiles_q = nq_chunk_max / kFM * U;
+    const int64_t tiles_k = (nb - a_b_lo(p) + kFN - 1) / kFN;
+    int64_t nsplit = (2 * (int64_t)sms + tiles_q - 1) / tiles_q;
+    nsplit = std::max<int64_t>(1, std::min<int64_t>(nsplit, tiles_k / 8));
+    int32_t* ghist = nsplit > 1 ? A.alloc<int32_t>(U * nq_chunk_max * kBins) : nullptr;
     if (A.status != LSA_OK) return A.status;
     cudaError_t e = cudaMemsetAsync(absmax, 0, sizeof(uint32_t), s);
     if (e != cudaSuccess) return cuda_status(e);
@@ -385,7 +453,7 @@ int launch_fullscan_tc(const lsa_index* ix, const lsa_select_params* sp, const f
     FsArgs a{};
     a.nb = nb;
     a.nb_pad = nb_pad;
-    a.b_lo = (p.sink + p.pool - 1) / p.pool;
+    a.b_lo = a_b_lo(p);
     a.hkv = hkv;
     a.pool = p.pool;
     a.window = sp->window;
@@ -397,6 +465,8 @@ int launch_fullscan_tc(const lsa_index* ix, const lsa_select_params* sp, const f
     a.cand = cand;
     a.ccount = ccount;
     a.err = ix->err;
+    a.nsplit = (int)nsplit;
+    a.ghist = ghist;
     for (int64_t q0 = 0; q0 < nq; q0 += nq_chunk_max) {
         const int64_t nqc = std::min(nq_chunk_max, nq - q0);
         const int64_t nqc_pad = (nqc + kFM - 1) / kFM * kFM;

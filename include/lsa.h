@@ -224,7 +224,7 @@ int lsa_pca_map(const void* K, int64_t batch, int64_t n_tokens, int64_t ld_token
 
 /* The quadratic baseline indexer: every candidate block is scored, no tree.
  * Same arguments and output format as lsa_select (beam is ignored).
- * Calls of 512 or more (query, KV head) pairs with r <= 64 first filter on the
+ * Calls of 64 or more (query, KV head) pairs with r <= 64 first filter on the
  * tensor cores (fp16 scores of 128 queries x 256 blocks per tile; a per-query
  * histogram gives a threshold that provably keeps every block of the exact
  * top ceil(K/P)), then rank the survivors with the exact fp32 arithmetic of

@@ -37,6 +37,22 @@ def test_traffic_record_holds_only_for_the_captured_source(tmp_path, monkeypatch
     assert bench.recorded_traffic("kern<1>", "wl", "k.cu") is None
 
 
+def test_traffic_record_over_several_source_files(tmp_path, monkeypatch):
+    a, b = "__global__ void k() {}\n", "// helper header\n"
+    sha = hashlib.sha256((a + b).encode()).hexdigest()[:16]
+    csrc = tmp_path / "hierarchical_latent_key_gemm_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "k.cu").write_text(a)
+    (csrc / "h.cuh").write_text(b)
+    prof = tmp_path / "profiles"
+    prof.mkdir()
+    (prof / "traffic.txt").write_text(f"kern<1> | wl | k.cu+h.cuh | {sha} | 777 | test record\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    assert bench.recorded_traffic("kern<1>", "wl", "k.cu+h.cuh") == 777
+    (csrc / "h.cuh").write_text(b + "// edited\n")      # a change in any of the files voids it
+    assert bench.recorded_traffic("kern<1>", "wl", "k.cu+h.cuh") is None
+
+
 def test_traffic_record_absent(tmp_path, monkeypatch):
     (tmp_path / "hierarchical_latent_key_gemm_b200" / "csrc").mkdir(parents=True)
     (tmp_path / "hierarchical_latent_key_gemm_b200" / "csrc" / "k.cu").write_text("x")

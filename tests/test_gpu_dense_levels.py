@@ -1,4 +1,6 @@
-"""Dense-level scoring of large selections (node_scores.cu).  The upper tree
+"""Paths that must give the same bits as the per-query search.
+
+Dense-level scoring of large selections (node_scores.cu).  The upper tree
 levels whose parents all fit in the beam are scored for tiles of queries
 before the per-query search, which then reads one score per node of those
 levels.  The selection must be the same, bit for bit, as that of the
@@ -6,7 +8,12 @@ per-query search scoring every node itself (the scores are the same fp32
 values), with one buffer of scores and with the buffer forced small so that
 the queries run in several chunks.  The per-query search is the path the
 other parity tests check against the oracle; this pins the dense form to it
-on every tree shape the workloads use."""
+on every tree shape the workloads use.
+
+Full scan: calls of 64 or more (query, KV head) pairs filter on the tensor
+cores and rank the survivors exactly (a few query tiles split the block range
+over CTAs); smaller calls scan every block per query.  All must give the same
+selection for the same query."""
 import pytest
 import torch
 
@@ -99,4 +106,24 @@ def test_dense_levels_scored_blocks():
     for o in outs[1:]:
         for a, b in zip(outs[0], o):
             assert torch.equal(a, b)
+    ix.free()
+
+
+@pytest.mark.parametrize("name,over", [
+    ("int_exact_16k", {}),
+    ("gqa_128k", dict(n_tokens=16384 + 5, needles=0, components=512)),
+])
+def test_fullscan_tensor_core_filter_matches_per_query_scan(name, over):
+    w = WORKLOADS[name].scaled(**over)
+    inp = make_inputs(w, seed=34, device="cuda")
+    ix = lsa.lsa_build_index(TU.build_params(w), inp["K"], inp["W"])
+    sp = TU.select_params(w)
+    big_i, big_c = lsa.lsa_fullscan_select(ix, sp, inp["Q"])          # tensor-core filter, whole tiles
+    small = 60 // w.hkv                                                # under 64 pairs: per-query scan
+    for q0 in (0, 5000, w.n_tokens - 300):
+        for n in (small, 300):                                         # 300: tensor cores, split block range
+            Q = inp["Q"][:, q0:q0 + n].contiguous()
+            i, c = lsa.lsa_fullscan_select(ix, sp, Q, q_pos0=q0)
+            assert torch.equal(c, big_c[:, q0:q0 + n]) and torch.equal(i, big_i[:, q0:q0 + n])
+    assert lsa.lsa_check(ix) == lsa.LSA_OK
     ix.free()
