@@ -300,6 +300,67 @@ __device__ __forceinline__ int find_owner(const int* pre, int nk, int t) {
     return lo;
 }
 
+// Bitonic sort of IPT * THREADS ids (ids[0, nsel) padded with INT32_MAX), IPT
+// per thread in registers: item i = IPT tid + k; strides below IPT inside a
+// thread, up to 16 IPT across lanes by shuffles, 32 IPT and up through shared
+// memory.  Leaves the sorted items in arr (which may alias ids), then a barrier.
+template <int IPT, int THREADS>
+__device__ void bitonic_ids(const int* ids, int nsel, int* arr) {
+    constexpr int M = IPT * THREADS;
+    int v[IPT];
+#pragma unroll
+    for (int k = 0; k < IPT; ++k) {
+        const int i = IPT * threadIdx.x + k;
+        v[k] = i < nsel ? ids[i] : INT32_MAX;
+    }
+    __syncthreads();   // ids and arr may be read and written below
+    for (int size = 2; size <= M; size <<= 1) {
+        for (int stride = size >> 1; stride > 0; stride >>= 1) {
+            if (stride >= 32 * IPT) {
+#pragma unroll
+                for (int k = 0; k < IPT; ++k) arr[IPT * threadIdx.x + k] = v[k];
+                __syncthreads();
+#pragma unroll
+                for (int k = 0; k < IPT; ++k) {
+                    const int i = IPT * threadIdx.x + k;
+                    const int y = arr[i ^ stride];
+                    const bool asc = (i & size) == 0;
+                    const bool lower = (i & stride) == 0;
+                    v[k] = (lower == asc) ? min(v[k], y) : max(v[k], y);
+                }
+                __syncthreads();
+            } else if (stride >= IPT) {
+#pragma unroll
+                for (int k = 0; k < IPT; ++k) {
+                    const int i = IPT * threadIdx.x + k;
+                    const int y = __shfl_xor_sync(0xffffffffu, v[k], stride / IPT);
+                    const bool asc = (i & size) == 0;
+                    const bool lower = (i & stride) == 0;
+                    v[k] = (lower == asc) ? min(v[k], y) : max(v[k], y);
+                }
+            } else {
+                // pairs (k, k + stride) inside the thread; every stride is
+                // unrolled so every register index is a constant
+#pragma unroll
+                for (int st = IPT / 2; st >= 1; st >>= 1) {
+                    if (st != stride) continue;
+#pragma unroll
+                    for (int k = 0; k < IPT; ++k) {
+                        if (k & st) continue;
+                        const bool asc = ((IPT * (int)threadIdx.x + k) & size) == 0;
+                        const int lo = min(v[k], v[k + st]), hi = max(v[k], v[k + st]);
+                        v[k] = asc ? lo : hi;
+                        v[k + st] = asc ? hi : lo;
+                    }
+                }
+            }
+        }
+    }
+#pragma unroll
+    for (int k = 0; k < IPT; ++k) arr[IPT * threadIdx.x + k] = v[k];
+    __syncthreads();
+}
+
 // The selection row of the query at position pos: the nsel chosen block ids
 // (ids[0, nsel), any order) sorted ascending (in `work`, which needs room for
 // max(nsel, THREADS * kSortIpt) ints and may alias nothing else), then sink
@@ -323,65 +384,10 @@ __device__ void emit_row(const int* ids, int* work, int nsel, int64_t pos, int s
         }
         __syncthreads();
     } else if (nsel <= kSortIpt * THREADS) {
-        // bitonic sort of IPT * THREADS items (padded with INT32_MAX), IPT per
-        // thread in registers: item i = IPT tid + k; strides below IPT inside
-        // a thread, up to 16 IPT across lanes by shuffles, 32 IPT and up
-        // through shared memory
-        constexpr int IPT = kSortIpt;
-        constexpr int M = IPT * THREADS;
-        int v[IPT];
-        const int* src = ids;
-#pragma unroll
-        for (int k = 0; k < IPT; ++k) {
-            const int i = IPT * threadIdx.x + k;
-            v[k] = i < nsel ? src[i] : INT32_MAX;
-        }
-        __syncthreads();   // src and arr may be read and written below
-        for (int size = 2; size <= M; size <<= 1) {
-            for (int stride = size >> 1; stride > 0; stride >>= 1) {
-                if (stride >= 32 * IPT) {
-#pragma unroll
-                    for (int k = 0; k < IPT; ++k) arr[IPT * threadIdx.x + k] = v[k];
-                    __syncthreads();
-#pragma unroll
-                    for (int k = 0; k < IPT; ++k) {
-                        const int i = IPT * threadIdx.x + k;
-                        const int y = arr[i ^ stride];
-                        const bool asc = (i & size) == 0;
-                        const bool lower = (i & stride) == 0;
-                        v[k] = (lower == asc) ? min(v[k], y) : max(v[k], y);
-                    }
-                    __syncthreads();
-                } else if (stride >= IPT) {
-#pragma unroll
-                    for (int k = 0; k < IPT; ++k) {
-                        const int i = IPT * threadIdx.x + k;
-                        const int y = __shfl_xor_sync(0xffffffffu, v[k], stride / IPT);
-                        const bool asc = (i & size) == 0;
-                        const bool lower = (i & stride) == 0;
-                        v[k] = (lower == asc) ? min(v[k], y) : max(v[k], y);
-                    }
-                } else {
-                    // pairs (k, k + stride) inside the thread; every stride is
-                    // unrolled so every register index is a constant
-#pragma unroll
-                    for (int st = IPT / 2; st >= 1; st >>= 1) {
-                        if (st != stride) continue;
-#pragma unroll
-                        for (int k = 0; k < IPT; ++k) {
-                            if (k & st) continue;
-                            const bool asc = ((IPT * (int)threadIdx.x + k) & size) == 0;
-                            const int lo = min(v[k], v[k + st]), hi = max(v[k], v[k + st]);
-                            v[k] = asc ? lo : hi;
-                            v[k + st] = asc ? hi : lo;
-                        }
-                    }
-                }
-            }
-        }
-#pragma unroll
-        for (int k = 0; k < IPT; ++k) arr[IPT * threadIdx.x + k] = v[k];
-        __syncthreads();
+        // the smallest network that holds nsel (nsel is the same in every thread)
+        if (kSortIpt >= 1 && nsel <= THREADS) bitonic_ids<1, THREADS>(ids, nsel, arr);
+        else if (kSortIpt >= 2 && nsel <= 2 * THREADS) bitonic_ids<(kSortIpt >= 2 ? 2 : 1), THREADS>(ids, nsel, arr);
+        else bitonic_ids<kSortIpt, THREADS>(ids, nsel, arr);
     } else {
         // bitonic sort, padded to a power of two
         int M = 1;
