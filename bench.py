@@ -364,16 +364,16 @@ def decode_measure(w, dev, seed, warmup, world=1, extra=True):
     e1.record()
     torch.cuda.synchronize()
     build_ms = e0.elapsed_time(e1)
-    idx = torch.empty((w.batch, 1, w.hkv, w.max_sel), dtype=torch.int32, device=dev)
-    cnt = torch.empty((w.batch, 1, w.hkv), dtype=torch.int32, device=dev)
-    O = torch.empty((w.batch, 1, w.hq, w.d), dtype=torch.bfloat16, device=dev)
-    lse = torch.empty((w.batch, 1, w.hq), dtype=torch.float32, device=dev)
     qs = [Q[:, s:s + 1].contiguous() for s in range(w.decode_steps)]
+    # decode through the public decode path: the append as a call, select +
+    # attention replayed from the CUDA graph captured at set-up (pipeline.DecodeStep)
+    from hierarchical_latent_key_gemm_b200.pipeline import DecodeStep
+    c0 = lsa.lsa_launch_count()
+    ds = DecodeStep(ix, sp, K, V, w.hq, w.max_sel)
+    per_replay = (lsa.lsa_launch_count() - c0) // 2     # set-up ran select + attention eagerly once, then captured
 
     def step(s):
-        lsa.lsa_append(ix, K, 1)
-        lsa.lsa_select(ix, sp, qs[s], q_pos0=N + s, idx=idx, cnt=cnt, max_sel=w.max_sel)
-        lsa.lsa_sparse_attn(qs[s], K, V, idx, cnt, w.hkv, O=O, lse=lse)
+        ds.step(qs[s], N + s)
 
     warm = min(warmup, w.decode_steps // 4)
     for s in range(warm):
@@ -390,12 +390,14 @@ def decode_measure(w, dev, seed, warmup, world=1, extra=True):
     clk = clocks.stop()
     n_timed = w.decode_steps - warm
     ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / n_timed
-    launches = lsa.lsa_launch_count() - launches0
+    # appends launch as calls; every replay runs the captured select + attention kernels
+    launches = lsa.lsa_launch_count() - launches0 + n_timed * per_replay
     st = lsa.lsa_check(ix)
     info = ix.info()
+    del ds
     ext = decode_extra(w, inp, ix, sp, dev) if extra else None
     ix.free()
-    del inp, idx, cnt, O, lse, qs
+    del inp, qs
     torch.cuda.empty_cache()
     return {"ms_per_step": ms, "steps": n_timed, "warmup": warm, "build_ms": build_ms,
             "index_device_bytes": int(info.device_bytes), "gpu_launches": launches, "status": lsa.strerror(st),

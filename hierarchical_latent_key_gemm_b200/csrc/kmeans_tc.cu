@@ -133,6 +133,7 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
                      int64_t n, int64_t n_pad, int k, int k_pad, const float* __restrict__ cc,
                      const uint32_t* __restrict__ absmax, int32_t* __restrict__ labels, int64_t ldl, int32_t* err) {
     constexpr int KS = split_k(R) / kKC;             // K-chunks
+    constexpr int KSTEPS = (3 * R + 2 + 15) / 16;    // 16-wide MMA steps that hold data (the rest are zero)
     constexpr int A_CHUNK = kTM * 128;               // bytes per A chunk
     constexpr int B_CHUNK = kTN * 128;               // bytes per B stage
     extern __shared__ unsigned char smem_raw[];
@@ -216,6 +217,8 @@ __global__ void __launch_bounds__(kThreadsTC, 1)
                     asm volatile("tcgen05.fence::after_thread_sync;");
 #pragma unroll
                     for (int kk = 0; kk < kKC / 16; ++kk) {
+                        // the zero padding after column 3r + 2 adds nothing: its steps are skipped
+                        if (c * (kKC / 16) + kk >= KSTEPS) break;
                         const uint64_t da = umma_desc(As + c * A_CHUNK + kk * 32);
                         const uint64_t db = umma_desc(Bs + s * B_CHUNK + kk * 32);
                         umma_f16(d, da, db, (c | kk) ? 1u : 0u);
