@@ -5,8 +5,8 @@
 // key band [0, S) and [i0-W+1, i1] with the per-row mask
 // j <= i && (j < S || j >= i-W+1), and write the unnormalised partial
 // (acc, running max, sum of weights) that the long-range gather kernel
-// continues from (LSA explainer, "How does LSA work?" step 3: the selected
-// long-range keys plus the attention sink and a local window).
+// continues from (LSA explainer, "How does LSA work?" step 3: attention
+// covers the chosen distant keys, the first S tokens and the last W).
 //
 // One CTA per 128 rows (one UMMA M), two CTAs per SM:
 //   warp 4   TMA: the Q tile once, then K and V tiles of 32 keys through a

@@ -62,9 +62,9 @@ typedef enum { LSA_F32 = 0, LSA_BF16 = 1 } lsa_dtype;
 
 #define LSA_MAX_LEVELS 4
 
-/* Index construction parameters.  [p5 "How does LSA work?" step 1: keys are
- * pooled and clustered into buckets in a learned latent space, organised as a
- * hierarchy; p2: the hierarchical tree variant.] */
+/* Index construction parameters.  [p5 "How does LSA work?" step 1: blocks of
+ * keys are averaged, mapped to a low-rank latent space and grouped into
+ * buckets that form a tree; p2: the hierarchical tree variant.] */
 typedef struct {
     int64_t batch;          /* sequences (>= 1) */
     int64_t n_tokens;       /* tokens per sequence to index (>= 1) */
@@ -157,8 +157,8 @@ int lsa_build_index_from_tree(const lsa_build_params* params, const void* K, con
  * lower id.  The row of idx lists, ascending, the sink [0, min(S, i+1)), the
  * tokens of the chosen blocks and the window [max(0, i-W+1), i]; cnt holds its
  * length and the rest of the row is -1.  max_sel must be at least
- * ceil(K/P)*P + S + W.  [p3 TL;DR "scores cluster centroids and descends into
- * the best few buckets"; p1; p5 steps 2-3] */
+ * ceil(K/P)*P + S + W.  [p3 TL;DR: the query is compared with centroids first
+ * and only a few buckets are searched; p1; p5 steps 2-3] */
 int lsa_select(const lsa_index* index, const lsa_select_params* params, const void* Q,
                int64_t nq, const int64_t* q_pos, int64_t q_pos0,
                int32_t* idx, int32_t* cnt, int32_t max_sel, void* stream);
@@ -203,8 +203,8 @@ int lsa_select_work(const lsa_index* index, const lsa_select_params* params, con
                     void* stream);
 
 /* Training-free latent map: W = the r leading principal directions of the
- * pooled keys ([p5] "How does LSA work?", the D-LSA options: a training-free
- * option that uses a PCA map).  Every (sequence, KV head)'s keys are pooled as
+ * pooled keys ([p5] "How does LSA work?", the D-LSA options, one of which
+ * needs no training and takes a PCA map).  Every (sequence, KV head)'s keys are pooled as
  * in the build (mean of `pool` consecutive keys, complete blocks only) and all
  * pooled keys form one sample; their covariance (centred, divided by the
  * count, accumulated in fp64) is diagonalised on the device (parallel cyclic
@@ -338,8 +338,8 @@ int lsa_sparse_attn(const void* Q, const void* K, const void* V, const int32_t* 
  *  - bf16 with hq/hkv in {1, 2, 4, 8, 16} takes the band path; other cases
  *    run the lsa_sparse_attn kernels.
  *  - Needs batch*nq*hq*(d+2) floats of stream-ordered scratch (pool memory).
- * [p5 step 3 "selected long-range keys plus the attention sink and a local
- * window"; the kernel is unchanged] */
+ * [p5 step 3: attention covers the chosen distant keys, the first S tokens
+ * and the last W; the attention kernel itself is unchanged] */
 int lsa_sparse_attn_banded(const void* Q, const void* K, const void* V, const int32_t* idx,
                            const int32_t* cnt, int64_t batch, int64_t nq, int64_t q_pos0,
                            int32_t hq, int32_t hkv, int32_t d, int32_t dtype, int32_t max_sel,
@@ -358,8 +358,8 @@ int lsa_sparse_attn_banded(const void* Q, const void* K, const void* V, const in
 int lsa_append(lsa_index* index, const void* K, int64_t n_new, void* stream);
 
 /* Decode maintenance, part 1 (the pages say nothing about keeping the index
- * up during decode beyond "each new token attends back over the whole
- * history", p5 "Prefill, decode and training"; this is the plainest
+ * up during decode, only that every generated token looks at all earlier
+ * tokens, p5 "Prefill, decode and training"; this is the plainest
  * upkeep that leaves the selection rule unchanged).  Lays the leaf buckets of
  * every unit out again from the current leaf labels: each leaf's blocks in
  * ascending order, the blocks that lsa_append gave to a full leaf

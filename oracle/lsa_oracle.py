@@ -28,14 +28,15 @@ Sources, cited below by key and section:
        They Compare Against", section "How does LSA work?" (steps 1-3) and
        section "Prefill, decode and training"
 
-What the pages fix: keys are pooled and clustered into buckets in a latent
-space, organised as a hierarchy [p5 step 1; p2; p4]; a query scores the bucket
-centroids, descends into the best few buckets and scores the keys inside them
-[p1; p3 TL;DR; p5 step 2]; the query then attends exactly to the selected
-long-range keys plus the attention sink and a local window, with an unchanged
-attention kernel [p5 step 3; p3 flowchart, the sparse-attention node].  The old
-indexer scores every key [p3 flowchart, red path].  Decode attends each new
-token over the whole history [p5 "Prefill, decode and training"].
+What the pages fix: blocks of keys are averaged, mapped to a latent space and
+grouped into buckets that form a tree [p5 step 1; p2; p4]; a query is compared with
+the bucket centroids, goes on into a few of the best buckets only, and compares
+itself with the keys in those [p1; p3 TL;DR; p5 step 2]; exact attention then
+covers the chosen distant keys, the first S tokens and the last W tokens, the
+attention itself being unchanged [p5 step 3; p3 flowchart, the sparse-attention
+node].  The old
+indexer scores every key [p3 flowchart, red path].  In decode, every generated
+token looks at all earlier tokens [p5 "Prefill, decode and training"].
 
 Readings where the pages are silent:
   R1  one latent map W (d x r) serves keys and queries.
@@ -69,8 +70,8 @@ Readings where the pages are silent:
       the latent keys of its blocks, appended ones included; an upper node
       from its children's refreshed centroids), by the rules of
       ``kmeans_update``.  Right after a build this changes nothing (R10).
-  R17 the training-free map [p5 "How does LSA work?", the D-LSA options: "a
-      training-free option that uses a PCA map"]: W = the r leading principal
+  R17 the training-free map [p5 "How does LSA work?", the D-LSA options, one
+      of which needs no training and takes a PCA map]: W = the r leading principal
       directions of the pooled keys of every (sequence, KV head), i.e. the
       eigenvectors of their covariance (centred, divided by the count) for the
       r largest eigenvalues, in descending order; each column's entry of
@@ -424,8 +425,8 @@ def sparse_attention(q: np.ndarray, K: np.ndarray, V: np.ndarray, sel: np.ndarra
 
 
 # ---------------------------------------------------------------------------
-# Decode  [p5 "Prefill, decode and training": each generated token attends over
-# the whole history; p4 "Prompt processing is not response generation"]
+# Decode  [p5 "Prefill, decode and training": every generated token looks at
+# all earlier tokens; p4 "Prompt processing is not response generation"]
 # ---------------------------------------------------------------------------
 def nearest_leaf(tree: Tree, x: np.ndarray) -> int:
     """argmin over all leaves of ||x - c||^2 with frozen centroids (R13, R7)."""
