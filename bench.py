@@ -48,6 +48,8 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-extra", action="store_true")
+    ap.add_argument("--e2e-chunks", type=int, default=16,
+                    help="query chunks of the end-to-end pipeline (each chunk's O goes down while the next computes)")
     ap.add_argument("--cpu-sample-queries", type=int, default=CPU_SAMPLE_QUERIES)
     ap.add_argument("--query-range", default=None,
                     help="START:COUNT - profiling case: full index, select+attention on that query range only")
@@ -460,7 +462,7 @@ def run_e2e(args, w, inp, bp, sp, idx, cnt, O, lse, dev, world):
     """Same metric through the public API with HOST buffers: every step copies
     Q, K, V, W from pinned host memory and reads O back
     (hierarchical_latent_key_gemm_b200.pipeline.HostPrefill: K, W up, index
-    build while V and then Q go up (Q in 16 chunks), select + banded attention
+    build while V and then Q go up (Q in --e2e-chunks chunks), select + banded attention
     per chunk, each O chunk back while the next computes)."""
     import torch
     from hierarchical_latent_key_gemm_b200.pipeline import HostPrefill
@@ -469,7 +471,7 @@ def run_e2e(args, w, inp, bp, sp, idx, cnt, O, lse, dev, world):
     hV = inp["V"].cpu().pin_memory()
     hW = inp["W"].cpu().pin_memory()
     hO = torch.empty(O.shape, dtype=O.dtype, pin_memory=True)
-    hp = HostPrefill(bp, sp, hQ, hK, hV, hW, hO, w.sink, w.window, chunks=16, device=dev)
+    hp = HostPrefill(bp, sp, hQ, hK, hV, hW, hO, w.sink, w.window, chunks=args.e2e_chunks, device=dev)
 
     n = max(1, min(args.steps, 3))
     hp.run().free()
@@ -484,7 +486,8 @@ def run_e2e(args, w, inp, bp, sp, idx, cnt, O, lse, dev, world):
     ms = max_over_ranks(t0.elapsed_time(t1), world, dev) / n
     return {"value": world * w.n_tokens * w.batch / (ms / 1e3), "unit": UNIT, "ms_per_step": ms,
             "h2d_bytes_per_step": hp.h2d_bytes, "d2h_bytes_per_step": hp.d2h_bytes,
-            "pipeline": "3 streams; K, W up, then V during the build; Q up and O down in 16 chunks overlapped with select + attention"}
+            "pipeline": (f"3 streams; K, W up, then V during the build; Q up and O down in {args.e2e_chunks} chunks "
+                         "overlapped with select + attention")}
 
 
 def run_extra(w, inp, bp, sp, dev, select_ms, idx, cnt):
@@ -676,12 +679,23 @@ def stage_rooflines(w, inp, bp, dev, peaks, build_ms, select_ms, attn_ms, nodes,
     attn_flops = sel_tokens * d * 4 * G
     attn_bytes = sel_tokens * d * 2 * 2
     attn_tf = attn_flops / (attn_ms / 1e3) / 1e12
+    # the projections also do d x r fused multiply-adds per mean row on CUDA cores: their fp32 rate
+    # against the peak from unit counts and clock (SMs x 128 FP32 lanes x 2 flops x 1.965 GHz)
+    fp32_peak = torch.cuda.get_device_properties(dev).multi_processor_count * 128 * 2 * 1.965e9 / 1e12
+    a1_fl = units * nb * d * r * 2
+    a5_fl = w.batch * nq * w.hkv * d * r * 2
+
+    def alu(fl, ms):
+        return {"flops": fl, "achieved_TFLOPs": fl / (ms / 1e3) / 1e12, "peak_TFLOPs": fp32_peak,
+                "frac": fl / (ms / 1e3) / 1e12 / fp32_peak,
+                "note": "fp32 FMA work of the projection of the mean rows; peak from SM count x 128 lanes x "
+                        "2 flops x 1.965 GHz"}
     return {
         "build": {"ms": build_ms, "note": "a1 + a2 + upper levels + bucket layout, in the step"},
         "a1_project_pool": {"ms": t_a1, "bytes": a1, "achieved_GBps": a1 / (t_a1 / 1e3) / 1e9, "peak_GBps": hbm,
-                            "frac": a1 / (t_a1 / 1e3) / 1e9 / hbm, "bound": "hbm"},
+                            "frac": a1 / (t_a1 / 1e3) / 1e9 / hbm, "bound": "hbm", "alu": alu(a1_fl, t_a1)},
         "a5_query_latent": {"ms": t_a5, "bytes": a5, "achieved_GBps": a5 / (t_a5 / 1e3) / 1e9, "peak_GBps": hbm,
-                            "frac": a5 / (t_a5 / 1e3) / 1e9 / hbm, "bound": "hbm"},
+                            "frac": a5 / (t_a5 / 1e3) / 1e9 / hbm, "bound": "hbm", "alu": alu(a5_fl, t_a5)},
         "a2_leaf_kmeans": {"ms": t_a2, "flops": a2, "rounds": w.lloyd_iters,
                            "achieved_TFLOPs": a2 / (t_a2 / 1e3) / 1e12, "peak_TFLOPs": tf,
                            "frac": a2 / (t_a2 / 1e3) / 1e12 / tf, "bound": "tensor",
