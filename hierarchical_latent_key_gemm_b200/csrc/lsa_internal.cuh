@@ -189,6 +189,13 @@ struct PreScores {
     int64_t ld;
     int levels;
     int off[LSA_MAX_LEVELS];
+    // optional (leaf tiles): per row the kept nodes of the last dense level
+    // [row][beam] and their count (-1: the row runs the whole search), and the
+    // scores of their children, row-major [row][s2_ld] in kept-node order
+    const int32_t* b1;
+    const int32_t* nb1;
+    const float* S2;
+    int64_t s2_ld;
 };
 int launch_select_rows(const lsa_index* ix, const lsa_select_params* sp, const float* qbar, int64_t nq_stride,
                        int64_t nq, const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt, int max_sel,

@@ -19,7 +19,7 @@
 // not depend on which kernel scored a node.
 #include <atomic>
 
-#include "lsa_internal.cuh"
+#include "select_common.cuh"
 
 namespace lsa {
 namespace {
@@ -148,6 +148,391 @@ __global__ __launch_bounds__(kNsThreads) void node_scores_kernel(const NsArgs a)
     }
 }
 
+// ------------------------------------------------------------ leaf tiles
+// When the tree's only sparse level is its leaf level, the leaves are scored
+// for many queries at a time as well:
+//   1. beam_dense_kernel (one warp per (query, KV head) row): the kept nodes of
+//      the last dense level, i.e. the best `beam` of all its eligible nodes by
+//      (score desc, id asc), from the dense scores; and for each kept node the
+//      first slot of its children in the row's leaf-score buffer;
+//   2. the (row, kept node) pairs grouped by node (counting sort);
+//   3. leaf_scores_kernel: per node, 64 of its pairs x 64 of its children at a
+//      time, the register-tiled fp32 product in the per-query kernel's order,
+//      each score written to its row's slot;
+//   4. the per-query kernel starts from those kept nodes and reads each leaf
+//      candidate's score from its slot (one lane per candidate) instead of
+//      scoring its row.
+// The selection of step 1 is exact (radix select on the order-preserving
+// key, ties by id), so the kept set equals the per-query search's.  A row
+// whose kept nodes have more than kLtCap children falls back to the
+// per-query search.
+constexpr int kLtCap = 3072;    // leaf slots per row
+constexpr int kLtPairs = 128;   // (row, kept node) pairs per leaf_scores CTA
+constexpr int kLtKids = 32;     // children per pass of a leaf_scores CTA
+constexpr int kLtWarps = 8;     // rows per beam kernel CTA
+constexpr int kLtMaxBeam = 128;    // leaf tiles for beams up to this
+
+struct LtArgs {
+    int64_t rows, nqc, nq_stride, units;
+    int hkv, beam, window, pool;
+    const int64_t* q_pos;       // the chunk's positions (sequence stride nq_stride), or null
+    int64_t q_pos0;
+    int64_t pos_shift;
+    const float* qbar;          // the chunk's latent queries (sequence stride nq_stride)
+    const float* S;             // dense scores, rows (bseq * nqc + qi) * hkv + h
+    int64_t ld;
+    int off1, n1;               // last dense level: its column in S and its size
+    const int64_t* mp1;         // its minpos [units * n1] (tree order)
+    const int32_t* id1;         // its ids
+    const int32_t* coff1;       // [units * n1 + 1] global child positions in the leaf level
+    int n2;                     // leaves per unit
+    const float* cent2;         // leaf centroids [units * n2][r], tree order
+    const int64_t* mp2;
+    const int32_t* id2;
+    int32_t* b1;                // [rows][beam] kept positions of the last dense level
+    int32_t* nb1;               // [rows] their count; -1: the row falls back
+    int32_t* sb;                // [rows][beam + 1] first leaf slot of each kept node; [n] = total
+    float* S2;                  // [rows][kLtCap] leaf scores
+    int32_t* ncnt;              // [units * n1] pairs per node (zero on entry, zero on exit)
+    int32_t* noff;              // [units * n1 + 1]
+    int32_t* list;              // [rows * beam] pairs row * beam + e, grouped by node
+    int32_t* toff;              // [units * n1 + 1] first tile of each node
+    int32_t* tnode;             // [max tiles] node of each tile
+};
+
+__device__ __forceinline__ int warp_sum(int v) {
+#pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    return v;
+}
+
+// The k-th largest of the values v (v != 0 only) the enumerator visits, by
+// 8-bit radix passes over a 256-bin histogram of this warp.  Returns the
+// value and in *need how many items equal to it belong to the k largest.
+template <class Enum>
+__device__ uint32_t warp_kth(int k, int* hist, Enum&& each, int* need) {
+    const int lane = threadIdx.x & 31;
+    uint32_t prefix = 0, mask = 0;
+    int kk = k;
+#pragma unroll 1
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int b = lane; b < 256; b += 32) hist[b] = 0;
+        __syncwarp();
+        // lanes that hit the same bin add once for all of them (the scores of a
+        // row share their leading bits, so most lanes hit one bin)
+        each([&](bool valid, uint32_t v) {
+            const bool in = valid && v != 0u && (v & mask) == prefix;
+            const int bin = in ? (int)((v >> shift) & 255u) : -1;
+            const unsigned grp = __match_any_sync(0xffffffffu, bin);
+            if (in && (threadIdx.x & 31) == __ffs(grp) - 1) atomicAdd(&hist[bin], __popc(grp));
+        });
+        __syncwarp();
+        int c[8], sum = 0;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+            c[q] = hist[255 - lane * 8 - q];
+            sum += c[q];
+        }
+        const int incl = warp_incl_scan(sum);
+        const int excl = incl - sum;
+        int dsel = -1, above = 0;
+        if (excl < kk && kk <= incl) {
+            int run = excl;
+#pragma unroll
+            for (int q = 0; q < 8; ++q) {
+                if (dsel < 0 && run + c[q] >= kk) {
+                    dsel = 255 - lane * 8 - q;
+                    above = run;
+                }
+                run += c[q];
+            }
+        }
+        const unsigned bal = __ballot_sync(0xffffffffu, dsel >= 0);
+        const int src = __ffs(bal) - 1;
+        dsel = __shfl_sync(0xffffffffu, dsel, src);
+        above = __shfl_sync(0xffffffffu, above, src);
+        prefix |= (uint32_t)dsel << shift;
+        mask |= 255u << shift;
+        kk -= above;
+        __syncwarp();
+    }
+    *need = kk;
+    return prefix;
+}
+
+// Exact top k by (key desc, id asc) of the candidates the enumerator visits
+// (key 0: not eligible), one warp.  each(f) calls f(valid, key, id, t) for
+// every candidate, 32 at a time with the warp converged; emit(slot, t) is
+// called once per chosen candidate (slots 0 .. count-1, in visiting order).
+// Returns the count, min(k, eligible).
+template <class Each, class Emit>
+__device__ int warp_topk(int k, int* hist, Each&& each, Emit&& emit) {
+    const unsigned lt = (1u << (threadIdx.x & 31)) - 1u;
+    int nel = 0;
+    each([&](bool valid, uint32_t key, int, int) { nel += valid && key != 0u; });
+    nel = warp_sum(nel);
+    uint32_t T = 1u, I = 0xFFFFFFFFu;
+    bool all_eq = true;
+    if (nel > k) {
+        int need;
+        T = warp_kth(k, hist, [&](auto&& f) { each([&](bool valid, uint32_t key, int, int) { f(valid, key); }); },
+                     &need);
+        int neq = 0;
+        each([&](bool valid, uint32_t key, int, int) { neq += valid && key == T; });
+        neq = warp_sum(neq);
+        all_eq = neq == need;
+        if (!all_eq) {
+            // the need smallest ids among the keys equal to T: the need largest of ~id
+            int need2;
+            const uint32_t P = warp_kth(need, hist, [&](auto&& f) {
+                each([&](bool valid, uint32_t key, int id, int) { f(valid && key == T, ~(uint32_t)id); });
+            }, &need2);
+            I = ~P;
+        }
+    }
+    int base = 0;
+    each([&](bool valid, uint32_t key, int id, int t) {
+        const bool take = valid && key != 0u &&
+                          (nel <= k || key > T || (key == T && (all_eq || (uint32_t)id <= I)));
+        const unsigned bal = __ballot_sync(0xffffffffu, take);
+        if (take) emit(base + __popc(bal & lt), t);
+        base += __popc(bal);
+    });
+    return base;
+}
+
+__device__ __forceinline__ void lt_row(const LtArgs& a, int64_t row, int64_t* u, int64_t* bound) {
+    const int h = (int)(row % a.hkv);
+    const int64_t bq = row / a.hkv;
+    const int64_t qi = bq % a.nqc, bseq = bq / a.nqc;
+    *u = bseq * a.hkv + h;
+    const int64_t pos = (a.q_pos ? a.q_pos[bseq * a.nq_stride + qi] : a.q_pos0 + qi) - a.pos_shift;
+    *bound = pos - a.window - a.pool + 1;
+}
+
+__global__ __launch_bounds__(kLtWarps * 32) void beam_dense_kernel(const LtArgs a) {
+    extern __shared__ uint32_t lt_smem[];
+    __shared__ int hist_all[kLtWarps][256];
+    const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+    const int64_t row = (int64_t)blockIdx.x * kLtWarps + w;
+    if (row >= a.rows) return;   // warp-uniform; no CTA barrier below
+    int64_t u, bound;
+    lt_row(a, row, &u, &bound);
+    const float* sr = a.S + row * a.ld + a.off1;
+    const int64_t* mp = a.mp1 + u * a.n1;
+    const int32_t* id = a.id1 + u * a.n1;
+    int32_t* out = a.b1 + row * a.beam;
+    uint32_t* keyc = lt_smem + (size_t)w * a.n1;
+    for (int t0 = 0; t0 < a.n1; t0 += 128) {
+        int64_t mpv[4];
+        float sv[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int t = t0 + j * 32 + lane;
+            mpv[j] = INT64_MAX;
+            sv[j] = 0.f;
+            if (t < a.n1) {
+                mpv[j] = __ldg(mp + t);
+                sv[j] = __ldg(sr + t);
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int t = t0 + j * 32 + lane;
+            if (t < a.n1) keyc[t] = mpv[j] <= bound ? fkey(sv[j]) : 0u;
+        }
+    }
+    __syncwarp();
+    auto each = [&](auto&& f) {
+        for (int t0 = 0; t0 < a.n1; t0 += 32) {
+            const int t = t0 + lane;
+            const bool valid = t < a.n1;
+            const uint32_t key = valid ? keyc[t] : 0u;
+            // ids matter only for ties at the threshold and are read then
+            f(valid, key, key != 0u ? __ldg(id + t) : 0, t);
+        }
+    };
+    const int n = warp_topk(a.beam, hist_all[w], each, [&](int slot, int t) { out[slot] = t; });
+    __syncwarp();
+    // first leaf slot of each kept node's children, in kept order
+    const int32_t* co = a.coff1 + u * a.n1;
+    int32_t* sbr = a.sb + row * (a.beam + 1);
+    int carry = 0;
+    for (int e0 = 0; e0 < n; e0 += 32) {
+        const int e = e0 + lane;
+        int c = 0;
+        if (e < n) {
+            const int q = out[e];
+            c = __ldg(co + q + 1) - __ldg(co + q);
+        }
+        const int incl = warp_incl_scan(c);
+        if (e < n) sbr[e] = carry + incl - c;
+        carry += __shfl_sync(0xffffffffu, incl, 31);
+    }
+    if (lane == 0) {
+        sbr[n] = carry;
+        a.nb1[row] = carry <= kLtCap ? n : -1;
+    }
+}
+
+// sort key of every (row, kept node) pair: the node (units * n1 for a pair
+// that does not exist, which sorts last); value: row * beam + e
+__global__ void lt_keys_kernel(const LtArgs a, uint32_t* __restrict__ keys, int32_t* __restrict__ vals) {
+    const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (e >= a.rows * a.beam) return;
+    const int64_t row = e / a.beam;
+    const int k = (int)(e % a.beam);
+    const int n = a.nb1[row];
+    uint32_t key = (uint32_t)(a.units * a.n1);
+    if (k < n) {   // (n < 0: the row falls back)
+        const int64_t u = (row / a.hkv / a.nqc) * a.hkv + row % a.hkv;
+        key = (uint32_t)(u * a.n1 + a.b1[row * a.beam + k]);
+    }
+    keys[e] = key;
+    vals[e] = (int32_t)e;
+}
+
+// first pair of every node in the sorted keys (noff[g] = lower bound of g),
+// and the node's tile count
+__global__ void lt_bounds_kernel(const LtArgs a, const uint32_t* __restrict__ skeys, int64_t npairs) {
+    const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    const int64_t nodes = a.units * a.n1;
+    if (g > nodes) return;
+    int64_t lo = 0, hi = npairs;   // first index with key >= g
+    while (lo < hi) {
+        const int64_t mid = (lo + hi) >> 1;
+        if (skeys[mid] < (uint32_t)g) lo = mid + 1; else hi = mid;
+    }
+    a.noff[g] = (int32_t)lo;
+}
+
+// node of every tile (each node's thread writes its run of tiles)
+__global__ void lt_tile_nodes_kernel(const LtArgs a) {
+    const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (g >= a.units * a.n1) return;
+    for (int t = a.toff[g]; t < a.toff[g + 1]; ++t) a.tnode[t] = (int32_t)g;
+}
+
+__global__ void lt_tiles_kernel(const LtArgs a) {
+    const int64_t g = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+    if (g >= a.units * a.n1) return;
+    a.ncnt[g] = (a.noff[g + 1] - a.noff[g] + kLtPairs - 1) / kLtPairs;
+}
+
+// out[i][j] (pairs 4 tq + i, children 4 tn + j) = what lane g of a group of
+// r/16 lanes holds before the butterfly (see chain/tree above), with the pair
+// and child operands transposed in shared memory at strides PQ and PC
+template <int R, int PQ, int PC>
+__device__ __forceinline__ void lt_chain(const float* qs, const float* cs, int tq, int tn, int c,
+                                         float (&acc)[16]) {
+#pragma unroll
+    for (int e = 0; e < 16; ++e) acc[e] = 0.f;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        const int d = 8 * c + j;
+        const float4 x = *reinterpret_cast<const float4*>(qs + d * PQ + 4 * tq);
+        const float4 y = *reinterpret_cast<const float4*>(cs + d * PC + 4 * tn);
+        const float av[4] = {x.x, x.y, x.z, x.w}, bv[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[i * 4 + k] = __fmaf_rn(av[i], bv[k], acc[i * 4 + k]);
+    }
+}
+template <int R, int PQ, int PC, int G, int O>
+__device__ __forceinline__ void lt_tree(const float* qs, const float* cs, int tq, int tn, float (&out)[16]) {
+    constexpr int LPC = R / 16;
+    if constexpr (O == LPC) {
+        float t[16];
+        lt_chain<R, PQ, PC>(qs, cs, tq, tn, G, out);
+        lt_chain<R, PQ, PC>(qs, cs, tq, tn, LPC + G, t);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) out[e] = __fadd_rn(out[e], t[e]);
+    } else {
+        float t[16];
+        lt_tree<R, PQ, PC, G, 2 * O>(qs, cs, tq, tn, out);
+        lt_tree<R, PQ, PC, (G ^ O), 2 * O>(qs, cs, tq, tn, t);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) out[e] = __fadd_rn(out[e], t[e]);
+    }
+}
+
+// One CTA per tile of up to 128 pairs of one node: the pairs' latent queries
+// and the node's children (32 at a time) transposed into shared memory, the
+// 128 x 32 scores in the per-query kernel's order, each into its row's slot.
+template <int R>
+__global__ __launch_bounds__(kNsThreads) void leaf_scores_kernel(const LtArgs a) {
+    constexpr int PQ = kLtPairs + 4, PC = kLtKids + 4;
+    __shared__ __align__(16) float qs[R * PQ];
+    __shared__ __align__(16) float cs[R * PC];
+    __shared__ int64_t prow[kLtPairs];
+    __shared__ int pslot[kLtPairs];
+    const int64_t nodes = a.units * a.n1;
+    const int64_t t = blockIdx.x;
+    if (t >= a.toff[nodes]) return;   // CTA-uniform
+    const int64_t g = a.tnode[t];     // toff[g] <= t < toff[g + 1]
+    const int64_t j0 = a.noff[g] + (t - a.toff[g]) * kLtPairs;
+    const int np = (int)min((int64_t)kLtPairs, (int64_t)a.noff[g + 1] - j0);
+    const int tid = threadIdx.x;
+    const int tn = tid % (kLtKids / 4), tq = tid / (kLtKids / 4);   // 8 x 32 threads: 4 children x 4 pairs each
+    if (tid < kLtPairs) {
+        int64_t r = -1;
+        int sl = 0;
+        if (tid < np) {
+            const int64_t e = a.list[j0 + tid];
+            r = e / a.beam;
+            sl = a.sb[r * (a.beam + 1) + (int)(e % a.beam)];
+        }
+        prow[tid] = r;
+        pslot[tid] = sl;
+    }
+    __syncthreads();
+    // the pairs' latent queries, transposed (pairs past np are zero)
+    for (int e = tid; e < kLtPairs * (R / 4); e += kNsThreads) {
+        const int i = e / (R / 4), d4 = e % (R / 4);
+        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (i < np) {
+            const int64_t r = prow[i];
+            const int h = (int)(r % a.hkv);
+            const int64_t bq = r / a.hkv;
+            const int64_t qrow = ((bq / a.nqc) * a.nq_stride + bq % a.nqc) * a.hkv + h;
+            v = *reinterpret_cast<const float4*>(a.qbar + qrow * R + 4 * d4);
+        }
+        qs[(4 * d4 + 0) * PQ + i] = v.x;
+        qs[(4 * d4 + 1) * PQ + i] = v.y;
+        qs[(4 * d4 + 2) * PQ + i] = v.z;
+        qs[(4 * d4 + 3) * PQ + i] = v.w;
+    }
+    const int c_beg = a.coff1[g], nc = a.coff1[g + 1] - c_beg;   // global leaf positions
+    for (int c0 = 0; c0 < nc; c0 += kLtKids) {
+        __syncthreads();   // qs written; the previous pass is done with cs
+        for (int e = tid; e < kLtKids * (R / 4); e += kNsThreads) {
+            const int j = e / (R / 4), d4 = e % (R / 4);
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (c0 + j < nc) v = *reinterpret_cast<const float4*>(a.cent2 + ((int64_t)c_beg + c0 + j) * R + 4 * d4);
+            cs[(4 * d4 + 0) * PC + j] = v.x;
+            cs[(4 * d4 + 1) * PC + j] = v.y;
+            cs[(4 * d4 + 2) * PC + j] = v.z;
+            cs[(4 * d4 + 3) * PC + j] = v.w;
+        }
+        __syncthreads();
+        if (4 * tq < np) {
+            float sc[16];
+            lt_tree<R, PQ, PC, 0, 1>(qs, cs, tq, tn, sc);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int pi = 4 * tq + i;
+                if (pi < np) {
+                    float* o = a.S2 + prow[pi] * kLtCap + pslot[pi] + c0;
+#pragma unroll
+                    for (int k = 0; k < 4; ++k)
+                        if (c0 + 4 * tn + k < nc) o[4 * tn + k] = sc[i * 4 + k];
+                }
+            }
+        }
+    }
+}
+
 }  // namespace
 
 int dense_levels(const lsa_index* ix, int beam, int max_cols, int* col_off) {
@@ -200,9 +585,13 @@ int launch_node_scores(const lsa_index* ix, const float* qbar, int64_t nq_stride
 constexpr int64_t kDenseMinPairs = 4096;
 constexpr int kDenseMaxCols = 4096;
 constexpr int64_t kDenseChunkBytes = int64_t(1) << 30;
-// test hook (lsa_debug_dense_config): -1 = off, else the pair threshold; chunk bytes
+// test hook (lsa_debug_dense_config): -1 = off, else the pair threshold; chunk bytes;
+// leaf tiles on or off
 std::atomic<int64_t> g_dense_min_pairs{kDenseMinPairs};
 std::atomic<int64_t> g_dense_chunk_bytes{kDenseChunkBytes};
+std::atomic<int> g_leaf_tiles{1};
+// the leaf-tile path runs in chunks whose buffers stay under this
+constexpr int64_t kLtChunkBytes = int64_t(2) << 30;
 
 int launch_select_tree(const lsa_index* ix, const lsa_select_params* sp, const float* qbar, int64_t nq,
                        const int64_t* q_pos, int64_t q_pos0, int32_t* idx, int32_t* cnt, int max_sel,
@@ -218,18 +607,117 @@ int launch_select_tree(const lsa_index* ix, const lsa_select_params* sp, const f
         return launch_select(ix, sp, qbar, nq, q_pos, q_pos0, idx, cnt, max_sel, false, s, work, scored);
     pre.ld = (col_off[pre.levels] + 3) / 4 * 4;
     for (int l = 0; l < pre.levels; ++l) pre.off[l] = col_off[l];
-    const int64_t row_bytes = (int64_t)p.batch * p.hkv * pre.ld * 4;   // one query of every sequence
-    int64_t chunk = g_dense_chunk_bytes.load() / row_bytes;
+    const int64_t hkv = p.hkv;
+    // leaf tiles: the leaf level is the only sparse one (not for the scored-row counter,
+    // which counts the per-query search's own candidates)
+    const bool lt = g_leaf_tiles.load() != 0 && work == nullptr && pre.levels == p.levels - 1 &&
+                    sp->beam <= kLtMaxBeam;
+    const int beam = sp->beam;
+    const int l1 = pre.levels - 1, n1 = p.level_sizes[l1];
+    const int64_t per_row = (int64_t)pre.ld * 4 + (lt ? (int64_t)kLtCap * 4 + (int64_t)(4 * beam + 3) * 4 : 0);
+    const int64_t row_bytes = (int64_t)p.batch * p.hkv * per_row;   // one query of every sequence
+    int64_t chunk = (lt ? kLtChunkBytes : g_dense_chunk_bytes.load()) / row_bytes;
+    if (lt && g_dense_chunk_bytes.load() != kDenseChunkBytes) chunk = g_dense_chunk_bytes.load() / row_bytes;
     if (chunk < 1) chunk = 1;
     if (chunk > nq) chunk = nq;
-    float* S = A.alloc<float>(chunk * p.batch * p.hkv * pre.ld);
+    const int64_t crow = chunk * p.batch * p.hkv;
+    float* S = A.alloc<float>(crow * pre.ld);
+    LtArgs la{};
+    int32_t* scan_scr = nullptr;
+    uint32_t* lt_k0 = nullptr;
+    int32_t* lt_v0 = nullptr;
+    uint32_t* lt_k1 = nullptr;
+    int32_t* lt_v1 = nullptr;
+    int32_t* lt_rs = nullptr;
+    if (lt) {
+        const int64_t nodes = ix->units * n1;
+        la.S2 = A.alloc<float>(crow * kLtCap);
+        la.b1 = A.alloc<int32_t>(crow * beam);
+        la.nb1 = A.alloc<int32_t>(crow);
+        la.sb = A.alloc<int32_t>(crow * (beam + 1));
+        lt_v0 = A.alloc<int32_t>(crow * beam);
+        la.ncnt = A.alloc<int32_t>(nodes);
+        la.noff = A.alloc<int32_t>(nodes + 1);
+        la.toff = A.alloc<int32_t>(nodes + 1);
+        la.tnode = A.alloc<int32_t>((crow * beam + kLtPairs - 1) / kLtPairs + nodes);
+        lt_k0 = A.alloc<uint32_t>(crow * beam);
+        lt_k1 = A.alloc<uint32_t>(crow * beam);
+        lt_v1 = A.alloc<int32_t>(crow * beam);
+        lt_rs = A.alloc<int32_t>(radix_scratch_elems(crow * beam));
+        scan_scr = A.alloc<int32_t>(scan_scratch_elems(nodes) + 1);
+    }
     if (A.status != LSA_OK) return A.status;
     pre.S = S;
-    const int64_t hkv = p.hkv;
+    if (lt) {
+        la.units = ix->units;
+        la.hkv = p.hkv;
+        la.beam = beam;
+        la.window = sp->window;
+        la.pool = p.pool;
+        la.pos_shift = scored ? scored->pos_shift : 0;
+        la.S = S;
+        la.ld = pre.ld;
+        la.off1 = col_off[l1];
+        la.n1 = n1;
+        la.mp1 = ix->ord_mp[l1];
+        la.id1 = ix->ord_id[l1];
+        la.coff1 = ix->ord_coff[l1];
+        la.n2 = p.level_sizes[l1 + 1];
+        la.cent2 = ix->ord_cent[l1 + 1];
+        la.mp2 = ix->ord_mp[l1 + 1];
+        la.id2 = ix->ord_id[l1 + 1];
+        la.nq_stride = nq;
+    }
     for (int64_t q0 = 0; q0 < nq; q0 += chunk) {
         const int64_t nqc = (nq - q0) < chunk ? (nq - q0) : chunk;
-        int st = launch_node_scores(ix, qbar + q0 * hkv * p.r, nq, nqc, pre.levels, col_off, S, pre.ld, s);
+        const float* qb = qbar + q0 * hkv * p.r;
+        int st = launch_node_scores(ix, qb, nq, nqc, pre.levels, col_off, S, pre.ld, s);
         if (st != LSA_OK) return st;
+        if (lt) {
+            la.rows = nqc * p.batch * p.hkv;
+            la.nqc = nqc;
+            la.q_pos = q_pos ? q_pos + q0 : nullptr;
+            la.q_pos0 = q_pos0 + q0;
+            la.qbar = qb;
+            const int64_t nodes = ix->units * n1;
+            const int64_t pairs = la.rows * beam;
+            const size_t dense_smem = (size_t)kLtWarps * n1 * sizeof(uint32_t);
+            cudaError_t e0 = cudaFuncSetAttribute(beam_dense_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                  (int)dense_smem);
+            if (e0 != cudaSuccess) return cuda_status(e0);
+            note_launch();
+            beam_dense_kernel<<<(unsigned)((la.rows + kLtWarps - 1) / kLtWarps), kLtWarps * 32, dense_smem, s>>>(la);
+            // the pairs grouped by node: a stable radix sort on the node
+            note_launch();
+            lt_keys_kernel<<<(unsigned)((pairs + 255) / 256), 256, 0, s>>>(la, lt_k0, lt_v0);
+            int kbits = 8;
+            while (kbits < 32 && ((int64_t)1 << kbits) <= nodes) kbits += 8;
+            uint32_t* skeys;
+            int32_t* svals;
+            radix_sort(lt_k0, lt_v0, lt_k1, lt_v1, pairs, kbits, lt_rs, s, &skeys, &svals);
+            la.list = svals;
+            note_launch();
+            lt_bounds_kernel<<<(unsigned)((nodes + 1 + 255) / 256), 256, 0, s>>>(la, skeys, pairs);
+            note_launch();
+            lt_tiles_kernel<<<(unsigned)((nodes + 255) / 256), 256, 0, s>>>(la);
+            scan_exclusive(la.ncnt, la.toff, nodes, scan_scr, s);
+            note_launch();
+            lt_tile_nodes_kernel<<<(unsigned)((nodes + 255) / 256), 256, 0, s>>>(la);
+            // tiles: at most one partial tile per node beyond the full ones
+            const int64_t max_tiles = (pairs + kLtPairs - 1) / kLtPairs + nodes;
+            note_launch();
+            switch (p.r) {
+                case 16: leaf_scores_kernel<16><<<(unsigned)max_tiles, kNsThreads, 0, s>>>(la); break;
+                case 32: leaf_scores_kernel<32><<<(unsigned)max_tiles, kNsThreads, 0, s>>>(la); break;
+                default: leaf_scores_kernel<64><<<(unsigned)max_tiles, kNsThreads, 0, s>>>(la); break;
+            }
+            st = cuda_status(cudaGetLastError());
+            if (st != LSA_OK) return st;
+            pre.b1 = la.b1;
+            pre.nb1 = la.nb1;
+            pre.S2 = la.S2;
+            pre.s2_ld = kLtCap;
+        }
         ScoredOut so{};
         if (scored) {
             so = *scored;
@@ -237,7 +725,7 @@ int launch_select_tree(const lsa_index* ix, const lsa_select_params* sp, const f
             so.block += q0 * hkv * scored->kb_cap;
             so.n += q0 * hkv;
         }
-        st = launch_select_rows(ix, sp, qbar + q0 * hkv * p.r, nq, nqc, q_pos ? q_pos + q0 : nullptr, q_pos0 + q0,
+        st = launch_select_rows(ix, sp, qb, nq, nqc, q_pos ? q_pos + q0 : nullptr, q_pos0 + q0,
                                 idx ? idx + q0 * hkv * max_sel : nullptr, cnt ? cnt + q0 * hkv : nullptr, max_sel,
                                 false, s, work, scored ? &so : nullptr, &pre);
         if (st != LSA_OK) return st;
@@ -251,3 +739,5 @@ extern "C" void lsa_debug_dense_config(int64_t min_pairs, int64_t chunk_bytes) {
     lsa::g_dense_min_pairs.store(min_pairs == 0 ? lsa::kDenseMinPairs : (min_pairs < 0 ? -1 : min_pairs));
     lsa::g_dense_chunk_bytes.store(chunk_bytes > 0 ? chunk_bytes : lsa::kDenseChunkBytes);
 }
+
+extern "C" void lsa_debug_leaf_tiles(int32_t on) { lsa::g_leaf_tiles.store(on ? 1 : 0); }

@@ -86,6 +86,14 @@ struct SelArgs {
     int64_t pre_nq, pre_ld;
     int pre_levels;
     int pre_off[LSA_MAX_LEVELS];
+    // leaf tiles (node_scores.cu): per row of the dense-score numbering the
+    // kept nodes of the last dense level [row][beam] and their count (-1: the
+    // row searches every level here), and their children's scores [row][s2_ld]
+    // in kept-node order
+    const int32_t* lt_b1;
+    const int32_t* lt_nb1;
+    const float* lt_s2;
+    int64_t lt_ld;
 };
 
 // THREADS = kSelThreads for large grids; small grids (decode: a few queries)
@@ -268,7 +276,32 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
     };
 
     if (!FULL) {
-        for (int l = 0; l < a.levels; ++l) {
+        int l_first = 0;
+        const float* s2 = nullptr;
+        if (a.lt_b1) {
+            const int64_t srow = (bseq * a.pre_nq + qi) * a.hkv + h;
+            const int n1 = a.lt_nb1[srow];
+            if (n1 >= 0) {
+                // the dense levels' kept nodes come from the leaf tiles, in the
+                // order of their children's score slots: the search starts at
+                // the leaf level and reads those scores
+                const int lb = a.pre_levels;   // the leaf level
+                const int32_t* co = a.ocoff[lb - 1] + (int64_t)u * a.n_l[lb - 1];
+                const int child_base = u * a.n_l[lb];
+                for (int e = threadIdx.x; e < n1; e += blockDim.x) {
+                    const int q = a.lt_b1[srow * a.beam + e];
+                    kk[e] = q;
+                    lo[e] = co[q] - child_base;
+                    pre[e] = co[q + 1] - co[q];
+                }
+                scan_pre(pre, n1);
+                if (threadIdx.x == 0) sh.nkept = n1;
+                __syncthreads();
+                l_first = lb;
+                s2 = a.lt_s2 + srow * a.lt_ld;
+            }
+        }
+        for (int l = l_first; l < a.levels; ++l) {
             const int nl = a.n_l[l];
             const float* cent = a.ocent[l] + (int64_t)u * nl * R;
             const int64_t* mp = a.omp[l] + (int64_t)u * nl;
@@ -277,7 +310,17 @@ __global__ __launch_bounds__(THREADS, THREADS == kSelThreads ? LSA_SELECT_MIN_BL
             const int total = (l == 0) ? nl : pre[nk];
             if (threadIdx.x == 0) sh.count = 0;
             __syncthreads();
-            if (l < a.pre_levels) {
+            if (s2 && l == l_first) {
+                // leaf scores from the leaf tiles: candidate t's score is in slot t
+                stream_topk(total, a.beam, std::true_type{},
+                            [&](int t, OwnerState* state, bool* el, int* id, int* p, float* y) {
+                                const int q = slot_of(t, nk, state);
+                                y[0] = __ldg(s2 + t);
+                                *id = __ldg(oid + q);
+                                *p = q;
+                                *el = __ldg(mp + q) <= bound;
+                            });
+            } else if (l < a.pre_levels) {
                 const float* ps = a.pre + ((bseq * a.pre_nq + qi) * a.hkv + h) * a.pre_ld + a.pre_off[l];
                 stream_topk(total, a.beam, std::true_type{},
                             [&](int t, OwnerState* state, bool* el, int* id, int* p, float* y) {
@@ -560,6 +603,10 @@ int launch_select_rows(const lsa_index* ix, const lsa_select_params* sp, const f
         a.pre_ld = pre->ld;
         a.pre_levels = pre->levels;
         for (int l = 0; l < pre->levels; ++l) a.pre_off[l] = pre->off[l];
+        a.lt_b1 = pre->b1;
+        a.lt_nb1 = pre->nb1;
+        a.lt_s2 = pre->S2;
+        a.lt_ld = pre->s2_ld;
     }
     if (scored) {
         a.pos_shift = scored->pos_shift;

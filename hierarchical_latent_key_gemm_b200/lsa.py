@@ -77,6 +77,7 @@ _SIGS = {
     "lsa_strerror": (C.c_char_p, [_i32]),
     "lsa_debug_fail_alloc_after": (None, [_i32]),
     "lsa_debug_dense_config": (None, [_i64, _i64]),
+    "lsa_debug_leaf_tiles": (None, [_i32]),
     "lsa_launch_count": (_i64, []),
     "lsa_select_blocks": (_i32, [_vp, C.POINTER(SelectParams), _vp, _i64, _vp, _i64, _i64, _vp, _vp, _vp, _i32,
                                  _vp]),
@@ -551,6 +552,11 @@ def lsa_debug_dense_config(min_pairs: int = 0, chunk_bytes: int = 0):
     selections off, 0 restores its default threshold; chunk_bytes bounds its
     score buffer (0: default)."""
     lib().lsa_debug_dense_config(int(min_pairs), int(chunk_bytes))
+
+
+def lsa_debug_leaf_tiles(on: bool = True):
+    """Test hook: turn the leaf tiles of large selections on or off."""
+    lib().lsa_debug_leaf_tiles(1 if on else 0)
 
 
 def exported_symbols_from_header(header_path: str) -> list:

@@ -157,8 +157,14 @@ int lsa_build_index_from_tree(const lsa_build_params* params, const void* K, con
  * lower id.  The row of idx lists, ascending, the sink [0, min(S, i+1)), the
  * tokens of the chosen blocks and the window [max(0, i-W+1), i]; cnt holds its
  * length and the rest of the row is -1.  max_sel must be at least
- * ceil(K/P)*P + S + W.  [p3 TL;DR: the query is compared with centroids first
- * and only a few buckets are searched; p1; p5 steps 2-3] */
+ * ceil(K/P)*P + S + W.  Calls of 4,096 or more (query, KV head) pairs score
+ * the dense upper levels (and, when the leaf level is the only one below
+ * them, the kept nodes' leaves) for tiles of queries first, with the same
+ * arithmetic, so the rows are the same bits; that takes stream-ordered
+ * scratch (pool memory) of at most 1 GiB, or 2 GiB with the leaf scores, per
+ * call, the queries running in chunks that fit.  [p3 TL;DR: the query is
+ * compared with centroids first and only a few buckets are searched; p1;
+ * p5 steps 2-3] */
 int lsa_select(const lsa_index* index, const lsa_select_params* params, const void* Q,
                int64_t nq, const int64_t* q_pos, int64_t q_pos0,
                int32_t* idx, int32_t* cnt, int32_t max_sel, void* stream);
@@ -449,6 +455,14 @@ void lsa_debug_fail_alloc_after(int32_t n);
  * chunk_bytes > 0 bounds the score buffer (queries run in chunks that fit),
  * 0 restores the default of 1 GiB. */
 void lsa_debug_dense_config(int64_t min_pairs, int64_t chunk_bytes);
+
+/* Test hook for the leaf tiles of large selections (when the leaf level is the
+ * only level below the dense ones: the kept nodes of the last dense level and
+ * the kept leaves are chosen for all queries by exact warp-wide selections,
+ * and the leaves' scores computed per node for many queries at a time; the
+ * selection is bit-identical either way): on = 0 turns them off, 1 on (the
+ * default). */
+void lsa_debug_leaf_tiles(int32_t on);
 
 /* Number of kernels the library has launched in this process (a host-side
  * counter, incremented at every launch; for accounting in benchmarks). */

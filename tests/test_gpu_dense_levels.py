@@ -8,7 +8,11 @@ per-query search scoring every node itself (the scores are the same fp32
 values), with one buffer of scores and with the buffer forced small so that
 the queries run in several chunks.  The per-query search is the path the
 other parity tests check against the oracle; this pins the dense form to it
-on every tree shape the workloads use.
+on every tree shape the workloads use.  When the leaf level is the only
+level below the dense ones, the kept nodes and the kept leaves are chosen by
+warp-wide exact selections for all queries and the leaves scored per node
+(leaf tiles); the selection must be the same bits with them on and off,
+ties included (the integer workload in a three-level tree).
 
 Full scan: calls of 64 or more (query, KV head) pairs filter on the tensor
 cores and rank the survivors exactly (a few query tiles split the block range
@@ -35,15 +39,26 @@ def _cuda():
     torch.cuda.synchronize()
 
 
-def _three_ways(ix, sp, Q, **kw):
+def _ways(ix, sp, Q, **kw):
+    """per-query search; dense levels + leaf tiles; the same in small chunks;
+    dense levels without leaf tiles"""
     out = []
     try:
-        for min_pairs, chunk in ((-1, 0), (1, 0), (1, 1 << 20)):
+        for min_pairs, chunk, tiles in ((-1, 0, 1), (1, 0, 1), (1, 1 << 20, 1), (1, 0, 0)):
             lsa.lsa_debug_dense_config(min_pairs, chunk)
+            lsa.lsa_debug_leaf_tiles(tiles)
             out.append(lsa.lsa_select(ix, sp, Q, **kw))
     finally:
         lsa.lsa_debug_dense_config(0, 0)
+        lsa.lsa_debug_leaf_tiles(1)
     return out
+
+
+def _same(outs):
+    (i0, c0) = outs[0]
+    for k, (i, c) in enumerate(outs[1:], 1):
+        assert torch.equal(c0, c), f"counts differ (way {k})"
+        assert torch.equal(i0, i), f"rows differ (way {k})"
 
 
 @pytest.mark.parametrize("name,over,beam", [
@@ -52,17 +67,19 @@ def _three_ways(ix, sp, Q, **kw):
     ("gqa_128k", dict(n_tokens=16384 + 5, needles=0, components=512), None),   # 32 x 1024, beam 32, 4 KV heads
     ("gqa_128k", dict(n_tokens=16384 + 5, needles=0, components=512), 31),     # beam below the top level: one level
     ("prefill_1m", dict(n_tokens=65536 + 7, level_sizes=(16, 128, 1024), needles=0, components=1024,
-                        drift_every=1 << 14), None),                    # three levels, the leaves per query
+                        drift_every=1 << 14), None),                    # three levels, leaf tiles
+    ("prefill_1m", dict(n_tokens=32768 + 3, level_sizes=(16, 512, 4096), needles=0, components=1024,
+                        drift_every=1 << 13), None),                    # the bench's upper levels, leaf tiles
+    ("int_exact_16k", dict(level_sizes=(4, 16, 256)), 4),               # integer scores: ties at every level
 ])
 def test_dense_levels_match_the_per_query_search(name, over, beam):
     w = WORKLOADS[name].scaled(**over)
     inp = make_inputs(w, seed=31, device="cuda")
     ix = lsa.lsa_build_index(TU.build_params(w), inp["K"], inp["W"])
     sp = TU.select_params(w, beam=beam)
-    (i0, c0), (i1, c1), (i2, c2) = _three_ways(ix, sp, inp["Q"])
+    outs = _ways(ix, sp, inp["Q"])
     assert lsa.lsa_check(ix) == lsa.LSA_OK
-    assert torch.equal(c0, c1) and torch.equal(i0, i1)
-    assert torch.equal(c0, c2) and torch.equal(i0, i2)
+    _same(outs)
     ix.free()
 
 
@@ -78,23 +95,31 @@ def test_dense_levels_batch_and_given_positions():
     g = torch.Generator().manual_seed(5)
     pos = torch.randint(0, w.n_tokens, (w.batch, nq), generator=g).to(torch.int64).cuda()
     Q = inp["Q"][:, :nq].contiguous()
-    (i0, c0), (i1, c1), (i2, c2) = _three_ways(ix, sp, Q, q_pos=pos)
+    outs = _ways(ix, sp, Q, q_pos=pos)
     assert lsa.lsa_check(ix) == lsa.LSA_OK
-    assert torch.equal(c0, c1) and torch.equal(i0, i1)
-    assert torch.equal(c0, c2) and torch.equal(i0, i2)
+    _same(outs)
+    # three levels with a sparse leaf level (leaf tiles) over several sequences
+    w2 = w.scaled(level_sizes=(8, 32, 256))
+    ix2 = lsa.lsa_build_index(TU.build_params(w2), inp["K"], inp["W"])
+    outs = _ways(ix2, TU.select_params(w2, beam=16), Q, q_pos=pos)
+    assert lsa.lsa_check(ix2) == lsa.LSA_OK
+    _same(outs)
     ix.free()
+    ix2.free()
 
 
 def test_dense_levels_scored_blocks():
-    """The scored-blocks form (context-parallel shards) through the dense path."""
-    w = WORKLOADS["gqa_128k"].scaled(n_tokens=8192 + 1, needles=0, components=256)
+    """The scored-blocks form (context-parallel shards) through the dense path
+    and the leaf tiles (three levels, the leaf level sparse)."""
+    w = WORKLOADS["gqa_128k"].scaled(n_tokens=8192 + 1, level_sizes=(8, 64, 512), needles=0, components=256)
     inp = make_inputs(w, seed=33, device="cuda")
     ix = lsa.lsa_build_index(TU.build_params(w), inp["K"], inp["W"])
     sp = TU.select_params(w)
     outs = []
     try:
-        for min_pairs, chunk in ((-1, 0), (1, 0), (1, 1 << 18)):
+        for min_pairs, chunk, tiles in ((-1, 0, 1), (1, 0, 1), (1, 1 << 18, 1), (1, 0, 0)):
             lsa.lsa_debug_dense_config(min_pairs, chunk)
+            lsa.lsa_debug_leaf_tiles(tiles)
             sc, bl, ct = lsa.lsa_select_blocks(ix, sp, inp["Q"], 0)
             # the kept blocks come in no particular order: sort each row by block id
             key = torch.where(bl >= 0, bl, torch.full_like(bl, 2 ** 31 - 1))
@@ -102,6 +127,7 @@ def test_dense_levels_scored_blocks():
             outs.append((torch.gather(sc, -1, order), key, ct))
     finally:
         lsa.lsa_debug_dense_config(0, 0)
+        lsa.lsa_debug_leaf_tiles(1)
     assert lsa.lsa_check(ix) == lsa.LSA_OK
     for o in outs[1:]:
         for a, b in zip(outs[0], o):
