@@ -285,7 +285,8 @@ def run_ours(args):
     stages = stage_rooflines(w, inp, bp, dev, peaks, build_ms, select_ms, attn_ms, nodes, blocks, sel_tokens,
                              q0, nq)
     sel = stages["select"]
-    roofline = {"bound": "hbm", "kernel": "select_kernel<64, tree> (select stage: query latents + select)",
+    roofline = {"bound": "hbm", "kernel": ("select_kernel<64, tree> (select stage: query latents, dense-level scores, "
+                                           "leaf tiles, select)"),
                 "achieved": sel["achieved_GBps"], "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": sel["frac"],
                 "traffic": recorded_traffic("select_kernel<64, tree>", w.name, "select.cu+select_common.cuh"),
                 "algorithmic_bytes_per_launch": sel["algorithmic_bytes"], "peak_source": peaks["source"],
