@@ -461,7 +461,7 @@ __device__ __forceinline__ void lt_tree(const float* qs, const float* cs, int tq
 // and the node's children (32 at a time) transposed into shared memory, the
 // 128 x 32 scores in the per-query kernel's order, each into its row's slot.
 template <int R>
-__global__ __launch_bounds__(kNsThreads) void leaf_scores_kernel(const LtArgs a) {
+__global__ __launch_bounds__(kNsThreads, 3) void leaf_scores_kernel(const LtArgs a) {
     constexpr int PQ = kLtPairs + 4, PC = kLtKids + 4;
     __shared__ __align__(16) float qs[R * PQ];
     __shared__ __align__(16) float cs[R * PC];
