@@ -1,4 +1,5 @@
-// Scores of the dense upper tree levels for a tile of queries at a time.
+// Scores of the dense upper tree levels for a tile of queries at a time, and
+// (leaf tiles, below) of the leaves of each query's kept nodes.
 //
 // The tree search (tree-search wiki note, TL;DR; LSA explainer, "How does LSA
 // work?" step 2) keeps, level by level, the best `beam` of the eligible nodes.
@@ -155,10 +156,11 @@ __global__ __launch_bounds__(kNsThreads) void node_scores_kernel(const NsArgs a)
 //      the last dense level, i.e. the best `beam` of all its eligible nodes by
 //      (score desc, id asc), from the dense scores; and for each kept node the
 //      first slot of its children in the row's leaf-score buffer;
-//   2. the (row, kept node) pairs grouped by node (counting sort);
-//   3. leaf_scores_kernel: per node, 64 of its pairs x 64 of its children at a
-//      time, the register-tiled fp32 product in the per-query kernel's order,
-//      each score written to its row's slot;
+//   2. the (row, kept node) pairs grouped by node (the library's radix sort
+//      on the node), every node's first pair and its tiles of 128 pairs;
+//   3. leaf_scores_kernel: per tile, its 128 pairs x 32 of the node's children
+//      at a time, the register-tiled fp32 product in the per-query kernel's
+//      order, each score written to its row's slot;
 //   4. the per-query kernel starts from those kept nodes and reads each leaf
 //      candidate's score from its slot (one lane per candidate) instead of
 //      scoring its row.
