@@ -30,6 +30,25 @@ constexpr int kNsTq = 64;   // queries per CTA tile
 constexpr int kNsTn = 64;   // nodes per pass
 constexpr int kNsPad = 4;   // shared row padding (keeps 16-byte alignment)
 
+// Rows 0 .. N-1 of R floats each, row i's float4 d4 given by src(i, d4), into
+// shared memory transposed: dst[d * P + i].  Two neighbouring lanes take the
+// two float4 of one 32-byte sector of a row and a warp takes 16 rows, so a
+// warp's loads use whole sectors and, with P = 4 (mod 32), each of its four
+// stores hits 32 distinct banks (16 * d4 + i covers them all).
+template <int N, int R, int P, class Src>
+__device__ __forceinline__ void stage_transposed(float* dst, int tid, Src&& src) {
+    static_assert(N % 16 == 0 && (R / 4) % 2 == 0 && P % 32 == 4, "conflict-free layout");
+    for (int e = tid; e < N * (R / 4); e += kNsThreads) {
+        const int p = e >> 1;
+        const int i = p % N, d4 = 2 * (p / N) + (e & 1);
+        const float4 v = src(i, d4);
+        dst[(4 * d4 + 0) * P + i] = v.x;
+        dst[(4 * d4 + 1) * P + i] = v.y;
+        dst[(4 * d4 + 2) * P + i] = v.z;
+        dst[(4 * d4 + 3) * P + i] = v.w;
+    }
+}
+
 struct NsArgs {
     const float* qbar;       // rows (bseq * nq_stride + qi) * hkv + h, qi in [0, nqc)
     int64_t nq_stride, nqc;
@@ -96,21 +115,14 @@ __global__ __launch_bounds__(kNsThreads) void node_scores_kernel(const NsArgs a)
     const int nqt = (int)min((int64_t)kNsTq, a.nqc - q0);
 
     // query tile, transposed: qs[d][i] (rows past the end are zero)
-    for (int e = tid; e < kNsTq * (R / 4); e += kNsThreads) {
-        const int i = e / (R / 4), d4 = e % (R / 4);
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (i < nqt)
-            v = *reinterpret_cast<const float4*>(a.qbar + ((bseq * a.nq_stride + q0 + i) * a.hkv + h) * R + 4 * d4);
-        qs[(4 * d4 + 0) * (kNsTq + kNsPad) + i] = v.x;
-        qs[(4 * d4 + 1) * (kNsTq + kNsPad) + i] = v.y;
-        qs[(4 * d4 + 2) * (kNsTq + kNsPad) + i] = v.z;
-        qs[(4 * d4 + 3) * (kNsTq + kNsPad) + i] = v.w;
-    }
+    stage_transposed<kNsTq, R, kNsTq + kNsPad>(qs, tid, [&](int i, int d4) {
+        if (i >= nqt) return make_float4(0.f, 0.f, 0.f, 0.f);
+        return *reinterpret_cast<const float4*>(a.qbar + ((bseq * a.nq_stride + q0 + i) * a.hkv + h) * R + 4 * d4);
+    });
     const int ncols = a.ncols;
     for (int c0 = 0; c0 < ncols; c0 += kNsTn) {
         __syncthreads();   // the previous pass is done with cs (and qs is written)
-        for (int e = tid; e < kNsTn * (R / 4); e += kNsThreads) {
-            const int j = e / (R / 4), d4 = e % (R / 4);
+        stage_transposed<kNsTn, R, kNsTn + kNsPad>(cs, tid, [&](int j, int d4) {
             const int col = c0 + j;
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
             if (col < ncols) {
@@ -127,11 +139,8 @@ __global__ __launch_bounds__(kNsThreads) void node_scores_kernel(const NsArgs a)
                 }
                 v = *reinterpret_cast<const float4*>(base + ((int64_t)u * nl + (col - off)) * R + 4 * d4);
             }
-            cs[(4 * d4 + 0) * (kNsTn + kNsPad) + j] = v.x;
-            cs[(4 * d4 + 1) * (kNsTn + kNsPad) + j] = v.y;
-            cs[(4 * d4 + 2) * (kNsTn + kNsPad) + j] = v.z;
-            cs[(4 * d4 + 3) * (kNsTn + kNsPad) + j] = v.w;
-        }
+            return v;
+        });
         __syncthreads();
         float sc[16];
         tree<R, 0, 1>(qs, cs, tq, tn, sc);
@@ -490,33 +499,21 @@ __global__ __launch_bounds__(kNsThreads, 3) void leaf_scores_kernel(const LtArgs
     }
     __syncthreads();
     // the pairs' latent queries, transposed (pairs past np are zero)
-    for (int e = tid; e < kLtPairs * (R / 4); e += kNsThreads) {
-        const int i = e / (R / 4), d4 = e % (R / 4);
-        float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (i < np) {
-            const int64_t r = prow[i];
-            const int h = (int)(r % a.hkv);
-            const int64_t bq = r / a.hkv;
-            const int64_t qrow = ((bq / a.nqc) * a.nq_stride + bq % a.nqc) * a.hkv + h;
-            v = *reinterpret_cast<const float4*>(a.qbar + qrow * R + 4 * d4);
-        }
-        qs[(4 * d4 + 0) * PQ + i] = v.x;
-        qs[(4 * d4 + 1) * PQ + i] = v.y;
-        qs[(4 * d4 + 2) * PQ + i] = v.z;
-        qs[(4 * d4 + 3) * PQ + i] = v.w;
-    }
+    stage_transposed<kLtPairs, R, PQ>(qs, tid, [&](int i, int d4) {
+        if (i >= np) return make_float4(0.f, 0.f, 0.f, 0.f);
+        const int64_t r = prow[i];
+        const int h = (int)(r % a.hkv);
+        const int64_t bq = r / a.hkv;
+        const int64_t qrow = ((bq / a.nqc) * a.nq_stride + bq % a.nqc) * a.hkv + h;
+        return *reinterpret_cast<const float4*>(a.qbar + qrow * R + 4 * d4);
+    });
     const int c_beg = a.coff1[g], nc = a.coff1[g + 1] - c_beg;   // global leaf positions
     for (int c0 = 0; c0 < nc; c0 += kLtKids) {
         __syncthreads();   // qs written; the previous pass is done with cs
-        for (int e = tid; e < kLtKids * (R / 4); e += kNsThreads) {
-            const int j = e / (R / 4), d4 = e % (R / 4);
-            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (c0 + j < nc) v = *reinterpret_cast<const float4*>(a.cent2 + ((int64_t)c_beg + c0 + j) * R + 4 * d4);
-            cs[(4 * d4 + 0) * PC + j] = v.x;
-            cs[(4 * d4 + 1) * PC + j] = v.y;
-            cs[(4 * d4 + 2) * PC + j] = v.z;
-            cs[(4 * d4 + 3) * PC + j] = v.w;
-        }
+        stage_transposed<kLtKids, R, PC>(cs, tid, [&](int j, int d4) {
+            if (c0 + j >= nc) return make_float4(0.f, 0.f, 0.f, 0.f);
+            return *reinterpret_cast<const float4*>(a.cent2 + ((int64_t)c_beg + c0 + j) * R + 4 * d4);
+        });
         __syncthreads();
         if (4 * tq < np) {
             float sc[16];

@@ -83,6 +83,25 @@ def test_dense_levels_match_the_per_query_search(name, over, beam):
     ix.free()
 
 
+def test_leaf_tiles_rows_that_fall_back():
+    """Kept nodes with about 3,072 leaves between them: some rows exceed the
+    leaf-score slots of the leaf tiles and search every level themselves,
+    the others use the tiles; every row must equal the per-query search."""
+    w = WORKLOADS["gqa_128k"].scaled(n_tokens=32768 + 5, level_sizes=(4, 8, 6144), needles=0, components=512)
+    inp = make_inputs(w, seed=35, device="cuda")
+    ix = lsa.lsa_build_index(TU.build_params(w), inp["K"], inp["W"])
+    # children per level-1 node: the 4 largest hold more than the 3,072 slots,
+    # the 4 smallest fewer, so both kinds of rows can occur
+    par = ix.get(lsa.LSA_GET_PARENT, 2).long().cpu()
+    kids = torch.stack([torch.bincount(par[u], minlength=8) for u in range(par.shape[0])]).sort(dim=1).values
+    assert bool((kids[:, -4:].sum(1) > 3072).any()) and bool((kids[:, :4].sum(1) <= 3072).any()), kids
+    sp = TU.select_params(w, beam=4)
+    outs = _ways(ix, sp, inp["Q"])
+    assert lsa.lsa_check(ix) == lsa.LSA_OK
+    _same(outs)
+    ix.free()
+
+
 def test_dense_levels_batch_and_given_positions():
     """Several sequences (row index (b * nq + qi) * hkv + h in the score
     buffer) and query positions given per query."""
