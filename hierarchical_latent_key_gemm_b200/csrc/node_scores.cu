@@ -321,7 +321,12 @@ __device__ __forceinline__ void lt_row(const LtArgs& a, int64_t row, int64_t* u,
     *bound = pos - a.window - a.pool + 1;
 }
 
-__global__ __launch_bounds__(kLtWarps * 32) void beam_dense_kernel(const LtArgs a) {
+// the row's eligible level-1 scores as order-preserving keys (0: not
+// eligible), kept in registers (KPL per lane, node t = 32 j + lane) when the
+// level has at most 32 KPL nodes, else in this warp's shared row (KPL = 0);
+// 32 keys a lane run at two CTAs per SM (128 registers), the others at four
+template <int KPL>
+__global__ __launch_bounds__(kLtWarps * 32, KPL == 32 ? 2 : 4) void beam_dense_kernel(const LtArgs a) {
     extern __shared__ uint32_t lt_smem[];
     __shared__ int hist_all[kLtWarps][256];
     const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
@@ -333,13 +338,14 @@ __global__ __launch_bounds__(kLtWarps * 32) void beam_dense_kernel(const LtArgs 
     const int64_t* mp = a.mp1 + u * a.n1;
     const int32_t* id = a.id1 + u * a.n1;
     int32_t* out = a.b1 + row * a.beam;
+    uint32_t kr[KPL > 0 ? KPL : 1];
     uint32_t* keyc = lt_smem + (size_t)w * a.n1;
-    for (int t0 = 0; t0 < a.n1; t0 += 128) {
-        int64_t mpv[4];
-        float sv[4];
+    if constexpr (KPL > 0) {
+        int64_t mpv[KPL];
+        float sv[KPL];
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int t = t0 + j * 32 + lane;
+        for (int j = 0; j < KPL; ++j) {
+            const int t = j * 32 + lane;
             mpv[j] = INT64_MAX;
             sv[j] = 0.f;
             if (t < a.n1) {
@@ -348,19 +354,44 @@ __global__ __launch_bounds__(kLtWarps * 32) void beam_dense_kernel(const LtArgs 
             }
         }
 #pragma unroll
-        for (int j = 0; j < 4; ++j) {
-            const int t = t0 + j * 32 + lane;
-            if (t < a.n1) keyc[t] = mpv[j] <= bound ? fkey(sv[j]) : 0u;
+        for (int j = 0; j < KPL; ++j) kr[j] = mpv[j] <= bound ? fkey(sv[j]) : 0u;
+    } else {
+        for (int t0 = 0; t0 < a.n1; t0 += 128) {
+            int64_t mpv[4];
+            float sv[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int t = t0 + j * 32 + lane;
+                mpv[j] = INT64_MAX;
+                sv[j] = 0.f;
+                if (t < a.n1) {
+                    mpv[j] = __ldg(mp + t);
+                    sv[j] = __ldg(sr + t);
+                }
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int t = t0 + j * 32 + lane;
+                if (t < a.n1) keyc[t] = mpv[j] <= bound ? fkey(sv[j]) : 0u;
+            }
         }
+        __syncwarp();
     }
-    __syncwarp();
+    // ids matter only for ties at the threshold and are read then
     auto each = [&](auto&& f) {
-        for (int t0 = 0; t0 < a.n1; t0 += 32) {
-            const int t = t0 + lane;
-            const bool valid = t < a.n1;
-            const uint32_t key = valid ? keyc[t] : 0u;
-            // ids matter only for ties at the threshold and are read then
-            f(valid, key, key != 0u ? __ldg(id + t) : 0, t);
+        if constexpr (KPL > 0) {
+#pragma unroll
+            for (int j = 0; j < KPL; ++j) {
+                const int t = j * 32 + lane;
+                f(t < a.n1, kr[j], kr[j] != 0u ? __ldg(id + t) : 0, t);
+            }
+        } else {
+            for (int t0 = 0; t0 < a.n1; t0 += 32) {
+                const int t = t0 + lane;
+                const bool valid = t < a.n1;
+                const uint32_t key = valid ? keyc[t] : 0u;
+                f(valid, key, key != 0u ? __ldg(id + t) : 0, t);
+            }
         }
     };
     const int n = warp_topk(a.beam, hist_all[w], each, [&](int slot, int t) { out[slot] = t; });
@@ -680,12 +711,19 @@ int launch_select_tree(const lsa_index* ix, const lsa_select_params* sp, const f
             la.qbar = qb;
             const int64_t nodes = ix->units * n1;
             const int64_t pairs = la.rows * beam;
-            const size_t dense_smem = (size_t)kLtWarps * n1 * sizeof(uint32_t);
-            cudaError_t e0 = cudaFuncSetAttribute(beam_dense_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                  (int)dense_smem);
-            if (e0 != cudaSuccess) return cuda_status(e0);
+            const unsigned bd_grid = (unsigned)((la.rows + kLtWarps - 1) / kLtWarps);
             note_launch();
-            beam_dense_kernel<<<(unsigned)((la.rows + kLtWarps - 1) / kLtWarps), kLtWarps * 32, dense_smem, s>>>(la);
+            if (n1 <= 16 * 32) {
+                beam_dense_kernel<16><<<bd_grid, kLtWarps * 32, 0, s>>>(la);
+            } else if (n1 <= 32 * 32) {
+                beam_dense_kernel<32><<<bd_grid, kLtWarps * 32, 0, s>>>(la);
+            } else {
+                const size_t dense_smem = (size_t)kLtWarps * n1 * sizeof(uint32_t);
+                cudaError_t e0 = cudaFuncSetAttribute(beam_dense_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                      (int)dense_smem);
+                if (e0 != cudaSuccess) return cuda_status(e0);
+                beam_dense_kernel<0><<<bd_grid, kLtWarps * 32, dense_smem, s>>>(la);
+            }
             // the pairs grouped by node: a stable radix sort on the node
             note_launch();
             lt_keys_kernel<<<(unsigned)((pairs + 255) / 256), 256, 0, s>>>(la, lt_k0, lt_v0);

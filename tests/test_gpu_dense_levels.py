@@ -71,6 +71,10 @@ def _same(outs):
     ("prefill_1m", dict(n_tokens=32768 + 3, level_sizes=(16, 512, 4096), needles=0, components=1024,
                         drift_every=1 << 13), None),                    # the bench's upper levels, leaf tiles
     ("int_exact_16k", dict(level_sizes=(4, 16, 256)), 4),               # integer scores: ties at every level
+    ("gqa_128k", dict(n_tokens=65536 + 5, level_sizes=(8, 1024, 8192), needles=0, components=512), None),
+                                                                        # 1,024 kept-node candidates: 32 keys a lane
+    ("gqa_128k", dict(n_tokens=65536 + 5, level_sizes=(8, 2048, 8192), needles=0, components=512), None),
+                                                                        # 2,048: keys in shared memory
 ])
 def test_dense_levels_match_the_per_query_search(name, over, beam):
     w = WORKLOADS[name].scaled(**over)
