@@ -644,7 +644,7 @@ def time_ms(fn, reps: int = 3) -> float:
 
 
 def stage_rooflines(w, inp, bp, dev, peaks, build_ms, select_ms, attn_ms, nodes, blocks, sel_tokens, q0, nq):
-    """Every stage against its roofline, on the survey's algorithmic work:
+    """Every stage against its roofline, on each stage's algorithmic work:
       a1 project + pool   HBM: K read (2 B per element) + latent keys written (r x 4 B per block)
       a5 query latent     HBM: Q read + latent queries written (r x 4 B per (query, KV head))
       a2 leaf k-means     tensor (bf16 dense peak): 2 x blocks x leaves x r flops per round
