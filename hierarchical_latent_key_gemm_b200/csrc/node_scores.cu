@@ -516,7 +516,11 @@ __global__ __launch_bounds__(kNsThreads, 3) void leaf_scores_kernel(const LtArgs
     const int64_t j0 = a.noff[g] + (t - a.toff[g]) * kLtPairs;
     const int np = (int)min((int64_t)kLtPairs, (int64_t)a.noff[g + 1] - j0);
     const int tid = threadIdx.x;
-    const int tn = tid % (kLtKids / 4), tq = tid / (kLtKids / 4);   // 8 x 32 threads: 4 children x 4 pairs each
+    // 8 x 32 threads, 4 children x 4 pairs each; a warp takes 16 children x
+    // 32 pairs, so in a pass over at most 16 children the warps of the upper
+    // half have nothing to score and skip it
+    const int wq = (tid >> 5) & 3, wc = tid >> 7;
+    const int tn = (tid & 3) + 4 * wc, tq = ((tid & 31) >> 2) + 8 * wq;
     if (tid < kLtPairs) {
         int64_t r = -1;
         int sl = 0;
@@ -546,7 +550,7 @@ __global__ __launch_bounds__(kNsThreads, 3) void leaf_scores_kernel(const LtArgs
             return *reinterpret_cast<const float4*>(a.cent2 + ((int64_t)c_beg + c0 + j) * R + 4 * d4);
         });
         __syncthreads();
-        if (4 * tq < np) {
+        if (4 * tq < np && 16 * wc < nc - c0) {
             float sc[16];
             lt_tree<R, PQ, PC, 0, 1>(qs, cs, tq, tn, sc);
 #pragma unroll
