@@ -85,6 +85,9 @@ _SIGS = {
                                    _vp, _vp, _i32, _vp]),
     "lsa_localize_rows": (_i32, [_vp, _vp, _i64, _i32, _i64, _i64, _vp, _vp, _vp]),
     "lsa_merge_attn": (_i32, [_i32, _vp, _vp, _i64, _i32, _i32, _i32, _vp, _vp, _vp]),
+    "lsa_prefill_create": (_i32, [C.POINTER(BuildParams), C.POINTER(SelectParams), _i64, _i32, _vp]),
+    "lsa_prefill_run": (_i32, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp]),
+    "lsa_prefill_free": (None, [_vp]),
 }
 
 _lib = None
@@ -533,6 +536,58 @@ def lsa_merge_attn(O_parts, lse_parts, O=None, lse=None, want_lse=True, stream=N
                              int(hq), int(d), dtype_code(O), _ptr(O), _typed(lse, torch.float32, "lse"),
                              _stream(stream)), "lsa_merge_attn")
     return O, lse
+
+
+def _host_ptr(t, dtype, shape, name):
+    """Pointer of a host tensor after checking its type and shape (the C call
+    cannot see either)."""
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise ValueError(f"{name} must be a host tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    _shape(t, shape, name)
+    return C.c_void_p(t.data_ptr())
+
+
+class Prefill:
+    """Owner of an lsa_prefill context: one prefill layer from host memory per
+    run, the host-device copies overlapped with the build, select and
+    attention (lsa_prefill_create / run / free)."""
+
+    def __init__(self, params: BuildParams, sp: SelectParams, nq: int, chunks: int = 16):
+        self.params, self.sp, self.nq = params, sp, int(nq)
+        self.handle = C.c_void_p()
+        _ok(lib().lsa_prefill_create(C.byref(params), C.byref(sp), self.nq, int(chunks), C.byref(self.handle)),
+            "lsa_prefill_create")
+
+    def run(self, hQ, hK, hV, hW, hO, hlse=None, stream=None) -> Index:
+        """Enqueue one layer after the work on `stream` (default: the current
+        stream), which then waits for it; returns the layer's index (free it
+        once the stream has passed the run)."""
+        p, sp, nq = self.params, self.sp, self.nq
+        dt = {LSA_F32: torch.float32, LSA_BF16: torch.bfloat16}[p.dtype]
+        kv = (1, p.ld_tokens, p.hkv, p.d)
+        args = (_host_ptr(hQ, dt, (1, nq, sp.hq, p.d), "hQ"), _host_ptr(hK, dt, kv, "hK"),
+                _host_ptr(hV, dt, kv, "hV"), _host_ptr(hW, torch.float32, (p.d, p.r), "hW"),
+                _host_ptr(hO, dt, (1, nq, sp.hq, p.d), "hO"), _host_ptr(hlse, torch.float32, (1, nq, sp.hq), "hlse"))
+        h = C.c_void_p()
+        _ok(lib().lsa_prefill_run(self.handle, *args, _stream(stream), C.byref(h)), "lsa_prefill_run")
+        return Index(h, p)
+
+    def free(self):
+        if self.handle:
+            lib().lsa_prefill_free(self.handle)
+            self.handle = C.c_void_p(None)
+
+    def __del__(self):
+        try:
+            self.free()
+        except Exception:
+            pass
 
 
 def lsa_check(index: Index | None = None, stream=None) -> int:

@@ -464,6 +464,46 @@ void lsa_debug_dense_config(int64_t min_pairs, int64_t chunk_bytes);
  * default). */
 void lsa_debug_leaf_tiles(int32_t on);
 
+/* One prefill layer from host memory: build the index of K, select for every
+ * query position 0 .. nq-1, and attend (banded form), with the host-device
+ * copies overlapped with the kernels.  [p5 "How does LSA work?" steps 1-3:
+ * the keys are bucketed, each query searches the buckets, attention covers
+ * the chosen keys, the sink and the window; p4 "Prompt processing is not
+ * response generation": prefill selects for every position at once]
+ * A context holds the device copies of Q, K, V, W, O and lse, the selection
+ * rows of one chunk, three streams and their events:
+ *  - lsa_prefill_create: params->batch must be 1; 1 <= nq <= n_tokens; the
+ *    queries are split into min(chunks, nq) chunks of consecutive positions
+ *    (chunks >= 1).  Allocates with cudaMalloc (synchronous).  On failure
+ *    *out is NULL and nothing is left allocated.
+ *  - lsa_prefill_run enqueues one layer after the work already on `stream`
+ *    and makes `stream` wait for all of it:
+ *      hK, hV: host [1][ld_tokens][hkv][d] of dtype (all ld_tokens rows are
+ *        copied); hW: host float [d][r]; hQ: host [1][nq][hq][d] of dtype;
+ *      hO: host [1][nq][hq][d] of dtype, written; hlse: host float [1][nq][hq]
+ *        or NULL (then the lse is not copied back).
+ *    K and W go up first and the index is built while V and then the queries
+ *    go up chunk by chunk; each chunk is selected and attended as soon as its
+ *    queries are up, and its output comes down while the next chunk
+ *    computes.  Results are those of lsa_build_index, lsa_select and
+ *    lsa_sparse_attn_banded called per chunk (q_pos0 = the chunk's first
+ *    position) with the same parameters.  Host buffers must stay valid until
+ *    `stream` passes the run; pinned (page-locked) memory lets the copies
+ *    overlap, pageable memory works but serialises them.  Runs on one
+ *    context are ordered among themselves whatever streams they are given.
+ *    On success *index_out receives the layer's index, owned by the caller
+ *    (lsa_free_index once `stream` has passed the run); on an error it is
+ *    NULL, the work already enqueued still completes before `stream` goes on,
+ *    and the context stays usable.  The current device must be the one the
+ *    context was created on.
+ *  - lsa_prefill_free synchronises the context's streams and frees it. */
+typedef struct lsa_prefill lsa_prefill;
+int lsa_prefill_create(const lsa_build_params* params, const lsa_select_params* sp, int64_t nq,
+                       int32_t chunks, lsa_prefill** out);
+int lsa_prefill_run(lsa_prefill* prefill, const void* hQ, const void* hK, const void* hV, const float* hW,
+                    void* hO, float* hlse, void* stream, lsa_index** index_out);
+void lsa_prefill_free(lsa_prefill* prefill);
+
 /* Number of kernels the library has launched in this process (a host-side
  * counter, incremented at every launch; for accounting in benchmarks). */
 int64_t lsa_launch_count(void);

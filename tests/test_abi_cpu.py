@@ -151,3 +151,49 @@ def test_binding_checks_shapes_before_the_call():
                                                         O=a["O"], lse=a["lse"])):
             with pytest.raises(ValueError, match=msg):
                 fn(a)
+
+
+def test_host_prefill_refuses_bad_arguments_before_any_cuda_call():
+    """lsa_prefill_create / run check their arguments on the host first
+    (batch 1, 1 <= nq <= n_tokens, chunks >= 1, hq a multiple of hkv, a valid
+    dtype, non-null buffers), and the binding checks the host tensors' types
+    and shapes before the call."""
+    import torch
+    L = lsa.lib()
+    bp = lsa.make_build_params(1, 64, 64, 2, 64, 16, 1, lsa.LSA_BF16, (2, 4), 1, 0, 0, 0)
+    sp = lsa.make_select_params(4, 2, 8, 0, 4)
+    out = C.c_void_p(0x1)
+    for over, nq, chunks in ((dict(batch=2), 64, 4), ({}, 0, 4), ({}, 65, 4), ({}, 64, 0),
+                             (dict(dtype=7), 64, 4), (dict(ld_tokens=32), 64, 4)):
+        b = lsa.BuildParams.from_buffer_copy(bp)
+        for k, v in over.items():
+            setattr(b, k, v)
+        assert L.lsa_prefill_create(C.byref(b), C.byref(sp), nq, chunks, C.byref(out)) == lsa.LSA_ERR_INVALID_ARG
+        assert not out.value
+        out = C.c_void_p(0x1)
+    sp3 = lsa.SelectParams.from_buffer_copy(sp)
+    sp3.hq = 3
+    assert L.lsa_prefill_create(C.byref(bp), C.byref(sp3), 64, 4, C.byref(out)) == lsa.LSA_ERR_INVALID_ARG
+    h = C.c_void_p()
+    assert L.lsa_prefill_run(None, None, None, None, None, None, None, None, C.byref(h)) == lsa.LSA_ERR_INVALID_ARG
+    assert not h.value
+    L.lsa_prefill_free(None)   # no-op
+    # the binding: host tensors of the right type and shape only
+    pf = lsa.Prefill.__new__(lsa.Prefill)
+    pf.params, pf.sp, pf.nq, pf.handle = bp, sp, 64, C.c_void_p(None)
+    bf = torch.bfloat16
+    ok = dict(hQ=torch.zeros(1, 64, 4, 64, dtype=bf), hK=torch.zeros(1, 64, 2, 64, dtype=bf),
+              hV=torch.zeros(1, 64, 2, 64, dtype=bf), hW=torch.zeros(64, 16), hO=torch.zeros(1, 64, 4, 64, dtype=bf))
+    cases = [
+        (dict(hQ=torch.zeros(1, 63, 4, 64, dtype=bf)), "hQ must have shape"),
+        (dict(hK=torch.zeros(1, 64, 2, 64)), "hK must be"),
+        (dict(hV=torch.zeros(1, 64, 1, 64, dtype=bf)), "hV must have shape"),
+        (dict(hW=torch.zeros(64, 32)), "hW must have shape"),
+        (dict(hO=torch.zeros(1, 64, 4, 64, dtype=bf)[:, ::2]), "hO must be contiguous"),
+        (dict(hlse=torch.zeros(1, 64, 2)), "hlse must have shape"),
+    ]
+    for over, msg in cases:
+        a = dict(ok, hlse=None)
+        a.update(over)
+        with pytest.raises(ValueError, match=msg):
+            pf.run(a["hQ"], a["hK"], a["hV"], a["hW"], a["hO"], hlse=a["hlse"], stream=0)

@@ -273,6 +273,39 @@ def test_host_prefill_pipeline_matches_device_path():
     ix.free()
 
 
+def test_host_prefill_c_entry_matches_the_stream_pipeline():
+    """lsa_prefill_run (one C-ABI call from host buffers: copies overlapped
+    with the build, select and banded attention in chunks) writes the same
+    bits as the same layer driven from Python on three streams with the same
+    chunks, on two runs of one context; its lse matches the device path's."""
+    from hierarchical_latent_key_gemm_b200.pipeline import HostPrefill
+    w = WORKLOADS["gqa_128k"].scaled(n_tokens=6000 + 7, level_sizes=(8, 64), needles=0, components=256)
+    inp = make_inputs(w, seed=15)
+    hQ, hK, hV, hW = (inp[k].pin_memory() for k in ("Q", "K", "V", "W"))
+    bp, sp = TU.build_params(w), TU.select_params(w)
+    hO_py = torch.empty(hQ.shape, dtype=hQ.dtype, pin_memory=True)
+    hp = HostPrefill(bp, sp, hQ, hK, hV, hW, hO_py, w.sink, w.window, chunks=5)
+    hp.run().free()
+    torch.cuda.synchronize()
+    pf = lsa.Prefill(bp, sp, w.n_tokens, chunks=5)
+    for _ in range(2):
+        hO = torch.full(hQ.shape, float("nan"), dtype=hQ.dtype).pin_memory()
+        hlse = torch.full((1, w.n_tokens, w.hq), float("nan")).pin_memory()
+        ix = pf.run(hQ, hK, hV, hW, hO, hlse=hlse)
+        torch.cuda.synchronize()
+        assert lsa.lsa_check(ix) == lsa.LSA_OK
+        ix.free()
+        assert torch.equal(hO.view(torch.int16), hO_py.view(torch.int16))
+    pf.free()
+    d = _dev(inp)
+    ix = lsa.lsa_build_index(bp, d["K"], d["W"])
+    idx, cnt = lsa.lsa_select(ix, sp, d["Q"])
+    _, lse = lsa.lsa_sparse_attn_banded(d["Q"], d["K"], d["V"], idx, cnt, w.hkv, w.sink, w.window)
+    ix.free()
+    ref = lse.cpu()
+    assert bool(((hlse - ref).abs() <= 1e-3 * ref.abs() + 1e-3).all())
+
+
 def test_select_and_banded_attention_capture_in_a_cuda_graph():
     """Selection runs on the device and every call is stream-ordered (scratch
     from the stream-ordered pool), so select + banded attention of a prefill
